@@ -1,0 +1,127 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by ``__graft_entry__.smoke()`` and
+by the CPU-baseline leg of ``bench.py``; never by the product package.  It
+shares no code with the CUDA library.
+
+Every function takes numpy arrays in the library's layout -- Q/O/dO
+``[B, Nq, Hq, d]``, K/V ``[B, Nk, Hkv, d]``, LSE ``[B, Hq, Nq]`` -- converts
+them to fp64 and calls the plain C implementation in ``attn_oracle.c``
+(row-by-row definition, two-pass softmax; see that file's header for the
+passages each step follows and the readings taken where the pages are silent).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        i = ctypes.c_int
+        lib.oracle_attn_fwd.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i,
+                                        ctypes.c_double, i, i, i, i]
+        lib.oracle_attn_fwd_blockwise.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i,
+                                                  ctypes.c_double, i, i, i, i, i]
+        lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i,
+                                        ctypes.c_double, i, i, i, i]
+        for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_blockwise, lib.oracle_attn_bwd):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except AttributeError:  # pragma: no cover
+        return max(1, os.cpu_count() or 1)
+
+
+def _f64(x):
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _dims(q, k, v):
+    if q.ndim != 4 or k.ndim != 4 or v.ndim != 4:
+        raise ValueError("expected 4-D [B, N, H, d] arrays")
+    B, Nq, Hq, d = q.shape
+    Bk, Nk, Hkv, dk = k.shape
+    if v.shape != k.shape or Bk != B or dk != d:
+        raise ValueError("shape mismatch between q, k and v")
+    return B, Nq, Nk, Hq, Hkv, d
+
+
+def _window(causal, window):
+    wl, wr = window if window is not None else (-1, -1)
+    return int(bool(causal)), int(wl), int(wr)
+
+
+def attn_fwd(q, k, v, scale=None, causal=False, window=(-1, -1), nthreads=None):
+    """Return (O [B,Nq,Hq,d], LSE [B,Hq,Nq]) in fp64 by the two-pass definition."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    o = np.empty((B, Nq, Hq, d), np.float64)
+    lse = np.empty((B, Hq, Nq), np.float64)
+    rc = _load().oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                 B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr,
+                                 nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("oracle_attn_fwd failed (%d)" % rc)
+    return o, lse
+
+
+def attn_fwd_blockwise(q, k, v, block_n, scale=None, causal=False, window=(-1, -1),
+                       nthreads=None):
+    """Return (O, LSE) by the online-softmax recurrence over key blocks of block_n."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    o = np.empty((B, Nq, Hq, d), np.float64)
+    lse = np.empty((B, Hq, Nq), np.float64)
+    rc = _load().oracle_attn_fwd_blockwise(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                           B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr,
+                                           int(block_n), nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("oracle_attn_fwd_blockwise failed (%d)" % rc)
+    return o, lse
+
+
+def attn_bwd(q, k, v, dout, scale=None, causal=False, window=(-1, -1), nthreads=None):
+    """Return (dQ, dK, dV) in fp64: gradients of sum(dout * O) by the explicit formulas."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    if dout.shape != q.shape:
+        raise ValueError("dout must have q's shape")
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    rc = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq),
+                                 _ptr(dk), _ptr(dv), B, Nq, Nk, Hq, Hkv, d, scale,
+                                 c, wl, wr, nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("oracle_attn_bwd failed (%d)" % rc)
+    return dq, dk, dv
+
+
+def fwd_flops(B, Nq, Nk, Hq, d, causal):
+    """Forward FLOP count of the metric: 4*B*Hq*Nq*Nk*d, halved when causal."""
+    f = 4.0 * B * Hq * Nq * Nk * d
+    return f / 2 if causal else f

@@ -1,0 +1,290 @@
+"""Pins for the fp64 oracle: things the pages and the mathematics fix, checked
+against the oracle so that it is not trusted on its own word.
+
+Each test names the fact it uses.  Together they are chosen so that a plausible
+slip in the oracle (a dropped rescale, a wrong sign, a transposed operand, the
+wrong GQA head, an off-by-one in the mask, a misplaced scale) fails at least
+one of them.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def _eval(x):
+    return eval(str(x), {"__builtins__": {}}, {"log": math.log, "inf": math.inf})
+
+
+def _arr(nested):
+    return np.vectorize(_eval, otypes=[np.float64])(np.array(nested, dtype=object))
+
+
+def _rand(shape, rng):
+    return rng.standard_normal(shape)
+
+
+def n_visible(i, Nq, Nk, causal, wl, wr):
+    """Count of visible keys for query i under the stated reading (inclusive
+    window bounds, bottom-right alignment, negative = unbounded)."""
+    delta = Nk - Nq
+    wr = 0 if causal else wr
+    lo = 0 if wl < 0 else max(0, i + delta - wl)
+    hi = Nk - 1 if wr < 0 else min(Nk - 1, i + delta + wr)
+    return max(0, hi - lo + 1), lo, hi
+
+
+# ---------------------------------------------------------------- golden cases
+
+with open(os.path.join(HERE, "golden", "closed_form_cases.json")) as f:
+    GOLDEN = json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", GOLDEN, ids=[c["name"] for c in GOLDEN])
+def test_golden_closed_form(case):
+    """Hand-derived exact values (tests/golden/closed_form_cases.json)."""
+    q, k, v = _arr(case["q"]), _arr(case["k"]), _arr(case["v"])
+    scale = _eval(case["scale"])
+    wl, wr = case["window"]
+    o, lse = oracle.attn_fwd(q, k, v, scale=scale, causal=case["causal"], window=(wl, wr),
+                             nthreads=2)
+    np.testing.assert_allclose(o, _arr(case["o"]), rtol=1e-13, atol=1e-13)
+    exp_lse = _arr(case["lse"])
+    assert np.array_equal(np.isinf(lse), np.isinf(exp_lse))
+    fin = np.isfinite(exp_lse)
+    np.testing.assert_allclose(lse[fin], exp_lse[fin], rtol=1e-13, atol=1e-13)
+    if "dq" in case:
+        dq, dk, dv = oracle.attn_bwd(q, k, v, _arr(case["do"]), scale=scale,
+                                     causal=case["causal"], window=(wl, wr), nthreads=1)
+        np.testing.assert_allclose(dq, _arr(case["dq"]), rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(dk, _arr(case["dk"]), rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(dv, _arr(case["dv"]), rtol=1e-13, atol=1e-13)
+
+
+# ------------------------------------------------------------ closed forms
+
+MASKS = [(False, -1, -1), (True, -1, -1), (True, 5, -1), (False, 3, 2), (False, -1, 4)]
+
+
+@pytest.mark.parametrize("causal,wl,wr", MASKS)
+@pytest.mark.parametrize("Nq,Nk", [(9, 9), (5, 12), (12, 5)])
+def test_identical_keys_give_mean_of_visible_values(causal, wl, wr, Nq, Nk):
+    """All keys equal -> P uniform over the visible keys: O_i is the mean of the
+    visible V rows and LSE_i = s_i + ln(n_visible_i).  Also pins the exact mask
+    reading through n_visible."""
+    rng = np.random.default_rng(1)
+    d, Hq, Hkv = 4, 4, 2
+    q = _rand((1, Nq, Hq, d), rng)
+    kvec = _rand((d,), rng)
+    k = np.broadcast_to(kvec, (1, Nk, Hkv, d)).copy()
+    v = _rand((1, Nk, Hkv, d), rng)
+    scale = 0.7
+    o, lse = oracle.attn_fwd(q, k, v, scale=scale, causal=causal, window=(wl, wr), nthreads=3)
+    for h in range(Hq):
+        hk = h // (Hq // Hkv)
+        for i in range(Nq):
+            n, lo, hi = n_visible(i, Nq, Nk, causal, wl, wr)
+            if n == 0:
+                assert np.all(o[0, i, h] == 0) and lse[0, h, i] == -np.inf
+                continue
+            np.testing.assert_allclose(o[0, i, h], v[0, lo:hi + 1, hk].mean(axis=0),
+                                       rtol=1e-12, atol=1e-12)
+            s = scale * q[0, i, h] @ kvec
+            assert abs(lse[0, h, i] - (s + math.log(n))) < 1e-12
+
+
+def test_dominant_score_selects_its_value_row():
+    """One key's scaled score exceeds all others by Delta ->
+    |O_i - V_j*| <= (n-1) e^-Delta max|V| (per element)."""
+    rng = np.random.default_rng(2)
+    Nk, d = 16, 8
+    q = np.zeros((1, 1, 1, d)); q[0, 0, 0, 0] = 1.0
+    k = 0.1 * _rand((1, Nk, 1, d), rng)
+    k[0, :, 0, 0] = rng.uniform(-1, 1, Nk)
+    jstar = 11
+    delta = 12.0
+    k[0, jstar, 0, 0] = k[0, :, 0, 0].max() + delta
+    v = _rand((1, Nk, 1, d), rng)
+    o, _ = oracle.attn_fwd(q, k, v, scale=1.0, nthreads=1)
+    bound = (Nk - 1) * math.exp(-delta) * np.abs(v).max()
+    assert np.abs(o[0, 0, 0] - v[0, jstar, 0]).max() <= bound
+
+
+def test_causal_row_zero_is_v0():
+    """Causal, Nq == Nk: row 0 sees only key 0, so O_0 = V_0 and LSE_0 = S_00."""
+    rng = np.random.default_rng(3)
+    q, k, v = (_rand((2, 7, 3, 5), rng) for _ in range(3))
+    o, lse = oracle.attn_fwd(q, k, v, scale=0.3, causal=True, nthreads=2)
+    np.testing.assert_array_equal(o[:, 0], v[:, 0])
+    np.testing.assert_allclose(lse[:, :, 0], 0.3 * np.einsum("bhc,bhc->bh", q[:, 0], k[:, 0]),
+                               rtol=1e-14, atol=1e-14)
+
+
+def test_two_keys_reduce_to_logistic():
+    """With two visible keys softmax is the logistic function:
+    O = v0 + (v1 - v0) * sigmoid(s1 - s0), LSE = s0 + log1p(exp(s1 - s0))."""
+    rng = np.random.default_rng(4)
+    q = _rand((1, 6, 2, 3), rng)
+    k = _rand((1, 2, 2, 3), rng)
+    v = _rand((1, 2, 2, 3), rng)
+    o, lse = oracle.attn_fwd(q, k, v, scale=1.3, nthreads=1)
+    for h in range(2):
+        s0 = 1.3 * q[0, :, h] @ k[0, 0, h]
+        s1 = 1.3 * q[0, :, h] @ k[0, 1, h]
+        sig = 1.0 / (1.0 + np.exp(-(s1 - s0)))
+        exp_o = v[0, 0, h] + (v[0, 1, h] - v[0, 0, h]) * sig[:, None]
+        np.testing.assert_allclose(o[0, :, h], exp_o, rtol=1e-13, atol=1e-13)
+        np.testing.assert_allclose(lse[0, h], s0 + np.log1p(np.exp(s1 - s0)), rtol=1e-13)
+
+
+# -------------------------------------------------- recurrence == definition
+
+@pytest.mark.parametrize("block", [1, 3, 16, 40])
+@pytest.mark.parametrize("causal,wl,wr", MASKS)
+def test_online_recurrence_equals_two_pass(block, causal, wl, wr):
+    """The blockwise online softmax (running max/sum and O rescaled by
+    exp(m_old - m_new)) equals the two-pass softmax to rounding."""
+    rng = np.random.default_rng(5)
+    q = 3.0 * _rand((1, 23, 4, 8), rng)   # peaked rows exercise the rescale
+    k = _rand((1, 40, 2, 8), rng)
+    v = _rand((1, 40, 2, 8), rng)
+    o1, l1 = oracle.attn_fwd(q, k, v, scale=0.5, causal=causal, window=(wl, wr), nthreads=2)
+    o2, l2 = oracle.attn_fwd_blockwise(q, k, v, block, scale=0.5, causal=causal,
+                                       window=(wl, wr), nthreads=2)
+    np.testing.assert_allclose(o2, o1, rtol=1e-13, atol=1e-13)
+    assert np.array_equal(np.isinf(l1), np.isinf(l2))
+    fin = np.isfinite(l1)
+    np.testing.assert_allclose(l2[fin], l1[fin], rtol=1e-13, atol=1e-13)
+
+
+# ------------------------------------------------------- finite differences
+
+def _loss(q, k, v, do, **kw):
+    o, _ = oracle.attn_fwd(q, k, v, nthreads=1, **kw)
+    return float(np.sum(do * o))
+
+
+@pytest.mark.parametrize("shape,causal,wl,wr", [
+    ((1, 6, 2, 2, 4), False, -1, -1),
+    ((1, 7, 2, 1, 3), True, -1, -1),   # GQA 2:1, causal
+    ((2, 5, 4, 2, 3), True, 2, -1),    # window + GQA
+    ((1, 4, 1, 1, 5), False, 1, 1),    # band
+])
+def test_gradients_match_central_differences(shape, causal, wl, wr):
+    """Analytic dQ, dK, dV equal central differences of L = sum(dO * O)
+    (h = 1e-6) on tiny fp64 inputs; pins the backward formulas, the scale in
+    dQ/dK and the GQA reduction of dK/dV."""
+    B, N, Hq, Hkv, d = shape
+    rng = np.random.default_rng(6)
+    q = _rand((B, N, Hq, d), rng)
+    k = _rand((B, N + 1, Hkv, d), rng)   # Nq != Nk as well
+    v = _rand((B, N + 1, Hkv, d), rng)
+    do = _rand((B, N, Hq, d), rng)
+    kw = dict(scale=0.8, causal=causal, window=(wl, wr))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, nthreads=2, **kw)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args = {"q": q, "k": k, "v": v}
+            args[name] = xp
+            lp = _loss(args["q"], args["k"], args["v"], do, **kw)
+            args[name] = xm
+            lm = _loss(args["q"], args["k"], args["v"], do, **kw)
+            num[idx] = (lp - lm) / (2 * h)
+        err = np.abs(num - g).max() / max(1e-12, np.abs(g).max())
+        assert err < 1e-6, (name, err)
+
+
+# --------------------------------------------------------------- invariants
+
+def _rand_qkv(rng, B=1, Nq=17, Nk=17, Hq=2, Hkv=2, d=6):
+    return (_rand((B, Nq, Hq, d), rng), _rand((B, Nk, Hkv, d), rng),
+            _rand((B, Nk, Hkv, d), rng), _rand((B, Nq, Hq, d), rng))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gradient_sums(causal):
+    """Rows of P sum to 1 -> sum_j dV_j = sum_i dO_i; rows of dS sum to 0 ->
+    sum_j dK_j = 0 (per head, MHA, every row has a visible key)."""
+    rng = np.random.default_rng(7)
+    q, k, v, do = _rand_qkv(rng)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, scale=0.4, causal=causal, nthreads=2)
+    np.testing.assert_allclose(dv.sum(axis=1), do.sum(axis=1), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-12)
+
+
+def test_key_shift_invariance():
+    """Adding u to every key leaves O unchanged and shifts LSE_i by scale*q_i.u."""
+    rng = np.random.default_rng(8)
+    q, k, v, _ = _rand_qkv(rng)
+    u = 5.0 * _rand((6,), rng)
+    o1, l1 = oracle.attn_fwd(q, k, v, scale=0.5, causal=True, nthreads=2)
+    o2, l2 = oracle.attn_fwd(q, k + u, v, scale=0.5, causal=True, nthreads=2)
+    np.testing.assert_allclose(o2, o1, rtol=1e-11, atol=1e-11)
+    shift = 0.5 * np.einsum("bihc,c->bhi", q, u)
+    np.testing.assert_allclose(l2, l1 + shift, rtol=1e-11, atol=1e-11)
+
+
+def test_permutation_invariance_non_causal():
+    """Permuting keys and values together leaves O and LSE unchanged (no mask)."""
+    rng = np.random.default_rng(9)
+    q, k, v, _ = _rand_qkv(rng)
+    perm = rng.permutation(k.shape[1])
+    o1, l1 = oracle.attn_fwd(q, k, v, nthreads=2)
+    o2, l2 = oracle.attn_fwd(q, k[:, perm], v[:, perm], nthreads=2)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(l2, l1, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal,wl", [(False, -1), (True, 4)])
+def test_gqa_equals_mha_with_repeated_kv(causal, wl):
+    """GQA (Hq = 4, Hkv = 2) equals MHA with each KV head repeated for its group
+    (contiguous groups), and GQA dK/dV are the group sums of the MHA ones."""
+    rng = np.random.default_rng(10)
+    q, k, v, do = _rand_qkv(rng, Hq=4, Hkv=2)
+    kr, vr = np.repeat(k, 2, axis=2), np.repeat(v, 2, axis=2)
+    kw = dict(scale=0.6, causal=causal, window=(wl, -1), nthreads=2)
+    o1, l1 = oracle.attn_fwd(q, k, v, **kw)
+    o2, l2 = oracle.attn_fwd(q, kr, vr, **kw)
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=1e-13, atol=1e-13)
+    dq1, dk1, dv1 = oracle.attn_bwd(q, k, v, do, **kw)
+    dq2, dk2, dv2 = oracle.attn_bwd(q, kr, vr, do, **kw)
+    np.testing.assert_allclose(dq1, dq2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dk1, dk2.reshape(1, 17, 2, 2, 6).sum(axis=3), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dv1, dv2.reshape(1, 17, 2, 2, 6).sum(axis=3), rtol=1e-12, atol=1e-12)
+
+
+def test_output_is_convex_combination_of_values():
+    """O_i is a convex combination of V rows: min_j V_jc <= O_ic <= max_j V_jc."""
+    rng = np.random.default_rng(11)
+    q, k, v, _ = _rand_qkv(rng)
+    q *= 4
+    o, _ = oracle.attn_fwd(q, k, v, causal=False, nthreads=2)
+    assert np.all(o <= v.max(axis=1, keepdims=True) + 1e-12)
+    assert np.all(o >= v.min(axis=1, keepdims=True) - 1e-12)
+
+
+def test_thread_count_does_not_change_results():
+    """The oracle is reproducible: 1 and 5 threads give identical bits."""
+    rng = np.random.default_rng(12)
+    q, k, v, do = _rand_qkv(rng, Hq=4, Hkv=2)
+    a = oracle.attn_bwd(q, k, v, do, causal=True, nthreads=1)
+    b = oracle.attn_bwd(q, k, v, do, causal=True, nthreads=5)
+    for x, y in zip(a, b):
+        # dK/dV sums are re-associated across thread slices: equal to rounding
+        np.testing.assert_allclose(x, y, rtol=1e-13, atol=1e-13)
+    o1, _ = oracle.attn_fwd(q, k, v, nthreads=1)
+    o2, _ = oracle.attn_fwd(q, k, v, nthreads=5)
+    np.testing.assert_array_equal(o1, o2)
