@@ -1,0 +1,498 @@
+"""Benchmark of exact attention (forward + backward, bf16, causal) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole hot path over one batch: fa_fwd (O, LSE) then fa_bwd
+(dQ, dK, dV).  The headline workload is the training shape (B=2, H=16,
+N=2048, d=128, causal); the long wide shape (B=1, H=96, N=8192, d=128,
+causal) that the throughput target names is measured alongside it under
+``extra``.  FLOPs follow the metric: forward 4*B*H*N^2*d, halved when causal;
+forward+backward = 3.5x forward.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream with a 256 MiB write between steps to flush L2
+(outside the events); barrier + synchronize around the loop; with N > 1
+processes (torchrun) every rank runs its own batch (weak scaling, no
+collective on the data path) and the time is the max over ranks.  Rank 0
+prints one JSON line.
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm) on a
+bounded sample of the same workload on the host cores.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s fwd & fwd+bwd (bf16, causal) and % of B200 dense BF16 peak"
+DENSE_PEAK_TFLOPS = 2250.0  # NVIDIA B200 dense BF16 datasheet figure
+
+WORKLOADS = {
+    "train": dict(name="training-shape attention B=2 H=16 N=2048 d=128 causal fwd+bwd",
+                  B=2, N=2048, H=16, Hkv=16, d=128, causal=True, window=(-1, -1), seed=1002),
+    "wide": dict(name="long wide attention B=1 H=96 N=8192 d=128 causal fwd+bwd",
+                 B=1, N=8192, H=96, Hkv=96, d=128, causal=True, window=(-1, -1), seed=1005),
+    # a third of the wide shape: inputs still larger than L2, small enough for a
+    # full profiler capture of single launches
+    "mid": dict(name="attention B=1 H=32 N=8192 d=128 causal fwd+bwd",
+                B=1, N=8192, H=32, Hkv=32, d=128, causal=True, window=(-1, -1), seed=1006),
+}
+
+
+def fwd_flops(w):
+    f = 4.0 * w["B"] * w["H"] * w["N"] * w["N"] * w["d"]
+    return f / 2 if w["causal"] else f
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        import torch
+        try:
+            self.index = "GPU-%s" % torch.cuda.get_device_properties(device).uuid
+        except Exception:
+            self.index = str(device.index)
+        self.proc = None
+        self.tmp = None
+
+    def __enter__(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.index, "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.tmp is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.tmp.flush()
+        with open(self.tmp.name) as f:
+            rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("--gpus %d needs torchrun with %d processes" % (args.gpus, args.gpus))
+    return world, rank, local
+
+
+def max_over_ranks(value, world):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ GPU arm
+
+def make_device_inputs(w, rank, dev):
+    import torch
+    from seeded_inputs import make_inputs
+    inp = make_inputs(w["B"], w["N"], w["N"], w["H"], w["Hkv"], w["d"], w["seed"] + 7919 * rank)
+    return {n: t.to(dev) for n, t in inp.items()}, inp
+
+
+def time_gpu(w, steps, warmup, world, rank, dev, with_e2e=True, with_trace=True):
+    import torch
+    import exact_io_aware_89_b200 as fa
+
+    x, host = make_device_inputs(w, rank, dev)
+    q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+    B, N, H, Hkv, d = w["B"], w["N"], w["H"], w["Hkv"], w["d"]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(16, fa.fa_bwd_workspace_size(B, N, H, d)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    scale = 1.0 / math.sqrt(d)
+    c, (wl, wr) = int(w["causal"]), w["window"]
+
+    def step(q_, k_, v_, do_):
+        st = fa.fa_fwd(q_.data_ptr(), k_.data_ptr(), v_.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                       B, N, N, H, Hkv, d, scale, c, wl, wr, sp)
+        if st:
+            raise fa.FAError("fa_fwd", st)
+        st = fa.fa_bwd(q_.data_ptr(), k_.data_ptr(), v_.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                       do_.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, N, H, Hkv,
+                       d, scale, c, wl, wr, ws.data_ptr(), ws.numel(), sp)
+        if st:
+            raise fa.FAError("fa_bwd", st)
+
+    def fwd_only():
+        st = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                       B, N, N, H, Hkv, d, scale, c, wl, wr, sp)
+        if st:
+            raise fa.FAError("fa_fwd", st)
+
+    for _ in range(warmup):
+        step(q, k, v, do)
+    torch.cuda.synchronize()
+    if fa.fa_get_device_status(None) != 0:
+        raise RuntimeError("device status reports a timed-out wait")
+
+    # --- device-timed loop (inputs resident in HBM)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    if with_trace:
+        fa.fa_trace_enable(1)
+        fa.fa_trace_read()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clocks:
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step(q, k, v, do)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    trace_ms, trace_n = (fa.fa_trace_read() if with_trace else ({}, {}))
+    if with_trace:
+        fa.fa_trace_enable(0)
+
+    # --- forward alone (for the fwd TFLOP/s the metric also names)
+    fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        fev[i][0].record(stream)
+        fwd_only()
+        fev[i][1].record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = [a.elapsed_time(b) for a, b in fev]
+
+    out = dict(step_ms=step_ms, fwd_ms=fwd_ms, trace_ms=trace_ms, trace_n=trace_n,
+               clocks=clocks.summary())
+
+    # --- end to end through the public API: pinned host inputs in, results out
+    if with_e2e:
+        hin = {n: t.pin_memory() for n, t in host.items()}
+        hout = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv))}
+        dbuf = {n: torch.empty_like(x[n]) for n in ("q", "k", "v", "do")}
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in hout.values())
+        e_steps = max(3, min(steps, 10))
+        eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(e_steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(e_steps):
+            eev[i][0].record(stream)
+            for n in ("q", "k", "v", "do"):
+                dbuf[n].copy_(hin[n], non_blocking=True)
+            step(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["do"])
+            hout["o"].copy_(o, non_blocking=True)
+            hout["dq"].copy_(dq, non_blocking=True)
+            hout["dk"].copy_(dk, non_blocking=True)
+            hout["dv"].copy_(dv, non_blocking=True)
+            eev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        out["e2e_ms"] = [a.elapsed_time(b) for a, b in eev]
+        out["h2d"], out["d2h"] = h2d, d2h
+    if fa.fa_get_device_status(None) != 0:
+        raise RuntimeError("device status reports a timed-out wait")
+    del flush
+    return out
+
+
+def kernel_algorithmic(w):
+    """Algorithmic work per launch of each kernel kind (FLOPs for the tensor-core
+    kernels, bytes for the preprocess).  The backward's five contractions
+    (S, dP, dV, dK, dQ; 2.5x forward) are split between the dK/dV kernel (S,
+    dP, dV, dK = 2x forward) and the dQ kernel (dQ = 0.5x forward; its own
+    recomputation of S and dP is not algorithmic work)."""
+    F = fwd_flops(w)
+    rows = w["B"] * w["H"] * w["N"]
+    return {
+        "fwd": ("tensor", F),
+        "bwd_dkdv": ("tensor", 2.0 * F),
+        "bwd_dq": ("tensor", 0.5 * F),
+        "bwd_prep": ("hbm", rows * (2 * w["d"] * 2 + 4 + 8)),
+    }
+
+
+def roofline(w, res, peaks):
+    alg = kernel_algorithmic(w)
+    per = {}
+    for kind, (bound, work) in alg.items():
+        n = res["trace_n"].get(kind, 0)
+        if not n:
+            continue
+        avg_ms = res["trace_ms"][kind] / n
+        if bound == "tensor":
+            ach = work / (avg_ms * 1e-3) / 1e12
+            peak = peaks["bf16_sustained"]
+            unit = "TFLOP/s"
+        else:
+            ach = work / (avg_ms * 1e-3) / 1e9
+            peak = peaks["hbm_gbs"]
+            unit = "GB/s"
+        per[kind] = dict(bound=bound, achieved=round(ach, 2), peak=peak, unit=unit,
+                         frac=round(ach / peak, 4), avg_ms=round(avg_ms, 4), launches=n,
+                         share=None)
+    total = sum(res["trace_ms"].get(k, 0.0) for k in per)
+    for k in per:
+        per[k]["share"] = round(res["trace_ms"][k] / total, 4) if total else None
+    dom = max(per, key=lambda k: res["trace_ms"][k]) if per else None
+    return dom, per
+
+
+# ------------------------------------------------------------ CPU oracle arm
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_sample(w, max_heads=None, budget_s=20.0):
+    """Time the fp64 oracle's forward + backward on whole heads of the workload
+    (full N) until about budget_s has passed; return (TFLOP/s by the metric's
+    count, heads timed, seconds, threads)."""
+    import numpy as np
+    import oracle
+    from seeded_inputs import make_inputs
+    if w["name"] not in _ORACLE_INPUTS:
+        inp = make_inputs(w["B"], w["N"], w["N"], w["H"], w["Hkv"], w["d"], w["seed"])
+        _ORACLE_INPUTS[w["name"]] = {n: t.double().numpy() for n, t in inp.items()}
+    f64 = _ORACLE_INPUTS[w["name"]]
+    scale = 1.0 / math.sqrt(w["d"])
+    per_head = fwd_flops(w) / (w["B"] * w["H"]) * 3.5
+    nthreads = oracle.default_threads()
+    heads, t_total = 0, 0.0
+    total_heads = w["B"] * w["H"]
+    G = w["H"] // w["Hkv"]
+    while heads < (max_heads or total_heads):
+        b, h = divmod(heads, w["H"])
+        hk = h // G
+        sl = lambda a, hh: np.ascontiguousarray(a[b:b + 1, :, hh:hh + 1])
+        q, k, v, do = sl(f64["q"], h), sl(f64["k"], hk), sl(f64["v"], hk), sl(f64["do"], h)
+        t0 = time.perf_counter()
+        oracle.attn_fwd(q, k, v, scale=scale, causal=w["causal"], window=w["window"],
+                        nthreads=nthreads)
+        oracle.attn_bwd(q, k, v, do, scale=scale, causal=w["causal"], window=w["window"],
+                        nthreads=nthreads)
+        t_total += time.perf_counter() - t0
+        heads += 1
+        if t_total >= budget_s:
+            break
+    return per_head * heads / t_total / 1e12, heads, t_total, nthreads
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle as it stands, on the host cores.  Each
+    step is a bounded sample of the workload (one whole head at full N, forward
+    and backward); the batch time is extrapolated from the per-head median."""
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_sample(w, max_heads=1, budget_s=0.0)
+    samples, threads = [], 1
+    for _ in range(args.steps):
+        _, h_s, s_s, threads = oracle_sample(w, max_heads=1, budget_s=0.0)
+        samples.append(s_s / h_s)
+    per_head = fwd_flops(w) / (w["B"] * w["H"]) * 3.5
+    step_s = statistics.median(samples) * w["B"] * w["H"]
+    value = per_head * w["B"] * w["H"] / step_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), bf16-rounded)",
+        "config": {"workload": w["name"], "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
+                   "causal": w["causal"]},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": "1 of %d heads per step (full N, fwd+bwd), batch time "
+                                   "extrapolated from the per-head median" % (w["B"] * w["H"])},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    w = WORKLOADS[args.workload]
+    res = time_gpu(w, args.steps, args.warmup, world, rank, dev)
+    t_ms = sum(res["step_ms"])
+    t_max = max_over_ranks(t_ms, world)
+    F = fwd_flops(w)
+    total = 3.5 * F * world * args.steps
+    value = total / (t_max * 1e-3) / 1e12
+    fwd_tf = F * world * args.steps / (max_over_ranks(sum(res["fwd_ms"]), world) * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(sum(res["e2e_ms"]), world)
+    e2e_val = 3.5 * F * world * len(res["e2e_ms"]) / (e2e_ms * 1e-3) / 1e12
+    dom, per = roofline(w, res, peaks)
+    launches = int(sum(res["trace_n"].values()))
+
+    extra = []
+    if args.extra and args.workload != "wide":
+        we = WORKLOADS["wide"]
+        r2 = time_gpu(we, max(3, args.steps // 2), max(3, args.warmup), world, rank, dev,
+                      with_e2e=False)
+        F2 = fwd_flops(we)
+        tf2 = 3.5 * F2 * world * len(r2["step_ms"]) / (
+            max_over_ranks(sum(r2["step_ms"]), world) * 1e-3) / 1e12
+        ff2 = F2 * world * len(r2["fwd_ms"]) / (
+            max_over_ranks(sum(r2["fwd_ms"]), world) * 1e-3) / 1e12
+        d2, per2 = roofline(we, r2, peaks)
+        extra.append({"workload": we["name"], "fwd_bwd_tflops": round(tf2, 2),
+                      "fwd_tflops": round(ff2, 2),
+                      "fwd_bwd_pct_dense_peak": round(100 * tf2 / (world * DENSE_PEAK_TFLOPS), 2),
+                      "fwd_pct_dense_peak": round(100 * ff2 / (world * DENSE_PEAK_TFLOPS), 2),
+                      "ms_per_step": round(statistics.mean(r2["step_ms"]), 4),
+                      "kernels": per2, "clocks": r2["clocks"]})
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        tf_c, heads, secs, threads = oracle_sample(w, budget_s=args.oracle_budget)
+        cpu = {"value": round(tf_c, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": "%d of %d heads, full N, fwd+bwd, %.1f s" % (heads, w["B"] * w["H"], secs)}
+    dk = per.get(dom, {}) if dom else {}
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(statistics.mean(res["step_ms"]), 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1), bf16)",
+        "config": {"workload": w["name"], "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
+                   "causal": w["causal"], "global_batch": w["B"] * world,
+                   "parallelism": "dp%d" % world,
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "fwd_tflops": round(fwd_tf, 3),
+        "fwd_bwd_pct_dense_peak": round(100 * value / (world * DENSE_PEAK_TFLOPS), 2),
+        "fwd_pct_dense_peak": round(100 * fwd_tf / (world * DENSE_PEAK_TFLOPS), 2),
+        "roofline": {"kernel": dom, "bound": dk.get("bound"), "achieved": dk.get("achieved"),
+                     "peak": dk.get("peak"), "unit": dk.get("unit"), "frac": dk.get("frac"),
+                     "traffic": None,
+                     "peak_source": "%s, %s" % (peaks["source"],
+                                                "sustained" if dk.get("bound") == "tensor" else "copy")},
+        "kernels": per,
+        "gpu_launches": launches,
+        "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": res["h2d"],
+                "d2h_bytes_per_step": res["d2h"]},
+        "clocks": res["clocks"],
+        "cpu_baseline": cpu,
+        "extra": extra,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="train")
+    ap.add_argument("--no-extra", dest="extra", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-budget", type=float, default=15.0,
+                    help="seconds of oracle time for the CPU baseline sample")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)  # rank 0 alone; no process group
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,203 @@
+"""Python binding of libfa, exact IO-aware attention for NVIDIA B200 (sm_100a).
+
+The C ABI (include/fa.h) is the product boundary; this module only marshals
+arguments to it.  Two layers:
+
+* ``fa_fwd``, ``fa_bwd``, ``fa_fwd_f32``, ``fa_bwd_f32``, ``fa_bwd_workspace_size``,
+  ``fa_get_device_status``, ``fa_status_string``: the C entry points under the
+  same names, taking raw device pointers (ints) and sizes, returning the
+  status code.
+* ``attention_forward`` / ``attention_backward``: the same calls on torch CUDA
+  tensors (torch only allocates the outputs and supplies the current stream).
+
+There is no fallback: if libfa.so cannot be loaded or built, importing the
+tensor API raises, and every computation runs in the library's CUDA kernels.
+"""
+import ctypes
+import math
+import os
+
+__all__ = [
+    "FAError", "load_library", "library_path",
+    "fa_fwd", "fa_bwd", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
+    "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
+    "KERNEL_KINDS", "attention_forward", "attention_backward",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libfa.so")
+_lib = None
+
+FA_OK = 0
+
+
+class FAError(RuntimeError):
+    """A libfa entry point returned a non-zero status."""
+
+    def __init__(self, name, status):
+        super().__init__("%s failed: %s (%d)" % (name, fa_status_string(status), status))
+        self.status = status
+
+
+def library_path():
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libfa.so from the package directory, building it with nvcc if it is
+    missing.  Raises if neither works: there is no other implementation."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        from . import build as _build
+        _build.build()
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    sz = ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp]
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i,
+                           vp, sz, vp]
+    lib.fa_fwd_f32.argtypes = lib.fa_fwd.argtypes
+    lib.fa_bwd_f32.argtypes = lib.fa_bwd.argtypes
+    lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_bwd_workspace_size.restype = sz
+    lib.fa_get_device_status.argtypes = [vp]
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_trace_enable.argtypes = [i]
+    lib.fa_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+    for name in ("fa_fwd", "fa_bwd", "fa_fwd_f32", "fa_bwd_f32", "fa_get_device_status",
+                 "fa_trace_enable", "fa_trace_read"):
+        getattr(lib, name).restype = i
+    _lib = lib
+    return lib
+
+
+# ----------------------------------------------------------- C entry points
+
+def fa_fwd(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, stream):
+    return load_library().fa_fwd(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal,
+                                 win_l, win_r, stream)
+
+
+def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l,
+           win_r, workspace, workspace_bytes, stream):
+    return load_library().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale,
+                                 causal, win_l, win_r, workspace, workspace_bytes, stream)
+
+
+def fa_fwd_f32(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, stream):
+    return load_library().fa_fwd_f32(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal,
+                                     win_l, win_r, stream)
+
+
+def fa_bwd_f32(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l,
+               win_r, workspace, workspace_bytes, stream):
+    return load_library().fa_bwd_f32(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d,
+                                     scale, causal, win_l, win_r, workspace, workspace_bytes,
+                                     stream)
+
+
+def fa_bwd_workspace_size(B, Nq, Hq, d):
+    return load_library().fa_bwd_workspace_size(B, Nq, Hq, d)
+
+
+def fa_get_device_status(stream=None):
+    return load_library().fa_get_device_status(stream)
+
+
+def fa_status_string(status):
+    return load_library().fa_status_string(int(status)).decode()
+
+
+KERNEL_KINDS = ("fwd", "bwd_prep", "bwd_dq", "bwd_dkdv", "f32")
+
+
+def fa_trace_enable(on):
+    return load_library().fa_trace_enable(int(bool(on)))
+
+
+def fa_trace_read():
+    """Return ({kind: device ms}, {kind: launches}) accumulated since the last read."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_longlong * n)()
+    _check("fa_trace_read", load_library().fa_trace_read(ms, cnt))
+    return dict(zip(KERNEL_KINDS, ms)), dict(zip(KERNEL_KINDS, cnt))
+
+
+# ------------------------------------------------------------ tensor layer
+
+def _check(name, st):
+    if st != FA_OK:
+        raise FAError(name, st)
+
+
+def _dims(q, k, v):
+    import torch
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, N, H, d]")
+    B, Nq, Hq, d = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k and v must be [B, Nk, Hkv, d] with q's B and d")
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous CUDA tensors")
+        if t.dtype not in (torch.bfloat16, torch.float32) or t.dtype != q.dtype:
+            raise ValueError("tensors must all be bf16 (or all fp32)")
+    return B, Nq, k.shape[1], Hq, k.shape[2], d
+
+
+def _stream():
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _window(causal, window):
+    wl, wr = (-1, -1) if window is None else window
+    return int(bool(causal)), int(wl), int(wr)
+
+
+def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), out=None, lse=None):
+    """O, LSE = attention(q, k, v) on the current CUDA stream.
+
+    q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] contiguous, all bf16 (fa_fwd) or all fp32
+    (fa_fwd_f32).  Returns (o like q, lse [B,Hq,Nq] fp32).  ``window`` is
+    (left, right), negative = unbounded; ``causal`` aligns bottom-right.
+    """
+    import torch
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    fn = fa_fwd if q.dtype == torch.bfloat16 else fa_fwd_f32
+    _check(fn.__name__, fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, _stream()))
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1, -1),
+                       dq=None, dk=None, dv=None, workspace=None):
+    """dQ, dK, dV of sum(do * o) on the current CUDA stream (deterministic).
+
+    ``workspace``: optional uint8 CUDA tensor of at least
+    ``fa_bwd_workspace_size(B, Nq, Hq, d)`` bytes; allocated here if omitted.
+    """
+    import torch
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    wsb = fa_bwd_workspace_size(B, Nq, Hq, d)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
+    fn = fa_bwd if q.dtype == torch.bfloat16 else fa_bwd_f32
+    _check(fn.__name__, fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Nq, Nk,
+                           Hq, Hkv, d, scale, c, wl, wr, workspace.data_ptr(),
+                           workspace.numel() * workspace.element_size(), _stream()))
+    return dq, dk, dv

@@ -1,0 +1,374 @@
+// fa_api.cu -- the C ABI of libfa (declared in include/fa.h): argument
+// validation, TMA descriptor encoding and kernel launches on the caller's
+// stream.  No device memory is allocated here and nothing runs on the CPU
+// besides the checks.
+#include <cstdio>
+#include <mutex>
+#include <vector>
+
+#include "fa_bwd.cuh"
+#include "fa_f32.cuh"
+#include "fa_fwd.cuh"
+#include "fa_host.cuh"
+
+using namespace fa;
+
+namespace {
+
+// ---------------------------------------------------------------- tracing
+struct TraceRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::mutex g_trace_mu;
+bool g_trace_on = false;
+std::vector<cudaEvent_t> g_event_pool;
+std::vector<TraceRec> g_trace;
+constexpr int kEventPoolInit = 512;
+
+bool take_event(cudaEvent_t* e) {
+  if (!g_event_pool.empty()) {
+    *e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return true;
+  }
+  return cudaEventCreate(e) == cudaSuccess;
+}
+
+// Brackets one launch with events when tracing is on.
+struct TraceScope {
+  int kind;
+  cudaStream_t stream;
+  cudaEvent_t a = nullptr, b = nullptr;
+  bool active = false;
+  TraceScope(int k, cudaStream_t s) : kind(k), stream(s) {
+    std::lock_guard<std::mutex> lock(g_trace_mu);
+    if (!g_trace_on) return;
+    if (!take_event(&a) || !take_event(&b)) return;
+    active = cudaEventRecord(a, stream) == cudaSuccess;
+  }
+  ~TraceScope() {
+    if (!active) return;
+    std::lock_guard<std::mutex> lock(g_trace_mu);
+    if (cudaEventRecord(b, stream) == cudaSuccess) g_trace.push_back({kind, a, b});
+  }
+};
+
+// A device-side wait gives up after this long (the kernels' own waits are
+// microseconds; the limit only matters when something is broken).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// fwd: {d, Q tiles per CTA, key tile, K/V ring depth}
+using Fwd64 = FwdCfg<64, 2, 128, 3>;
+using Fwd128 = FwdCfg<128, 2, 128, 2>;
+using Fwd256 = FwdCfg<256, 1, 64, 2>;
+// dQ: {d, Q tiles per CTA, key tile, K/V ring depth}
+using Dq64 = DqCfg<64, 2, 64, 3>;
+using Dq128 = DqCfg<128, 2, 64, 2>;
+using Dq256 = DqCfg<256, 1, 64, 1>;
+// dK/dV: {d, accumulated d slice, query tile, Q/dO ring depth}
+using Dkv64 = DkvCfg<64, 64, 64, 4>;
+using Dkv128 = DkvCfg<128, 128, 64, 3>;
+using Dkv256 = DkvCfg<256, 128, 64, 1>;
+
+constexpr int kMaxDevices = 64;
+
+template <typename Kernel>
+cudaError_t smem_attr_once(Kernel kernel, int bytes, int* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (!__atomic_load_n(&done[dev], __ATOMIC_ACQUIRE)) {
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    __atomic_store_n(&done[dev], 1, __ATOMIC_RELEASE);
+  }
+  return cudaSuccess;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+MaskSpec make_mask(int Nq, int Nk, int causal, int win_l, int win_r) {
+  MaskSpec m;
+  m.Nq = Nq;
+  m.Nk = Nk;
+  m.wl = win_l < 0 ? -1 : win_l;
+  m.wr = causal ? 0 : (win_r < 0 ? -1 : win_r);
+  return m;
+}
+
+int check_common(const void* q, const void* k, const void* v, int B, int Nq, int Nk, int Hq,
+                 int Hkv, float scale) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return FA_ERR_INVALID_ARG;
+  return check_sizes(B, Nq, Nk, Hq, Hkv, scale);
+}
+
+int pad_rows(int Nq) { return (Nq + 255) / 256 * 256; }
+
+// ------------------------------------------------------------------ forward
+template <class C>
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+               int Nk, int Hq, int Hkv, float scale, const MaskSpec& mask, cudaStream_t stream) {
+  static int attr_done[kMaxDevices] = {0};
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_bnhd(&tq, q, B, Nq, Hq, C::D, C::BM) || !encode_bnhd(&tk, k, B, Nk, Hkv, C::D, C::BN) ||
+      !encode_bnhd(&tv, v, B, Nk, Hkv, C::D, C::BN) || !encode_bnhd(&to, o, B, Nq, Hq, C::D, C::BM))
+    return FA_ERR_CUDA;
+  FwdParams p;
+  p.B = B; p.Nq = Nq; p.Nk = Nk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
+  p.scale_log2 = scale * kLog2e;
+  p.mask = mask;
+  p.n_qgroups = (Nq + C::NQT * C::BM - 1) / (C::NQT * C::BM);
+  p.lse = lse;
+  p.wait_limit_ns = kWaitLimitNs;
+  auto kern = fa_fwd_kernel<C>;
+  if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
+  const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
+  {
+    TraceScope tr(FA_KERNEL_FWD, stream);
+    kern<<<static_cast<unsigned>(grid), C::NTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+  }
+  return launch_status();
+}
+
+// ------------------------------------------------------------------ backward
+template <class CQ, class CKV>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
+               float scale, const MaskSpec& mask, float* ws, cudaStream_t stream) {
+  static int attr_dq[kMaxDevices] = {0};
+  static int attr_kv[kMaxDevices] = {0};
+  constexpr int D = CQ::D;
+  const int Nq_pad = pad_rows(Nq);
+  const long long rows_pad = static_cast<long long>(B) * Hq * Nq_pad;
+  {
+    const long long blocks = (rows_pad * 32 + 255) / 256;
+    TraceScope tr(FA_KERNEL_BWD_PREP, stream);
+    fa_bwd_prep_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, ws, B, Nq,
+        Hq, D, Nq_pad);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  BwdParams p;
+  p.B = B; p.Nq = Nq; p.Nk = Nk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.mask = mask;
+  p.Nq_pad = Nq_pad;
+  p.D = ws;
+  p.lse2 = ws + rows_pad;
+  p.n_qgroups = (Nq + CQ::NQT * CQ::BM - 1) / (CQ::NQT * CQ::BM);
+  p.n_kvtiles = (Nk + CKV::BN - 1) / CKV::BN;
+  p.wait_limit_ns = kWaitLimitNs;
+  {
+    CUtensorMap tq, tk, tv, tdo, tdq;
+    if (!encode_bnhd(&tq, q, B, Nq, Hq, D, CQ::BM) || !encode_bnhd(&tk, k, B, Nk, Hkv, D, CQ::BN) ||
+        !encode_bnhd(&tv, v, B, Nk, Hkv, D, CQ::BN) || !encode_bnhd(&tdo, dO, B, Nq, Hq, D, CQ::BM) ||
+        !encode_bnhd(&tdq, dq, B, Nq, Hq, D, CQ::BM))
+      return FA_ERR_CUDA;
+    auto kern = fa_bwd_dq_kernel<CQ>;
+    if (smem_attr_once(kern, CQ::SMEM_BYTES, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
+    const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
+    TraceScope tr(FA_KERNEL_BWD_DQ, stream);
+    kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  {
+    CUtensorMap tq, tk, tv, tdo, tdk, tdv;
+    if (!encode_bnhd(&tq, q, B, Nq, Hq, D, CKV::BM) || !encode_bnhd(&tk, k, B, Nk, Hkv, D, CKV::BN) ||
+        !encode_bnhd(&tv, v, B, Nk, Hkv, D, CKV::BN) || !encode_bnhd(&tdo, dO, B, Nq, Hq, D, CKV::BM) ||
+        !encode_bnhd(&tdk, dk, B, Nk, Hkv, D, CKV::BN) || !encode_bnhd(&tdv, dv, B, Nk, Hkv, D, CKV::BN))
+      return FA_ERR_CUDA;
+    auto kern = fa_bwd_dkdv_kernel<CKV>;
+    if (smem_attr_once(kern, CKV::SMEM_BYTES, attr_kv) != cudaSuccess) return FA_ERR_CUDA;
+    const dim3 grid(static_cast<unsigned>(static_cast<long long>(p.n_kvtiles) * B * Hkv), D / CKV::DV);
+    TraceScope tr(FA_KERNEL_BWD_DKDV, stream);
+    kern<<<grid, CKV::NTHREADS, CKV::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, p);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+size_t workspace_bytes(int B, int Nq, int Hq) {
+  if (B < 1 || Nq < 1 || Hq < 1) return 0;
+  return 2ull * static_cast<size_t>(B) * static_cast<size_t>(Hq) * static_cast<size_t>(pad_rows(Nq)) *
+         sizeof(float);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq, int Nk,
+           int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+           fa_stream_t stream) {
+  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_fwd<Fwd64>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, s);
+    case 128: return launch_fwd<Fwd128>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, s);
+    case 256: return launch_fwd<Fwd256>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, s);
+    default: return FA_ERR_UNSUPPORTED;
+  }
+}
+
+size_t fa_bwd_workspace_size(int B, int Nq, int Hq, int d) {
+  if (d < 1) return 0;
+  return workspace_bytes(B, Nq, Hq);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
+           int d, float scale, int causal, int win_l, int win_r, void* workspace,
+           size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(workspace) || workspace_bytes_ < workspace_bytes(B, Nq, Hq)) return FA_ERR_WORKSPACE;
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  switch (d) {
+    case 64:
+      return launch_bwd<Dq64, Dkv64>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+    case 128:
+      return launch_bwd<Dq128, Dkv128>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+    default:
+      return launch_bwd<Dq256, Dkv256>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+  }
+}
+
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Nq,
+               int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+               fa_stream_t stream) {
+  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if (d < 32 || d > 32 * kF32MaxPerLane || d % 32 != 0) return FA_ERR_UNSUPPORTED;
+  F32Params p;
+  p.B = B; p.Nq = Nq; p.Nk = Nk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv; p.d = d;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  p.Nq_pad = pad_rows(Nq);
+  p.D = nullptr;
+  p.lse2 = nullptr;
+  const long long warps = static_cast<long long>(B) * Nq * Hq;
+  const long long blocks = (warps + 3) / 4;
+  {
+    TraceScope tr(FA_KERNEL_F32, reinterpret_cast<cudaStream_t>(stream));
+    fa_fwd_f32_kernel<<<static_cast<unsigned>(blocks), 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        q, k, v, o, lse, p);
+  }
+  return launch_status();
+}
+
+int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* lse,
+               const float* dO, float* dq, float* dk, float* dv, int B, int Nq, int Nk, int Hq, int Hkv,
+               int d, float scale, int causal, int win_l, int win_r, void* workspace,
+               size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (d < 32 || d > 32 * kF32MaxPerLane || d % 32 != 0) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(workspace) || workspace_bytes_ < workspace_bytes(B, Nq, Hq)) return FA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  F32Params p;
+  p.B = B; p.Nq = Nq; p.Nk = Nk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv; p.d = d;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  p.Nq_pad = pad_rows(Nq);
+  float* ws = static_cast<float*>(workspace);
+  const long long rows_pad = static_cast<long long>(B) * Hq * p.Nq_pad;
+  p.D = ws;
+  p.lse2 = ws + rows_pad;
+  {
+    TraceScope tr(FA_KERNEL_F32, s);
+    fa_bwd_prep_kernel<float><<<static_cast<unsigned>((rows_pad * 32 + 255) / 256), 256, 0, s>>>(
+        o, dO, lse, ws, B, Nq, Hq, d, p.Nq_pad);
+  }
+  if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  const long long wq = static_cast<long long>(B) * Nq * Hq;
+  {
+    TraceScope tr(FA_KERNEL_F32, s);
+    fa_bwd_dq_f32_kernel<<<static_cast<unsigned>((wq + 3) / 4), 128, 0, s>>>(q, k, v, dO, dq, p);
+  }
+  if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  const long long wk = static_cast<long long>(B) * Nk * Hkv;
+  {
+    TraceScope tr(FA_KERNEL_F32, s);
+    fa_bwd_dkdv_f32_kernel<<<static_cast<unsigned>((wk + 3) / 4), 128, 0, s>>>(q, k, v, dO, dk, dv, p);
+  }
+  return launch_status();
+}
+
+int fa_get_device_status(fa_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return v == kDevTimeout ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+int fa_trace_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  if (on && !g_trace_on) {
+    while (static_cast<int>(g_event_pool.size()) < kEventPoolInit) {
+      cudaEvent_t e;
+      if (cudaEventCreate(&e) != cudaSuccess) return FA_ERR_CUDA;
+      g_event_pool.push_back(e);
+    }
+  }
+  g_trace_on = on != 0;
+  return FA_OK;
+}
+
+int fa_trace_read(double* ms, long long* launches) {
+  if (!ms || !launches) return FA_ERR_INVALID_ARG;
+  for (int i = 0; i < FA_KERNEL_KINDS; ++i) {
+    ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  std::lock_guard<std::mutex> lock(g_trace_mu);
+  int st = FA_OK;
+  for (const TraceRec& r : g_trace) {
+    float t = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+      st = FA_ERR_CUDA;
+    if (r.kind >= 0 && r.kind < FA_KERNEL_KINDS) {
+      ms[r.kind] += t;
+      launches[r.kind] += 1;
+    }
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_trace.clear();
+  return st;
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    default: return "FA_UNKNOWN_STATUS";
+  }
+}
+
+}  // extern "C"

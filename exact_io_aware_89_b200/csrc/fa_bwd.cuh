@@ -1,0 +1,670 @@
+// fa_bwd.cuh -- backward pass of exact attention on sm_100a.
+//
+// The pages fix only the strategy (abeam.tech FlashAttention summary,
+// "backward uses recomputation": keep the softmax statistics of the forward,
+// recompute attention blockwise instead of storing P).  The formulas are the
+// calculus of the loss L = sum(dO * O):
+//   P_ij  = exp(scale * q_i.k_j - LSE_i)         (recomputed from the saved LSE)
+//   D_i   = sum_c dO_ic O_ic
+//   dP_ij = dO_i . v_j,   dS_ij = P_ij (dP_ij - D_i)
+//   dV_j  = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j
+//
+// Three launches on the caller's stream:
+//   1. fa_bwd_prep_kernel : D_i and lse2_i = LSE_i * log2(e) into the workspace
+//                           (rows padded to a multiple of 256; padding rows get
+//                           lse2 = +inf so every P there is exactly 0).
+//   2. fa_bwd_dq_kernel   : query-stationary.  Per key tile: S = Q K^T and
+//                           dP = dO V^T (tcgen05, TMEM), dS in registers, dS
+//                           written back into TMEM as bf16, dQ += dS K with dS
+//                           read from TMEM.  dQ is accumulated in fp32 in TMEM
+//                           by one CTA in a fixed order, so it is deterministic
+//                           with no atomics and no extra workspace.
+//   3. fa_bwd_dkdv_kernel : key-stationary.  Per (query head of the group,
+//                           query tile): S^T = K Q^T and dP^T = V dO^T, then
+//                           P^T and dS^T (bf16, in TMEM over their sources),
+//                           dV += P^T dO and dK += dS^T Q.  dK/dV for a GQA group
+//                           are summed inside one CTA, in a fixed order.
+// Every contraction is a tcgen05 tile GEMM fed by TMA.
+#pragma once
+#include "fa_common.cuh"
+
+namespace fa {
+
+// =====================================================================
+// 1. preprocess: D = rowsum(dO * O), lse2 = LSE * log2(e)
+// =====================================================================
+template <typename T>
+__device__ __forceinline__ float load_as_float(const T* p);
+template <>
+__device__ __forceinline__ float load_as_float<float>(const float* p) {
+  return *p;
+}
+template <>
+__device__ __forceinline__ float load_as_float<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
+// one warp per (b, i, h) row; ws layout: D [B, Hq, Nq_pad] then lse2 [B, Hq, Nq_pad]
+template <typename T>
+__global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const T* __restrict__ o,
+                                                          const T* __restrict__ dout,
+                                                          const float* __restrict__ lse,
+                                                          float* __restrict__ ws, int B, int Nq,
+                                                          int Hq, int d, int Nq_pad) {
+  const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  const long long rows_pad = static_cast<long long>(B) * Hq * Nq_pad;
+  if (warp_id >= rows_pad) return;
+  const int i = static_cast<int>(warp_id % Nq_pad);
+  const long long bh = warp_id / Nq_pad;
+  const int h = static_cast<int>(bh % Hq);
+  const int b = static_cast<int>(bh / Hq);
+  float* Dp = ws + warp_id;
+  float* L2p = ws + rows_pad + warp_id;
+  if (i >= Nq) {
+    if (lane == 0) {
+      *Dp = 0.f;
+      *L2p = INFINITY;
+    }
+    return;
+  }
+  const size_t base = ((static_cast<size_t>(b) * Nq + i) * Hq + h) * d;
+  float acc = 0.f;
+  for (int c = lane; c < d; c += 32) acc += load_as_float(o + base + c) * load_as_float(dout + base + c);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    *Dp = acc;
+    const float L = lse[(static_cast<size_t>(b) * Hq + h) * Nq + i];
+    // a row with no visible key (LSE = -inf) has P = 0 everywhere
+    *L2p = (L == -INFINITY) ? INFINITY : L * kLog2e;
+  }
+}
+
+struct BwdParams {
+  int B, Nq, Nk, Hq, Hkv, group;
+  float scale;        // softmax scale (dQ, dK carry it)
+  float scale_log2;   // scale * log2(e)
+  MaskSpec mask;
+  int Nq_pad;
+  const float* D;     // [B, Hq, Nq_pad]
+  const float* lse2;  // [B, Hq, Nq_pad]
+  int n_qgroups;      // dq kernel: CTAs along the query axis
+  int n_kvtiles;      // dkdv kernel: CTAs along the key axis
+  unsigned long long wait_limit_ns;
+};
+
+// =====================================================================
+// 2. dQ: query-stationary
+// =====================================================================
+template <int D_, int NQT_, int BN_, int KST_>
+struct DqCfg {
+  static constexpr int D = D_, NQT = NQT_, BN = BN_, KST = KST_;
+  static constexpr int BM = 128;
+  static constexpr int NCHUNK = D / 64;
+  static constexpr int QCHUNK = BM * 128;
+  static constexpr int KCHUNK = BN * 128;
+  static constexpr int QTILE = NCHUNK * QCHUNK;
+  static constexpr int KTILE = NCHUNK * KCHUNK;
+  static constexpr int OFF_Q = 0;                             // Q tiles  [NQT]
+  static constexpr int OFF_DO = OFF_Q + NQT * QTILE;          // dO tiles [NQT]
+  static constexpr int OFF_K = OFF_DO + NQT * QTILE;          // K stages [KST]
+  static constexpr int OFF_V = OFF_K + KST * KTILE;           // V stages [KST]
+  static constexpr int OFF_BAR = OFF_V + KST * KTILE;
+  static constexpr int NBAR = 1 + 2 * KST + 2 * NQT + 1 + 1;  // q_full, kv_full/empty, sp_full/ds_full, dq_done, drain
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int NWARPS = 4 * NQT + 2;
+  static constexpr int NTHREADS = 32 * NWARPS;
+  static constexpr int TMA_WARP = 4 * NQT;
+  static constexpr int MMA_WARP = 4 * NQT + 1;
+  // TMEM: tile t: S at t*2*BN, dP at t*2*BN + BN (dS overlays dP's first BN/2), dQ at 2*BN*NQT + t*D
+  static constexpr int COL_DQ = 2 * BN * NQT;
+  static constexpr int TMEM_USED = COL_DQ + NQT * D;
+  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+  static_assert(TMEM_USED <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::NTHREADS, 1)
+    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+  constexpr int D = C::D, NQT = C::NQT, BN = C::BN, KST = C::KST, BM = C::BM;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = kv_full + KST;
+  uint64_t* sp_full = kv_empty + KST;  // [NQT]
+  uint64_t* ds_full = sp_full + NQT;   // [NQT]
+  uint64_t* dq_done = ds_full + NQT;
+  uint64_t* bar_drain = dq_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  const uint32_t sQ = sbase + C::OFF_Q, sdO = sbase + C::OFF_DO, sK = sbase + C::OFF_K,
+                 sV = sbase + C::OFF_V;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  const int BH = p.B * p.Hq;
+  const int bh = blockIdx.x % BH;
+  const int g = p.n_qgroups - 1 - blockIdx.x / BH;
+  const int b = bh / p.Hq, h = bh % p.Hq, hk = h / p.group;
+  const int r0 = g * NQT * BM;
+  const int r_last = min(p.Nq - 1, r0 + NQT * BM - 1);
+  const int key_lo = p.mask.lo(r0), key_hi = p.mask.hi(r_last);
+  const int j_begin = key_lo / BN;
+  const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int t = 0; t < NQT; ++t) {
+      mbar_init(&sp_full[t], 1);
+      mbar_init(&ds_full[t], BM);
+    }
+    mbar_init(dq_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::TMA_WARP) {
+    if (lane == 0 && n_kv > 0) {
+      mbar_expect_tx(q_full, 2 * NQT * C::QTILE);
+      for (int t = 0; t < NQT; ++t)
+        for (int c = 0; c < C::NCHUNK; ++c) {
+          tma_load_4d(sQ + t * C::QTILE + c * C::QCHUNK, &tm_q, q_full, c * 64, h, r0 + t * BM, b);
+          tma_load_4d(sdO + t * C::QTILE + c * C::QCHUNK, &tm_do, q_full, c * 64, h, r0 + t * BM, b);
+        }
+      int n_issued = 0;
+      for (int it = 0; it < n_kv; ++it) {
+        const int s = it % KST, use = it / KST;
+        const int krow = (j_begin + it) * BN;
+        if (use > 0 && !mbar_wait(&kv_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
+          break;
+        mbar_expect_tx(&kv_full[s], 2 * C::KTILE);
+        for (int c = 0; c < C::NCHUNK; ++c) {
+          tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, &kv_full[s], c * 64, hk, krow, b);
+          tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &kv_full[s], c * 64, hk, krow, b);
+        }
+        ++n_issued;
+      }
+      mbar_drain(q_full, 0, p.wait_limit_ns);
+      for (int s = 0; s < KST; ++s)
+        if (n_issued > s) mbar_drain(&kv_full[s], ((n_issued - 1 - s) / KST) & 1, p.wait_limit_ns);
+    }
+  } else if (warp == C::MMA_WARP) {
+    if (lane == 0 && n_kv > 0) {
+      constexpr uint32_t ID_S = idesc_bf16_f32(128, BN, false, false);
+      constexpr uint32_t ID_DQ = idesc_bf16_f32(128, D, false, true);
+      auto wait = [&](uint64_t* bar, uint32_t par) {
+        const bool ok = mbar_wait(bar, par, abort_flag, &g_status, p.wait_limit_ns);
+        tc_fence_after();
+        return ok;
+      };
+      // S_t = Q_t K_s^T and dP_t = dO_t V_s^T
+      auto issue_sdp = [&](int t, int s) {
+        const uint32_t d_s = tmem + t * 2 * BN, d_dp = d_s + BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2), kb = (kk & 3) * 32;
+          const uint32_t qo = t * C::QTILE + ko * C::QCHUNK + kb;
+          const uint32_t ks = s * C::KTILE + ko * C::KCHUNK + kb;
+          mma_ss(d_s, sdesc_sw128(sQ + qo, 16, 1024), sdesc_sw128(sK + ks, 16, 1024), ID_S, kk > 0);
+          mma_ss(d_dp, sdesc_sw128(sdO + qo, 16, 1024), sdesc_sw128(sV + ks, 16, 1024), ID_S, kk > 0);
+        }
+      };
+      // dQ_t (+)= dS_t K_s, dS from TMEM (bf16 over dP_t), K as MN-major B
+      auto issue_dq = [&](int t, int s, bool acc) {
+        const uint32_t d_dq = tmem + C::COL_DQ + t * D;
+        const uint32_t a_ds = tmem + t * 2 * BN + BN;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(d_dq, a_ds + kk * 8, sdesc_sw128(sK + s * C::KTILE + kk * 2048, C::KCHUNK, 1024),
+                 ID_DQ, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait(q_full, 0) && wait(&kv_full[0], 0);
+      if (ok) {
+        for (int t = 0; t < NQT; ++t) {
+          issue_sdp(t, 0);
+          tc_commit(&sp_full[t]);
+        }
+        for (int it = 0; it < n_kv && ok; ++it) {
+          const int s = it % KST, s1 = (it + 1) % KST;
+          for (int t = 0; t < NQT && ok; ++t) {
+            if (!(ok = wait(&ds_full[t], it & 1))) break;
+            issue_dq(t, s, it > 0);
+            if (t == NQT - 1) tc_commit(&kv_empty[s]);
+            if (it + 1 < n_kv) {
+              if (t == 0 && !(ok = wait(&kv_full[s1], ((it + 1) / KST) & 1))) break;
+              issue_sdp(t, s1);
+              tc_commit(&sp_full[t]);
+            }
+          }
+        }
+        tc_commit(dq_done);
+      }
+    }
+    if (lane == 0) {
+      tc_commit(bar_drain);
+      mbar_drain(bar_drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ dS warpgroups (thread = query row)
+    const int t = warp / 4;
+    const int r = threadIdx.x % BM;
+    const int row = r0 + t * BM + r;
+    const int lo = p.mask.lo(row), hi = p.mask.hi(row);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    const size_t srow = (static_cast<size_t>(b) * p.Hq + h) * p.Nq_pad + row;  // row < Nq_pad
+    const float lse2 = p.lse2[srow];
+    const float Drow = p.D[srow];
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < n_kv; ++it) {
+      ok = mbar_wait(&sp_full[t], it & 1, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[BN], dv[BN];
+      const uint32_t col_s = t * 2 * BN, col_dp = col_s + BN;
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        tmem_ld_x32(lane_base + col_s + cc * 32, &sv[cc * 32]);
+        tmem_ld_x32(lane_base + col_dp + cc * 32, &dv[cc * 32]);
+      }
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        tmem_ld_wait_x32(&sv[cc * 32]);
+        tmem_ld_wait_x32(&dv[cc * 32]);
+      }
+      float* sc = reinterpret_cast<float*>(sv);
+      const float* dp = reinterpret_cast<const float*>(dv);
+      const int k0 = (j_begin + it) * BN;
+      if (k0 < lo || k0 + BN - 1 > hi) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const int key = k0 + c;
+          if (key < lo || key > hi) sc[c] = -INFINITY;
+        }
+      }
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) {
+        const float p0 = ex2_approx(fmaf(sc[c], sl2, -lse2));
+        const float p1 = ex2_approx(fmaf(sc[c + 1], sl2, -lse2));
+        pk[c / 2] = pack_bf16x2(p0 * (dp[c] - Drow), p1 * (dp[c + 1] - Drow));
+      }
+#pragma unroll
+      for (int cc = 0; cc < BN / 64; ++cc) tmem_st_x32(lane_base + col_dp + cc * 32, &pk[cc * 32]);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ds_full[t]);
+    }
+    if (ok && n_kv > 0) {
+      ok = mbar_wait(dq_done, 0, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+    // epilogue: dQ * scale -> bf16 -> shared (this tile's Q buffer) -> TMA store
+    const uint32_t stage = sQ + t * C::QTILE;
+    if (ok) {
+#pragma unroll 1
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        uint32_t ov[64];
+        if (n_kv > 0) {
+          tmem_ld_x32(lane_base + C::COL_DQ + t * D + c * 64, ov);
+          tmem_ld_x32(lane_base + C::COL_DQ + t * D + c * 64 + 32, ov + 32);
+          tmem_ld_wait_x32(ov);
+          tmem_ld_wait_x32(ov + 32);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) ov[i] = 0u;
+        }
+        const float sc = p.scale;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float* f = reinterpret_cast<const float*>(ov + 8 * u);
+          st_shared_v4(stage + c * C::QCHUNK + sw128_offset(r, u), pack_bf16x2(f[0] * sc, f[1] * sc),
+                       pack_bf16x2(f[2] * sc, f[3] * sc), pack_bf16x2(f[4] * sc, f[5] * sc),
+                       pack_bf16x2(f[6] * sc, f[7] * sc));
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(1 + t, BM);
+    if (r == 0 && *abort_flag == 0 && r0 + t * BM < p.Nq) {
+      for (int c = 0; c < C::NCHUNK; ++c)
+        tma_store_4d(&tm_dq, stage + c * C::QCHUNK, c * 64, h, r0 + t * BM, b);
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == C::MMA_WARP) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// =====================================================================
+// 3. dK, dV: key-stationary
+// =====================================================================
+// D: head dim; DV: the slice of d whose dK/dV this CTA accumulates (D, or
+// 128 for D = 256, then blockIdx.y picks the slice); BM: query tile; ST: ring
+// depth of the (Q, dO, lse2, D) stages; LA: steps issued ahead (<= 2, <= ST).
+template <int D_, int DV_, int BM_, int ST_>
+struct DkvCfg {
+  static constexpr int D = D_, DV = DV_, BM = BM_, ST = ST_;
+  static constexpr int BN = 128;
+  static constexpr int LA = ST >= 2 ? 2 : 1;
+  static constexpr int NCHUNK = D / 64;
+  static constexpr int KCHUNK = BN * 128;
+  static constexpr int QCHUNK = BM * 128;
+  static constexpr int KTILE = NCHUNK * KCHUNK;
+  static constexpr int QTILE = NCHUNK * QCHUNK;
+  static constexpr int STAGE = 2 * QTILE;   // Q, dO (swizzled, 1 KiB aligned)
+  static constexpr int SSTAGE = 2 * BM * 4;  // lse2, D of the same step
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KTILE;
+  static constexpr int OFF_ST = OFF_V + KTILE;
+  static constexpr int OFF_STAT = OFF_ST + ST * STAGE;
+  static constexpr int OFF_BAR = OFF_STAT + ST * SSTAGE;
+  static constexpr int NBAR = 1 + 2 * ST + 2 + 2 + 1 + 1;  // kv_full, q_full/q_empty, sp_full[2], ds_full[2], acc_done, drain
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int NWARPS = 6;
+  static constexpr int NTHREADS = 32 * NWARPS;
+  static constexpr int TMA_WARP = 4, MMA_WARP = 5;
+  // TMEM: dK [0, DV), dV [DV, 2DV), slot u: S^T at 2DV + u*2BM, dP^T at +BM
+  static constexpr int COL_DK = 0, COL_DV = DV, COL_SLOT = 2 * DV;
+  static constexpr int TMEM_USED = 2 * DV + 4 * BM;
+  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+  static_assert(TMEM_USED <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(STAGE % 1024 == 0, "stages stay 1 KiB aligned");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::NTHREADS, 1)
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                       const BwdParams p) {
+  constexpr int D = C::D, DV = C::DV, BM = C::BM, BN = C::BN, ST = C::ST, LA = C::LA;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = q_full + ST;
+  uint64_t* sp_full = q_empty + ST;  // [2]
+  uint64_t* ds_full = sp_full + 2;   // [2]
+  uint64_t* acc_done = ds_full + 2;
+  uint64_t* bar_drain = acc_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sSt = sbase + C::OFF_ST;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // ---- work unit: key tile j (heaviest first for causal), (b, hk), d slice
+  const int BHk = p.B * p.Hkv;
+  const int j = blockIdx.x / BHk;
+  const int bhk = blockIdx.x % BHk;
+  const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
+  const int dslice = blockIdx.y;  // which DV-wide slice of d
+  const int k0 = j * BN;
+  const int k1 = min(p.Nk - 1, k0 + BN - 1);
+  // queries that see some key of this tile: i in [q_lo(k0), q_hi(k1)]
+  const int delta = p.mask.delta();
+  int q_lo = (p.mask.wr < 0) ? 0 : k0 - delta - p.mask.wr;
+  int q_hi = (p.mask.wl < 0) ? p.Nq - 1 : k1 - delta + p.mask.wl;
+  q_lo = max(q_lo, 0);
+  q_hi = min(q_hi, p.Nq - 1);
+  const int i_begin = q_lo / BM;
+  const int n_qt = (q_hi >= q_lo) ? (q_hi / BM - i_begin + 1) : 0;
+  const int n_steps = n_qt * p.group;  // (query head in group) x (query tile)
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&sp_full[u], 1);
+      mbar_init(&ds_full[u], BN);
+    }
+    mbar_init(acc_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto step_head = [&](int step) { return hk * p.group + step / n_qt; };
+  auto step_q0 = [&](int step) { return (i_begin + step % n_qt) * BM; };
+
+  if (warp == C::TMA_WARP) {
+    if (lane == 0 && n_steps > 0) {
+      mbar_expect_tx(kv_full, 2 * C::KTILE);
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        tma_load_4d(sK + c * C::KCHUNK, &tm_k, kv_full, c * 64, hk, k0, b);
+        tma_load_4d(sV + c * C::KCHUNK, &tm_v, kv_full, c * 64, hk, k0, b);
+      }
+      int n_issued = 0;
+      for (int it = 0; it < n_steps; ++it) {
+        const int s = it % ST, use = it / ST;
+        if (use > 0 && !mbar_wait(&q_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
+          break;
+        const int hq = step_head(it), q0 = step_q0(it);
+        const uint32_t st = sSt + s * C::STAGE;
+        mbar_expect_tx(&q_full[s], C::STAGE + C::SSTAGE);
+        for (int c = 0; c < C::NCHUNK; ++c) {
+          tma_load_4d(st + c * C::QCHUNK, &tm_q, &q_full[s], c * 64, hq, q0, b);
+          tma_load_4d(st + C::QTILE + c * C::QCHUNK, &tm_do, &q_full[s], c * 64, hq, q0, b);
+        }
+        const size_t srow = (static_cast<size_t>(b) * p.Hq + hq) * p.Nq_pad + q0;
+        const uint32_t stat = sbase + C::OFF_STAT + s * C::SSTAGE;
+        bulk_load(stat, p.lse2 + srow, BM * 4, &q_full[s]);
+        bulk_load(stat + BM * 4, p.D + srow, BM * 4, &q_full[s]);
+        ++n_issued;
+      }
+      mbar_drain(kv_full, 0, p.wait_limit_ns);
+      for (int s = 0; s < ST; ++s)
+        if (n_issued > s) mbar_drain(&q_full[s], ((n_issued - 1 - s) / ST) & 1, p.wait_limit_ns);
+    }
+  } else if (warp == C::MMA_WARP) {
+    if (lane == 0 && n_steps > 0) {
+      constexpr uint32_t ID_S = idesc_bf16_f32(128, BM, false, false);
+      constexpr uint32_t ID_ACC = idesc_bf16_f32(128, DV, false, true);
+      auto wait = [&](uint64_t* bar, uint32_t par) {
+        const bool ok = mbar_wait(bar, par, abort_flag, &g_status, p.wait_limit_ns);
+        tc_fence_after();
+        return ok;
+      };
+      // slot u: S^T = K Q^T, dP^T = V dO^T (M = keys, N = queries)
+      auto issue_sdp = [&](int u, int s) {
+        const uint32_t d_s = tmem + C::COL_SLOT + u * 2 * BM, d_dp = d_s + BM;
+        const uint32_t st = sSt + s * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2), kb = (kk & 3) * 32;
+          const uint32_t kofs = ko * C::KCHUNK + kb, qofs = ko * C::QCHUNK + kb;
+          mma_ss(d_s, sdesc_sw128(sK + kofs, 16, 1024), sdesc_sw128(st + qofs, 16, 1024), ID_S, kk > 0);
+          mma_ss(d_dp, sdesc_sw128(sV + kofs, 16, 1024), sdesc_sw128(st + C::QTILE + qofs, 16, 1024),
+                 ID_S, kk > 0);
+        }
+      };
+      // dV += P^T dO, dK += dS^T Q (A from TMEM, B MN-major over this CTA's d slice)
+      auto issue_acc = [&](int u, int s, bool acc) {
+        const uint32_t a_p = tmem + C::COL_SLOT + u * 2 * BM, a_ds = a_p + BM;
+        const uint32_t st = sSt + s * C::STAGE + dslice * (DV / 64) * C::QCHUNK;
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint32_t acc_k = (acc || kk > 0) ? 1u : 0u;
+          mma_ts(tmem + C::COL_DV, a_p + kk * 8,
+                 sdesc_sw128(st + C::QTILE + kk * 2048, C::QCHUNK, 1024), ID_ACC, acc_k);
+          mma_ts(tmem + C::COL_DK, a_ds + kk * 8, sdesc_sw128(st + kk * 2048, C::QCHUNK, 1024), ID_ACC,
+                 acc_k);
+        }
+      };
+      bool ok = wait(kv_full, 0);
+      for (int u = 0; u < LA && u < n_steps && ok; ++u) {
+        if (!(ok = wait(&q_full[u % ST], (u / ST) & 1))) break;
+        issue_sdp(u & 1, u % ST);
+        tc_commit(&sp_full[u & 1]);
+      }
+      for (int it = 0; it < n_steps && ok; ++it) {
+        const int u = it & 1, s = it % ST;
+        if (!(ok = wait(&ds_full[u], (it >> 1) & 1))) break;
+        issue_acc(u, s, it > 0);
+        tc_commit(&q_empty[s]);
+        const int nx = it + LA;
+        if (nx < n_steps) {
+          if (!(ok = wait(&q_full[nx % ST], (nx / ST) & 1))) break;
+          issue_sdp(nx & 1, nx % ST);
+          tc_commit(&sp_full[nx & 1]);
+        }
+      }
+      if (ok) tc_commit(acc_done);
+    }
+    if (lane == 0) {
+      tc_commit(bar_drain);
+      mbar_drain(bar_drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ P^T / dS^T warpgroup (thread = key row)
+    const int r = threadIdx.x;  // 0..127 == TMEM lane == key within the tile
+    const int key = k0 + r;
+    // queries that see this key: [kq_lo, kq_hi]
+    const int kq_lo = (p.mask.wr < 0) ? -0x3fffffff : key - delta - p.mask.wr;
+    const int kq_hi = (p.mask.wl < 0) ? 0x3fffffff : key - delta + p.mask.wl;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < n_steps; ++it) {
+      const int u = it & 1, s = it % ST;
+      ok = mbar_wait(&sp_full[u], (it >> 1) & 1, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      // the stage's lse2 / D landed with the same barrier the MMA already waited on
+      ok = mbar_wait(&q_full[s], (it / ST) & 1, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t col_s = C::COL_SLOT + u * 2 * BM, col_dp = col_s + BM;
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::OFF_STAT + s * C::SSTAGE);
+      const float* Dv = lse2 + BM;
+      const int q0 = step_q0(it);
+      const bool need_mask = (q0 < kq_lo) || (q0 + BM - 1 > kq_hi);
+#pragma unroll 1
+      for (int cc = 0; cc < BM / 32; ++cc) {
+        uint32_t sv[32], dv[32];
+        tmem_ld_x32(lane_base + col_s + cc * 32, sv);
+        tmem_ld_x32(lane_base + col_dp + cc * 32, dv);
+        tmem_ld_wait_x32(sv);
+        tmem_ld_wait_x32(dv);
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float x0 = __uint_as_float(sv[c]), x1 = __uint_as_float(sv[c + 1]);
+          if (need_mask) {
+            const int qi = q0 + cc * 32 + c;
+            if (qi < kq_lo || qi > kq_hi) x0 = -INFINITY;
+            if (qi + 1 < kq_lo || qi + 1 > kq_hi) x1 = -INFINITY;
+          }
+          const float p0 = ex2_approx(fmaf(x0, sl2, -lse2[cc * 32 + c]));
+          const float p1 = ex2_approx(fmaf(x1, sl2, -lse2[cc * 32 + c + 1]));
+          pp[c / 2] = pack_bf16x2(p0, p1);
+          dd[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - Dv[cc * 32 + c]),
+                                  p1 * (__uint_as_float(dv[c + 1]) - Dv[cc * 32 + c + 1]));
+        }
+        tmem_st_x16(lane_base + col_s + cc * 16, pp);
+        tmem_st_x16(lane_base + col_dp + cc * 16, dd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ds_full[u]);
+    }
+    if (ok && n_steps > 0) {
+      ok = mbar_wait(acc_done, 0, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+    // epilogue: dK * scale, dV -> bf16 -> shared (the K and V buffers) -> TMA store
+    if (ok) {
+#pragma unroll 1
+      for (int w = 0; w < 2; ++w) {
+        const uint32_t col = (w == 0) ? C::COL_DK : C::COL_DV;
+        const uint32_t stage = (w == 0) ? sK : sV;
+        const float sc = (w == 0) ? p.scale : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < DV / 64; ++c) {
+          uint32_t ov[64];
+          if (n_steps > 0) {
+            tmem_ld_x32(lane_base + col + c * 64, ov);
+            tmem_ld_x32(lane_base + col + c * 64 + 32, ov + 32);
+            tmem_ld_wait_x32(ov);
+            tmem_ld_wait_x32(ov + 32);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) ov[i] = 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const float* f = reinterpret_cast<const float*>(ov + 8 * u);
+            st_shared_v4(stage + c * C::KCHUNK + sw128_offset(r, u), pack_bf16x2(f[0] * sc, f[1] * sc),
+                         pack_bf16x2(f[2] * sc, f[3] * sc), pack_bf16x2(f[4] * sc, f[5] * sc),
+                         pack_bf16x2(f[6] * sc, f[7] * sc));
+          }
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(1, 128);
+    if (r == 0 && *abort_flag == 0) {
+      for (int c = 0; c < DV / 64; ++c) {
+        const int x = (dslice * (DV / 64) + c) * 64;
+        tma_store_4d(&tm_dk, sK + c * C::KCHUNK, x, hk, k0, b);
+        tma_store_4d(&tm_dv, sV + c * C::KCHUNK, x, hk, k0, b);
+      }
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == C::MMA_WARP) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace fa

@@ -1,0 +1,402 @@
+// fa_fwd.cuh -- forward pass of exact attention on sm_100a.
+//
+// What it computes (hysenlabs FlashAttention API page, outputs section;
+// Qiita Flash Attention tutorial, sections 4.2-4.3; abeam.tech FlashAttention
+// summary, "computing softmax blockwise correctly"): for each query row,
+//   O = sum_j softmax_j(scale * q . k_j) v_j,   LSE = ln sum_j exp(scale * q . k_j)
+// by walking the visible key/value tiles once with a running row max m and a
+// running sum l; when m grows, l and the partial O are rescaled by
+// exp(m_old - m_new), and O is divided by l once at the end.  S and P live in
+// tensor memory and never reach HBM.
+//
+// Design on B200 (one CTA per SM, warp-specialised):
+//   * TMA warp      : Q tile(s) once, then K_j / V_j through a KST-deep ring.
+//   * MMA warp      : one thread issues tcgen05.mma: S = Q K_j^T (both operands
+//                     from shared memory, fp32 into TMEM) and O += P V_j (P
+//                     read straight from TMEM, V from shared memory).
+//   * softmax warps : one warpgroup per 128-row Q tile; thread r owns TMEM
+//                     lane r, i.e. a whole score row, so the row max and row
+//                     sum need no shuffles.  exp2 with the scale folded into
+//                     one FMA; P is written back into TMEM as bf16 over its S.
+// With two Q tiles per CTA (d <= 128) the tensor core computes one tile's
+// S/PV while the other tile's softmax runs.  For d = 256 (one Q tile) the two
+// S slots alternate between consecutive key tiles instead.
+//
+// The running max is only moved (and O rescaled) when the tile max exceeds
+// it by more than 2^8 in the exp2 domain; otherwise the old reference is kept.
+// Every P stays <= 2^8, the result is the same exact softmax (the reference
+// cancels in O / l), and most O rescales are skipped.
+#pragma once
+#include "fa_common.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  int B, Nq, Nk, Hq, Hkv, group;  // group = Hq / Hkv
+  float scale_log2;               // softmax scale * log2(e)
+  MaskSpec mask;
+  int n_qgroups;                  // CTAs along the query axis
+  float* lse;                     // [B, Hq, Nq]
+  unsigned long long wait_limit_ns;
+};
+
+template <int D_, int NQT_, int BN_, int KST_>
+struct FwdCfg {
+  static constexpr int D = D_, NQT = NQT_, BN = BN_, KST = KST_;
+  static constexpr int BM = 128;
+  static constexpr int NCHUNK = D / 64;      // 128-byte swizzle chunks across d
+  static constexpr int QCHUNK = BM * 128;    // bytes of one 64-column chunk of a Q tile
+  static constexpr int KCHUNK = BN * 128;
+  static constexpr int QTILE = NCHUNK * QCHUNK;
+  static constexpr int KTILE = NCHUNK * KCHUNK;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + NQT * QTILE;
+  static constexpr int OFF_V = OFF_K + KST * KTILE;
+  static constexpr int OFF_BAR = OFF_V + KST * KTILE;
+  static constexpr int NBAR = 1 + 4 * KST + 6 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KiB
+  static constexpr int NWARPS = 4 * NQT + 2;
+  static constexpr int NTHREADS = 32 * NWARPS;
+  static constexpr int TMA_WARP = 4 * NQT;
+  static constexpr int MMA_WARP = 4 * NQT + 1;
+  static constexpr int COL_S = 0;        // S slot s: columns [s*BN, s*BN+BN); its P: first BN/2
+  static constexpr int COL_O = 2 * BN;   // O of Q tile t: columns [COL_O + t*D, +D)
+  static constexpr int TMEM_USED = 2 * BN + NQT * D;
+  static constexpr int TMEM_COLS = TMEM_USED <= 128 ? 128 : TMEM_USED <= 256 ? 256 : 512;
+  static_assert(TMEM_USED <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(D % 64 == 0 && BN % 64 == 0, "tile shapes");
+  static_assert(NQT == 1 || NQT == 2, "one or two Q tiles per CTA");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::NTHREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const FwdParams p) {
+  constexpr int D = C::D, NQT = C::NQT, BN = C::BN, KST = C::KST, BM = C::BM;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* bar_q = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + KST;
+  uint64_t* s_full = v_empty + KST;  // [2]
+  uint64_t* p_full = s_full + 2;     // [2]
+  uint64_t* o_done = p_full + 2;     // [2]
+  uint64_t* bar_drain = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  const uint32_t sQ = sbase + C::OFF_Q, sK = sbase + C::OFF_K, sV = sbase + C::OFF_V;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  // ---- work unit: (query group g, batch b, head h); heaviest groups first
+  const int BH = p.B * p.Hq;
+  const int bh = blockIdx.x % BH;
+  const int g = p.n_qgroups - 1 - blockIdx.x / BH;
+  const int b = bh / p.Hq, h = bh % p.Hq, hk = h / p.group;
+  const int r0 = g * NQT * BM;
+  const int r_last = min(p.Nq - 1, r0 + NQT * BM - 1);
+  const int key_lo = p.mask.lo(r0), key_hi = p.mask.hi(r_last);
+  const int j_begin = key_lo / BN;
+  const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], BM);
+      mbar_init(&o_done[s], 1);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == C::TMA_WARP && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::TMA_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_kv > 0) {
+      mbar_expect_tx(bar_q, NQT * C::QTILE);
+      for (int t = 0; t < NQT; ++t)
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sQ + t * C::QTILE + c * C::QCHUNK, &tm_q, bar_q, c * 64, h, r0 + t * BM, b);
+      int nk = 0, nv = 0;
+      for (int it = 0; it < n_kv; ++it) {
+        const int s = it % KST, use = it / KST;
+        const int krow = (j_begin + it) * BN;
+        if (use > 0 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
+          break;
+        mbar_expect_tx(&k_full[s], C::KTILE);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[s], c * 64, hk, krow, b);
+        ++nk;
+        if (use > 0 && !mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
+          break;
+        mbar_expect_tx(&v_full[s], C::KTILE);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[s], c * 64, hk, krow, b);
+        ++nv;
+      }
+      // every copy issued must land before the CTA may exit
+      mbar_drain(bar_q, 0, p.wait_limit_ns);
+      for (int s = 0; s < KST; ++s) {
+        if (nk > s) mbar_drain(&k_full[s], ((nk - 1 - s) / KST) & 1, p.wait_limit_ns);
+        if (nv > s) mbar_drain(&v_full[s], ((nv - 1 - s) / KST) & 1, p.wait_limit_ns);
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_kv > 0) {
+      constexpr uint32_t ID_QK = idesc_bf16_f32(128, BN, false, false);
+      constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
+      auto wait = [&](uint64_t* bar, uint32_t par) {
+        const bool ok = mbar_wait(bar, par, abort_flag, &g_status, p.wait_limit_ns);
+        tc_fence_after();
+        return ok;
+      };
+      // S[slot] = Q_t K_s^T
+      auto issue_s = [&](int slot, int t, int s) {
+        const uint32_t d_tmem = tmem + C::COL_S + slot * BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk >> 2), kb = (kk & 3) * 32;
+          mma_ss(d_tmem, sdesc_sw128(sQ + t * C::QTILE + ko * C::QCHUNK + kb, 16, 1024),
+                 sdesc_sw128(sK + s * C::KTILE + ko * C::KCHUNK + kb, 16, 1024), ID_QK, kk > 0);
+        }
+      };
+      // O_t (+)= P[slot] V_s
+      auto issue_pv = [&](int slot, int t, int s, bool acc) {
+        const uint32_t d_tmem = tmem + C::COL_O + t * D;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(d_tmem, tmem + C::COL_S + slot * BN + kk * 8,
+                 sdesc_sw128(sV + s * C::KTILE + kk * 2048, C::KCHUNK, 1024), ID_PV,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
+      if (ok) {
+        if constexpr (NQT == 2) {
+          issue_s(0, 0, 0);
+          tc_commit(&s_full[0]);
+          issue_s(1, 1, 0);
+          tc_commit(&s_full[1]);
+          tc_commit(&k_empty[0]);
+          for (int it = 0; it < n_kv && ok; ++it) {
+            const int s = it % KST;
+            const int s1 = (it + 1) % KST;
+            if (!(ok = wait(&v_full[s], (it / KST) & 1))) break;
+            for (int t = 0; t < 2 && ok; ++t) {
+              if (!(ok = wait(&p_full[t], it & 1))) break;
+              issue_pv(t, t, s, it > 0);
+              tc_commit(&o_done[t]);
+              if (t == 1) tc_commit(&v_empty[s]);
+              if (it + 1 < n_kv) {
+                if (t == 0 && !(ok = wait(&k_full[s1], ((it + 1) / KST) & 1))) break;
+                issue_s(t, t, s1);
+                tc_commit(&s_full[t]);
+                if (t == 1) tc_commit(&k_empty[s1]);
+              }
+            }
+          }
+        } else {
+          // one Q tile: S slots alternate between consecutive key tiles
+          issue_s(0, 0, 0);
+          tc_commit(&s_full[0]);
+          tc_commit(&k_empty[0]);
+          if (n_kv > 1) {
+            if ((ok = wait(&k_full[1 % KST], (1 / KST) & 1))) {
+              issue_s(1, 0, 1 % KST);
+              tc_commit(&s_full[1]);
+              tc_commit(&k_empty[1 % KST]);
+            }
+          }
+          for (int it = 0; it < n_kv && ok; ++it) {
+            const int slot = it & 1, s = it % KST;
+            if (!(ok = wait(&v_full[s], (it / KST) & 1))) break;
+            if (!(ok = wait(&p_full[slot], (it >> 1) & 1))) break;
+            issue_pv(slot, 0, s, it > 0);
+            tc_commit(&o_done[0]);
+            tc_commit(&v_empty[s]);
+            if (it + 2 < n_kv) {
+              const int s2 = (it + 2) % KST;
+              if (!(ok = wait(&k_full[s2], ((it + 2) / KST) & 1))) break;
+              issue_s(slot, 0, s2);
+              tc_commit(&s_full[slot]);
+              tc_commit(&k_empty[s2]);
+            }
+          }
+        }
+      }
+    }
+    if (lane == 0) {  // all MMAs this thread issued are complete before TMEM is released
+      tc_commit(bar_drain);
+      mbar_drain(bar_drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = warp / 4;          // Q tile of this warpgroup
+    const int r = threadIdx.x % BM;  // row within the tile == TMEM lane
+    const int row = r0 + t * BM + r;
+    const int lo = p.mask.lo(row), hi = p.mask.hi(row);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    const float sl2 = p.scale_log2;
+    float m_ref = -INFINITY;  // reference max, exp2 domain (scale folded in)
+    float l = 0.f;
+    bool ok = true;
+    for (int it = 0; it < n_kv; ++it) {
+      const int slot = (NQT == 2) ? t : (it & 1);
+      const uint32_t par = (NQT == 2) ? (it & 1) : ((it >> 1) & 1);
+      ok = mbar_wait(&s_full[slot], par, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t col_s = C::COL_S + slot * BN;
+      uint32_t sv[BN];
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) tmem_ld_x32(lane_base + col_s + cc * 32, &sv[cc * 32]);
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) tmem_ld_wait_x32(&sv[cc * 32]);
+      float* sc = reinterpret_cast<float*>(sv);
+      const int k0 = (j_begin + it) * BN;
+      if (k0 < lo || k0 + BN - 1 > hi) {
+#pragma unroll
+        for (int c = 0; c < BN; ++c) {
+          const int key = k0 + c;
+          if (key < lo || key > hi) sc[c] = -INFINITY;
+        }
+      }
+      float mx0 = sc[0], mx1 = sc[1], mx2 = sc[2], mx3 = sc[3];
+#pragma unroll
+      for (int c = 4; c < BN; c += 4) {
+        mx0 = fmaxf(mx0, sc[c]);
+        mx1 = fmaxf(mx1, sc[c + 1]);
+        mx2 = fmaxf(mx2, sc[c + 2]);
+        mx3 = fmaxf(mx3, sc[c + 3]);
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_new = fmaxf(m_ref, m_tile);
+      const bool grow = m_new > m_ref + 8.0f;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = ex2_approx(m_ref - m_new);
+        m_ref = m_new;
+      }
+      const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
+      uint32_t pk[BN / 2];
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) {
+        const float p0 = ex2_approx(fmaf(sc[c], sl2, -mb));
+        const float p1 = ex2_approx(fmaf(sc[c + 1], sl2, -mb));
+        rs0 += p0;
+        rs1 += p1;
+        pk[c / 2] = pack_bf16x2(p0, p1);
+      }
+      l = l * alpha + (rs0 + rs1);
+#pragma unroll
+      for (int cc = 0; cc < BN / 64; ++cc) tmem_st_x32(lane_base + col_s + cc * 32, &pk[cc * 32]);
+      if (it > 0 && __any_sync(0xffffffffu, grow)) {
+        if constexpr (NQT == 1) {
+          // O must hold PV of the previous key tile before it is rescaled
+          ok = mbar_wait(&o_done[0], (it - 1) & 1, abort_flag, &g_status, p.wait_limit_ns);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        const uint32_t col_o = C::COL_O + t * D;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t ov[32];
+          tmem_ld_x32(lane_base + col_o + cc * 32, ov);
+          tmem_ld_wait_x32(ov);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st_x32(lane_base + col_o + cc * 32, ov);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[slot]);
+    }
+    // ---- epilogue: O / l -> bf16 -> shared (reusing this tile's Q buffer) -> TMA store
+    if (ok && n_kv > 0) {
+      ok = mbar_wait(&o_done[NQT == 2 ? t : 0], (n_kv - 1) & 1, abort_flag, &g_status,
+                     p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+    const uint32_t sQt = sQ + t * C::QTILE;
+    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+    if (ok) {
+#pragma unroll 1
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        uint32_t ov[64];
+        if (n_kv > 0) {
+          tmem_ld_x32(lane_base + C::COL_O + t * D + c * 64, ov);
+          tmem_ld_x32(lane_base + C::COL_O + t * D + c * 64 + 32, ov + 32);
+          tmem_ld_wait_x32(ov);
+          tmem_ld_wait_x32(ov + 32);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) ov[i] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float* f = reinterpret_cast<const float*>(ov + 8 * u);
+          st_shared_v4(sQt + c * C::QCHUNK + sw128_offset(r, u),
+                       pack_bf16x2(f[0] * inv_l, f[1] * inv_l), pack_bf16x2(f[2] * inv_l, f[3] * inv_l),
+                       pack_bf16x2(f[4] * inv_l, f[5] * inv_l), pack_bf16x2(f[6] * inv_l, f[7] * inv_l));
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(1 + t, BM);
+    const bool aborted = *abort_flag != 0;
+    if (r == 0 && !aborted && r0 + t * BM < p.Nq) {
+      for (int c = 0; c < C::NCHUNK; ++c)
+        tma_store_4d(&tm_o, sQt + c * C::QCHUNK, c * 64, h, r0 + t * BM, b);
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+    if (!aborted && row < p.Nq) {
+      const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
+      p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Nq + row] =
+          (l > 0.f) ? (mb + log2f(l)) * kLn2 : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == C::MMA_WARP) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace fa

@@ -1,0 +1,151 @@
+/*
+ * fa.h -- C ABI of libfa: exact IO-aware scaled-dot-product attention for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (hysenlabs "FlashAttention: GPU-specific backends and the
+ * attention API", section on outputs and operations; Qiita Flash Attention
+ * tutorial, section 2.2):
+ *
+ *     O = softmax(Q K^T * scale) V
+ *
+ * computed by tiling with an online softmax so that the N x N score and
+ * probability matrices never reach device memory (Qiita tutorial, sections
+ * 4.2-4.3; abeam.tech FlashAttention summary, "computing softmax blockwise
+ * correctly" and "cutting memory traffic by tiling").  The forward pass also
+ * writes the per-row log-sum-exp; the backward pass recomputes P from it
+ * (abeam.tech summary, "backward uses recomputation").
+ *
+ * Tensor layout (row-major, last index contiguous, no padding):
+ *     q, o, dO, dq : [B, Nq, Hq,  d]
+ *     k, v, dk, dv : [B, Nk, Hkv, d]
+ *     lse          : [B, Hq, Nq]      fp32, natural log, scale included:
+ *                    lse[b,h,i] = ln sum_j exp(scale * q_i . k_j) over visible j
+ * bf16 entry points take and return __nv_bfloat16 data (passed as void*);
+ * the _f32 entry points take float data.  Accumulation is fp32 throughout.
+ *
+ * Masking (hysenlabs page, option list and changelog v2.1 / v2.3): with
+ * delta = Nk - Nq, key j is visible to query i iff
+ *     (wr < 0 || j <= i + delta + wr)  &&  (win_l < 0 || j >= i + delta - win_l)
+ * where wr = 0 when causal != 0 and wr = win_r otherwise.  Bounds are
+ * inclusive; a negative bound is unbounded.  The causal diagonal is aligned to
+ * the bottom-right corner when Nq != Nk.  A query row with no visible key gets
+ * O = 0, lse = -inf and zero gradients.
+ *
+ * MQA / GQA (hysenlabs page, option list): Hq must be divisible by Hkv; query
+ * head h reads key/value head h / (Hq / Hkv).
+ *
+ * Ownership and execution: the caller allocates and owns every buffer (device
+ * memory unless stated).  Calls are ordered on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and return without synchronising; the library
+ * allocates no device memory.  All pointers must be device pointers aligned to
+ * 16 bytes.  Argument errors are reported before anything is launched.  A
+ * kernel that gives up on a bounded wait records FA_ERR_TIMEOUT in a
+ * per-device status word that fa_get_device_status() reads.
+ *
+ * There is no CPU fallback: every entry point runs only its CUDA kernels.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fa_stream_t; /* same type as cudaStream_t */
+
+enum fa_status {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, Hq % Hkv != 0, non-finite scale */
+  FA_ERR_UNSUPPORTED = 2, /* head dim not in {64, 128, 256} (bf16) or > 256 (f32) */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
+  FA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than fa_bwd_workspace_size() */
+  FA_ERR_TIMEOUT = 5      /* a device-side bounded wait expired (see fa_get_device_status) */
+};
+
+/*
+ * Forward pass, bf16 in / bf16 out, fp32 accumulation.
+ *   q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] : inputs (bf16, device)
+ *   o [B,Nq,Hq,d]                   : output (bf16, device)
+ *   lse [B,Hq,Nq]                   : output (fp32, device)
+ *   d in {64, 128, 256}; scale is usually 1/sqrt(d).
+ * Returns FA_OK or an fa_status code.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+           int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+           fa_stream_t stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes: two fp32 arrays
+ * [B, Hq, Nq rounded up to 256], the row sums D = rowsum(dO * O) and the
+ * saved LSE in base 2.  Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int Nq, int Hq, int d);
+
+/*
+ * Backward pass, bf16, fp32 accumulation, deterministic (the same inputs give
+ * the same bits on every call).
+ *   q, k, v, o, lse : the forward's inputs and outputs
+ *   dO [B,Nq,Hq,d]  : gradient of the loss with respect to o (bf16)
+ *   dq [B,Nq,Hq,d], dk/dv [B,Nk,Hkv,d] : outputs (bf16); dk and dv are summed
+ *                     over the Hq/Hkv query heads that share a key/value head
+ *   workspace       : device buffer of at least fa_bwd_workspace_size() bytes,
+ *                     16-byte aligned, owned by the caller, contents ignored
+ * Gradients are those of sum(dO * O) with respect to q, k and v, with P
+ * recomputed from lse.  Returns FA_OK or an fa_status code.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
+           int d, float scale, int causal, int win_l, int win_r, void* workspace,
+           size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * fp32 variants for small problems (fp32 in, fp32 out, fp32 arithmetic on the
+ * CUDA cores).  Same arguments and semantics as fa_fwd / fa_bwd; d <= 256 and
+ * d a multiple of 32.
+ */
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B,
+               int Nq, int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l,
+               int win_r, fa_stream_t stream);
+int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, const float* lse,
+               const float* dO, float* dq, float* dk, float* dv, int B, int Nq, int Nk, int Hq,
+               int Hkv, int d, float scale, int causal, int win_l, int win_r, void* workspace,
+               size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of
+ * the current device: FA_OK, FA_ERR_TIMEOUT if a kernel gave up on a bounded
+ * wait since the last call, or FA_ERR_CUDA if the synchronisation failed.
+ */
+int fa_get_device_status(fa_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(int status);
+
+/*
+ * Kernel tracing.  While enabled, every kernel the library launches is
+ * bracketed by two CUDA events recorded on the caller's stream (events come
+ * from a pool created when tracing is switched on; no device memory is
+ * allocated).  fa_trace_read() waits for the recorded events, adds each
+ * launch's device time to ms[kind] and one to launches[kind] for the
+ * FA_KERNEL_KINDS kinds below (both arrays are caller-owned host memory of
+ * FA_KERNEL_KINDS entries, zeroed by the library), then forgets the records.
+ * Returns FA_OK, FA_ERR_INVALID_ARG (null array) or FA_ERR_CUDA.
+ */
+enum fa_kernel_kind {
+  FA_KERNEL_FWD = 0,      /* forward, bf16 (tcgen05) */
+  FA_KERNEL_BWD_PREP = 1, /* backward preprocess D = rowsum(dO * O) */
+  FA_KERNEL_BWD_DQ = 2,   /* backward dQ, bf16 (tcgen05) */
+  FA_KERNEL_BWD_DKDV = 3, /* backward dK/dV, bf16 (tcgen05) */
+  FA_KERNEL_F32 = 4,      /* any fp32-path kernel */
+  FA_KERNEL_KINDS = 5
+};
+int fa_trace_enable(int on);
+int fa_trace_read(double* ms, long long* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -33,7 +33,15 @@ def _load():
                                                   ctypes.c_double, i, i, i, i, i]
         lib.oracle_attn_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i,
                                         ctypes.c_double, i, i, i, i]
-        for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_blockwise, lib.oracle_attn_bwd):
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.oracle_attn_fwd_rows.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i,
+                                             ctypes.c_double, i, i, i, ip, i, i]
+        lib.oracle_attn_dq_rows.argtypes = [dp, dp, dp, dp, dp, i, i, i, i, i, i,
+                                            ctypes.c_double, i, i, i, ip, i, i]
+        lib.oracle_attn_dkdv_rows.argtypes = [dp, dp, dp, dp, dp, dp, i, i, i, i, i, i,
+                                              ctypes.c_double, i, i, i, ip, i, i]
+        for f in (lib.oracle_attn_fwd, lib.oracle_attn_fwd_blockwise, lib.oracle_attn_bwd,
+                  lib.oracle_attn_fwd_rows, lib.oracle_attn_dq_rows, lib.oracle_attn_dkdv_rows):
             f.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -119,6 +127,63 @@ def attn_bwd(q, k, v, dout, scale=None, causal=False, window=(-1, -1), nthreads=
     if rc != 0:
         raise RuntimeError("oracle_attn_bwd failed (%d)" % rc)
     return dq, dk, dv
+
+
+def _rows(rows):
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).ravel())
+    return r, r.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def attn_fwd_rows(q, k, v, rows, scale=None, causal=False, window=(-1, -1), nthreads=None):
+    """(O, LSE) for the listed absolute query rows only: O [B, n, Hq, d], LSE [B, Hq, n].
+    Each row is computed exactly as attn_fwd computes it."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    r, rp = _rows(rows)
+    o = np.empty((B, len(r), Hq, d), np.float64)
+    lse = np.empty((B, Hq, len(r)), np.float64)
+    rc = _load().oracle_attn_fwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Nq, Nk,
+                                      Hq, Hkv, d, scale, c, wl, wr, rp, len(r),
+                                      nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("oracle_attn_fwd_rows failed (%d)" % rc)
+    return o, lse
+
+
+def attn_dq_rows(q, k, v, dout, rows, scale=None, causal=False, window=(-1, -1), nthreads=None):
+    """dQ for the listed absolute query rows only: [B, n, Hq, d]."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    r, rp = _rows(rows)
+    dq = np.empty((B, len(r), Hq, d), np.float64)
+    rc = _load().oracle_attn_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), B, Nq, Nk,
+                                     Hq, Hkv, d, scale, c, wl, wr, rp, len(r),
+                                     nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("oracle_attn_dq_rows failed (%d)" % rc)
+    return dq
+
+
+def attn_dkdv_rows(q, k, v, dout, rows, scale=None, causal=False, window=(-1, -1),
+                   nthreads=None):
+    """(dK, dV) for the listed absolute key rows only: each [B, n, Hkv, d]."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    r, rp = _rows(rows)
+    dk = np.empty((B, len(r), Hkv, d), np.float64)
+    dv = np.empty((B, len(r), Hkv, d), np.float64)
+    rc = _load().oracle_attn_dkdv_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dk), _ptr(dv),
+                                       B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, rp, len(r),
+                                       nthreads or default_threads())
+    if rc != 0:
+        raise RuntimeError("oracle_attn_dkdv_rows failed (%d)" % rc)
+    return dk, dv
 
 
 def fwd_flops(B, Nq, Nk, Hq, d, causal):

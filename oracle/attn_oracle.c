@@ -363,3 +363,183 @@ int oracle_attn_bwd(const double* q, const double* k, const double* v,
   free(parts); free(th); free(tk);
   return rc;
 }
+
+/* ------------------------------------------------------ selected rows only */
+/*
+ * The same row-by-row definition as above, evaluated only for a list of
+ * absolute query rows (O, LSE, dQ) or key rows (dK, dV), so large problems can
+ * be checked on a sample.  Each selected row is computed exactly as in the
+ * full functions (same code path, same order), so a selected row equals the
+ * full function's row bit for bit.
+ *   o_rows  [B, nq, Hq, d], lse_rows [B, Hq, nq], dq_rows [B, nq, Hq, d]
+ *   dk_rows [B, nk, Hkv, d], dv_rows [B, nk, Hkv, d]
+ */
+typedef struct {
+  const oshape* s;
+  const double *q, *k, *v, *dout;
+  const int* qrows; int nq;
+  const int* krows; int nk;
+  double *o_rows, *lse_rows, *dq_rows;
+  double *dk_part, *dv_part; /* this thread's [B, nk, Hkv, d] accumulators */
+  long task_begin, task_end; /* flattened (b, h, i) over all Nq query rows */
+  int mode;                  /* 0: fwd rows, 1: dq rows, 2: dk/dv rows */
+  int failed;
+} rows_task;
+
+static void* rows_worker(void* arg) {
+  rows_task* t = (rows_task*)arg;
+  const oshape* s = t->s;
+  double* p = (double*)malloc(sizeof(double) * (size_t)s->Nk);
+  double* orow = (double*)malloc(sizeof(double) * (size_t)s->d);
+  if (!p || !orow) { free(p); free(orow); t->failed = 1; return NULL; }
+  for (long task = t->task_begin; task < t->task_end; ++task) {
+    long b, h, i, r = -1;
+    if (t->mode == 2) {
+      /* every query row (b, h, i) contributes to the selected key rows */
+      i = task % s->Nq; h = (task / s->Nq) % s->Hq; b = task / (s->Nq * s->Hq);
+    } else {
+      r = task % t->nq; h = (task / t->nq) % s->Hq; b = task / (t->nq * s->Hq);
+      i = t->qrows[r];
+    }
+    long hk = h / (s->Hq / s->Hkv);
+    if (t->mode == 0) {
+      double L = softmax_row(s, t->q, t->k, b, h, i, p);
+      double* oi = t->o_rows + ((b * t->nq + r) * s->Hq + h) * s->d;
+      for (long c = 0; c < s->d; ++c) oi[c] = 0.0;
+      for (long j = 0; j < s->Nk; ++j) {
+        if (p[j] == 0.0) continue;
+        const double* vj = krow(s, t->v, b, j, hk);
+        for (long c = 0; c < s->d; ++c) oi[c] += p[j] * vj[c];
+      }
+      t->lse_rows[(b * s->Hq + h) * t->nq + r] = L;
+      continue;
+    }
+    const double* qi = qrow(s, t->q, b, i, h);
+    const double* doi = qrow(s, t->dout, b, i, h);
+    if (t->mode == 2) {
+      /* skip query rows that see none of the selected keys */
+      int any = 0;
+      for (int kk = 0; kk < t->nk && !any; ++kk) any = visible(s, i, t->krows[kk]);
+      if (!any) continue;
+    }
+    double L = softmax_row(s, t->q, t->k, b, h, i, p);
+    double* dqi = (t->mode == 1) ? t->dq_rows + ((b * t->nq + r) * s->Hq + h) * s->d : NULL;
+    if (dqi) for (long c = 0; c < s->d; ++c) dqi[c] = 0.0;
+    if (L == -INFINITY) continue;
+    for (long c = 0; c < s->d; ++c) orow[c] = 0.0;
+    for (long j = 0; j < s->Nk; ++j) {
+      if (p[j] == 0.0) continue;
+      const double* vj = krow(s, t->v, b, j, hk);
+      for (long c = 0; c < s->d; ++c) orow[c] += p[j] * vj[c];
+    }
+    double D = 0.0;
+    for (long c = 0; c < s->d; ++c) D += doi[c] * orow[c];
+    if (t->mode == 1) {
+      for (long j = 0; j < s->Nk; ++j) {
+        if (p[j] == 0.0) continue;
+        const double* vj = krow(s, t->v, b, j, hk);
+        const double* kj = krow(s, t->k, b, j, hk);
+        double dP = 0.0;
+        for (long c = 0; c < s->d; ++c) dP += doi[c] * vj[c];
+        double dS = p[j] * (dP - D);
+        for (long c = 0; c < s->d; ++c) dqi[c] += s->scale * dS * kj[c];
+      }
+    } else {
+      for (int kk = 0; kk < t->nk; ++kk) {
+        long j = t->krows[kk];
+        if (p[j] == 0.0) continue;
+        const double* vj = krow(s, t->v, b, j, hk);
+        double dP = 0.0;
+        for (long c = 0; c < s->d; ++c) dP += doi[c] * vj[c];
+        double dS = p[j] * (dP - D);
+        double* dkj = t->dk_part + ((b * t->nk + kk) * s->Hkv + hk) * s->d;
+        double* dvj = t->dv_part + ((b * t->nk + kk) * s->Hkv + hk) * s->d;
+        for (long c = 0; c < s->d; ++c) {
+          dkj[c] += s->scale * dS * qi[c];
+          dvj[c] += p[j] * doi[c];
+        }
+      }
+    }
+  }
+  free(p); free(orow);
+  return NULL;
+}
+
+static int run_rows(const double* q, const double* k, const double* v, const double* dout,
+                    double* o_rows, double* lse_rows, double* dq_rows, double* dk_rows,
+                    double* dv_rows, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+                    double scale, int causal, int win_l, int win_r, const int* qrows,
+                    int nq, const int* krows, int nk, int mode, int nthreads) {
+  if (bad_shape(B, Nq, Nk, Hq, Hkv, d)) return 1;
+  oshape s;
+  make_shape(&s, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r);
+  for (int r = 0; r < nq; ++r) if (qrows[r] < 0 || qrows[r] >= Nq) return 1;
+  for (int r = 0; r < nk; ++r) if (krows[r] < 0 || krows[r] >= Nk) return 1;
+  long tasks = (mode == 2) ? s.B * s.Hq * s.Nq : s.B * s.Hq * (long)nq;
+  if (tasks == 0) return 0;
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > tasks) nthreads = (int)tasks;
+  size_t kslice = (size_t)B * (size_t)nk * (size_t)Hkv * (size_t)d;
+  double* parts = NULL;
+  if (mode == 2) {
+    parts = (double*)calloc(kslice * 2 * (size_t)nthreads + 1, sizeof(double));
+    if (!parts) return 2;
+  }
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  rows_task* tk = (rows_task*)malloc(sizeof(rows_task) * (size_t)nthreads);
+  if (!th || !tk) { free(th); free(tk); free(parts); return 2; }
+  for (int t = 0; t < nthreads; ++t) {
+    rows_task* x = &tk[t];
+    x->s = &s; x->q = q; x->k = k; x->v = v; x->dout = dout;
+    x->qrows = qrows; x->nq = nq; x->krows = krows; x->nk = nk;
+    x->o_rows = o_rows; x->lse_rows = lse_rows; x->dq_rows = dq_rows;
+    x->dk_part = parts ? parts + kslice * 2 * (size_t)t : NULL;
+    x->dv_part = parts ? parts + kslice * (2 * (size_t)t + 1) : NULL;
+    x->task_begin = tasks * t / nthreads;
+    x->task_end = tasks * (t + 1) / nthreads;
+    x->mode = mode; x->failed = 0;
+    pthread_create(&th[t], NULL, rows_worker, x);
+  }
+  int rc = 0;
+  for (int t = 0; t < nthreads; ++t) {
+    pthread_join(th[t], NULL);
+    if (tk[t].failed) rc = 2;
+  }
+  if (mode == 2 && rc == 0) {
+    for (size_t e = 0; e < kslice; ++e) { dk_rows[e] = 0.0; dv_rows[e] = 0.0; }
+    for (int t = 0; t < nthreads; ++t)
+      for (size_t e = 0; e < kslice; ++e) {
+        dk_rows[e] += parts[kslice * 2 * (size_t)t + e];
+        dv_rows[e] += parts[kslice * (2 * (size_t)t + 1) + e];
+      }
+  }
+  free(th); free(tk); free(parts);
+  return rc;
+}
+
+int oracle_attn_fwd_rows(const double* q, const double* k, const double* v, double* o_rows,
+                         double* lse_rows, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+                         double scale, int causal, int win_l, int win_r, const int* rows,
+                         int nrows, int nthreads) {
+  if (!q || !k || !v || !o_rows || !lse_rows || !rows) return 1;
+  return run_rows(q, k, v, NULL, o_rows, lse_rows, NULL, NULL, NULL, B, Nq, Nk, Hq, Hkv, d,
+                  scale, causal, win_l, win_r, rows, nrows, NULL, 0, 0, nthreads);
+}
+
+int oracle_attn_dq_rows(const double* q, const double* k, const double* v, const double* dout,
+                        double* dq_rows, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+                        double scale, int causal, int win_l, int win_r, const int* rows,
+                        int nrows, int nthreads) {
+  if (!q || !k || !v || !dout || !dq_rows || !rows) return 1;
+  return run_rows(q, k, v, dout, NULL, NULL, dq_rows, NULL, NULL, B, Nq, Nk, Hq, Hkv, d,
+                  scale, causal, win_l, win_r, rows, nrows, NULL, 0, 1, nthreads);
+}
+
+int oracle_attn_dkdv_rows(const double* q, const double* k, const double* v, const double* dout,
+                          double* dk_rows, double* dv_rows, int B, int Nq, int Nk, int Hq,
+                          int Hkv, int d, double scale, int causal, int win_l, int win_r,
+                          const int* krows, int nkrows, int nthreads) {
+  if (!q || !k || !v || !dout || !dk_rows || !dv_rows || !krows) return 1;
+  return run_rows(q, k, v, dout, NULL, NULL, NULL, dk_rows, dv_rows, B, Nq, Nk, Hq, Hkv, d,
+                  scale, causal, win_l, win_r, NULL, 0, krows, nkrows, 2, nthreads);
+}

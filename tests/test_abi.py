@@ -1,0 +1,115 @@
+"""CPU-side checks of the C ABI: the library loads, exports every entry point
+include/fa.h declares, and rejects bad arguments with the documented status
+codes before anything reaches the GPU (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_io_aware_89_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced on these paths
+MISALIGNED = 0x10008
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_expected_entry_points():
+    assert declared_functions() == sorted([
+        "fa_fwd", "fa_bwd", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
+        "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fa.library_path())
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert hasattr(fa, name), name
+
+
+def test_status_strings():
+    names = ["FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA",
+             "FA_ERR_WORKSPACE", "FA_ERR_TIMEOUT"]
+    for code, name in enumerate(names):
+        assert fa.fa_status_string(code) == name
+    assert fa.fa_status_string(99) == "FA_UNKNOWN_STATUS"
+    header = open(HEADER).read()
+    for code, name in enumerate(names):
+        assert re.search(r"\b%s\s*=\s*%d\b" % (name, code), header), name
+
+
+def test_workspace_size():
+    # D and lse2 rows, fp32, rows padded to a multiple of 256
+    assert fa.fa_bwd_workspace_size(2, 2048, 16, 128) == 2 * 2 * 16 * 2048 * 4
+    assert fa.fa_bwd_workspace_size(1, 1, 1, 64) == 2 * 256 * 4
+    assert fa.fa_bwd_workspace_size(1, 257, 3, 64) == 2 * 3 * 512 * 4
+    assert fa.fa_bwd_workspace_size(0, 128, 2, 64) == 0
+    assert fa.fa_bwd_workspace_size(1, 0, 2, 64) == 0
+
+
+def _fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Nq=128, Nk=128, Hq=2, Hkv=2, d=64,
+             scale=0.125, causal=0, win_l=-1, win_r=-1, stream=None)
+    a.update(kw)
+    return fa.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Nq"], a["Nk"], a["Hq"],
+                     a["Hkv"], a["d"], a["scale"], a["causal"], a["win_l"], a["win_r"], a["stream"])
+
+
+def _bwd(f32=False, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dO=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1,
+             Nq=128, Nk=128, Hq=2, Hkv=2, d=64, scale=0.125, causal=0, win_l=-1, win_r=-1,
+             ws=FAKE, wsb=1 << 20, stream=None)
+    a.update(kw)
+    fn = fa.fa_bwd_f32 if f32 else fa.fa_bwd
+    return fn(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dO"], a["dq"], a["dk"], a["dv"], a["B"],
+              a["Nq"], a["Nk"], a["Hq"], a["Hkv"], a["d"], a["scale"], a["causal"], a["win_l"],
+              a["win_r"], a["ws"], a["wsb"], a["stream"])
+
+
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 4
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=0), dict(k=0), dict(v=0), dict(o=0), dict(lse=0),
+    dict(q=MISALIGNED), dict(o=MISALIGNED),
+    dict(B=0), dict(Nq=0), dict(Nk=-1), dict(Hq=0), dict(Hkv=0),
+    dict(Hq=6, Hkv=4),                       # Hq % Hkv != 0
+    dict(scale=float("nan")), dict(scale=float("inf")), dict(scale=0.0), dict(scale=-1.0),
+])
+def test_fwd_rejects_invalid_arguments(kw):
+    assert _fwd(**kw) == INVALID
+
+
+@pytest.mark.parametrize("d", [0, 32, 96, 100, 192, 512])
+def test_fwd_rejects_unsupported_head_dim(d):
+    assert _fwd(d=d) == UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw", [dict(dO=0), dict(dq=MISALIGNED), dict(dk=0), dict(dv=0),
+                                dict(Hq=3, Hkv=2), dict(B=-2)])
+def test_bwd_rejects_invalid_arguments(kw):
+    assert _bwd(**kw) == INVALID
+    assert _bwd(f32=True, **kw) == INVALID
+
+
+def test_bwd_rejects_small_or_missing_workspace():
+    need = fa.fa_bwd_workspace_size(1, 128, 2, 64)
+    assert _bwd(wsb=need - 4) == WORKSPACE
+    assert _bwd(ws=0) == WORKSPACE
+    assert _bwd(ws=MISALIGNED, wsb=need) == WORKSPACE
+    assert _bwd(d=96) == UNSUPPORTED
+
+
+def test_f32_head_dim_limits():
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE)
+    for d in (16, 48, 288):
+        assert fa.fa_fwd_f32(a["q"], a["k"], a["v"], a["o"], a["lse"], 1, 8, 8, 1, 1, d, 0.1, 0, -1,
+                             -1, None) == UNSUPPORTED

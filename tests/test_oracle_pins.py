@@ -288,3 +288,25 @@ def test_thread_count_does_not_change_results():
     o1, _ = oracle.attn_fwd(q, k, v, nthreads=1)
     o2, _ = oracle.attn_fwd(q, k, v, nthreads=5)
     np.testing.assert_array_equal(o1, o2)
+
+
+# ------------------------------------------------------- selected-row oracle
+
+@pytest.mark.parametrize("causal,wl,wr", [(False, -1, -1), (True, -1, -1), (True, 3, -1)])
+def test_selected_rows_equal_full_functions(causal, wl, wr):
+    """The row-subset oracle (used to check large problems on a sample) returns
+    exactly the rows of the full functions, which the tests above pin."""
+    rng = np.random.default_rng(13)
+    q, k, v, do = (_rand(s, rng) for s in [(2, 11, 4, 5), (2, 14, 2, 5), (2, 14, 2, 5), (2, 11, 4, 5)])
+    kw = dict(scale=0.7, causal=causal, window=(wl, wr))
+    o, lse = oracle.attn_fwd(q, k, v, nthreads=3, **kw)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, nthreads=1, **kw)
+    rows = [0, 3, 10, 4]
+    o_r, lse_r = oracle.attn_fwd_rows(q, k, v, rows, nthreads=2, **kw)
+    np.testing.assert_array_equal(o_r, o[:, rows])
+    np.testing.assert_array_equal(lse_r, lse[:, :, rows])
+    np.testing.assert_array_equal(oracle.attn_dq_rows(q, k, v, do, rows, nthreads=2, **kw), dq[:, rows])
+    krows = [13, 0, 7]
+    dk_r, dv_r = oracle.attn_dkdv_rows(q, k, v, do, krows, nthreads=3, **kw)
+    np.testing.assert_allclose(dk_r, dk[:, krows], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(dv_r, dv[:, krows], rtol=1e-13, atol=1e-13)
