@@ -19,7 +19,7 @@ import os
 
 __all__ = [
     "FAError", "load_library", "library_path",
-    "fa_fwd", "fa_bwd", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
+    "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
     "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
     "KERNEL_KINDS", "attention_forward", "attention_backward",
 ]
@@ -58,6 +58,8 @@ def load_library():
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp]
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i,
                            vp, sz, vp]
+    lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i,
+                                   i, vp]
     lib.fa_fwd_f32.argtypes = lib.fa_fwd.argtypes
     lib.fa_bwd_f32.argtypes = lib.fa_bwd.argtypes
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
@@ -67,7 +69,8 @@ def load_library():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_trace_enable.argtypes = [i]
     lib.fa_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
-    for name in ("fa_fwd", "fa_bwd", "fa_fwd_f32", "fa_bwd_f32", "fa_get_device_status",
+    for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32",
+                 "fa_get_device_status",
                  "fa_trace_enable", "fa_trace_read"):
         getattr(lib, name).restype = i
     _lib = lib
@@ -85,6 +88,14 @@ def fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale, causal
            win_r, workspace, workspace_bytes, stream):
     return load_library().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale,
                                  causal, win_l, win_r, workspace, workspace_bytes, stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l,
+                   win_r, stream):
+    """fa_bwd for callers that cannot allocate device memory (no workspace
+    argument; the library's fixed scratch array is used instead)."""
+    return load_library().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d,
+                                         scale, causal, win_l, win_r, stream)
 
 
 def fa_fwd_f32(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, stream):

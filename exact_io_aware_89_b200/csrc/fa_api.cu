@@ -198,6 +198,34 @@ size_t workspace_bytes(int B, int Nq, int Hq) {
 
 }  // namespace
 
+// ------------------------------------------------- allocation-free backward
+// Scratch of fa_bwd_noalloc: the D and lse2 rows the backward preprocess
+// writes, held in a fixed array that is part of the library's device image
+// (every GPU that loads the library keeps these 16 MiB until the process
+// exits).  Host code must not hand the symbol itself to a kernel: on the host
+// it only names a stand-in, so the device address is looked up with
+// cudaGetSymbolAddress, once per device, with that device current.
+constexpr size_t kNoAllocScratchBytes = 16u << 20;
+static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_scratch_mu;
+float* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+int scratch_for_current_device(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    g_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_scratch_ptr[dev];
+  return FA_OK;
+}
+}  // namespace
+
 extern "C" {
 
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq, int Nk,
@@ -235,6 +263,34 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* ws = static_cast<float*>(workspace);
+  switch (d) {
+    case 64:
+      return launch_bwd<Dq64, Dkv64>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+    case 128:
+      return launch_bwd<Dq128, Dkv128>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+    default:
+      return launch_bwd<Dq256, Dkv256>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+  }
+}
+
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq,
+                   int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                   fa_stream_t stream) {
+  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (workspace_bytes(B, Nq, Hq) > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
+  float* ws = nullptr;
+  st = scratch_for_current_device(&ws);
+  if (st != FA_OK) return st;
+  // Every D / lse2 entry the kernels read is written by the preprocess kernel
+  // of the same call first, so nothing in the shared array needs clearing.
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (d) {
     case 64:
       return launch_bwd<Dq64, Dkv64>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);

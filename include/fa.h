@@ -101,6 +101,32 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
            size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_bwd without a workspace argument, for callers that cannot allocate
+ * device memory: code running inside a CUDA graph capture or a driver
+ * callback, an allocator-free runtime, or a host program with a fixed
+ * memory budget that has no cudaMalloc on its path.  The pages have no
+ * counterpart; it is an addition of this library.
+ *
+ * Same arguments, results and determinism as fa_bwd.  Its scratch (the
+ * 8 * B * Hq * ceil(Nq/256)*256 bytes fa_bwd_workspace_size() reports) lives in
+ * a fixed 16 MiB array inside the library's device image, so it handles
+ * problems with B * Hq * ceil(Nq / 256) * 256 <= 2097152 rows and returns
+ * FA_ERR_WORKSPACE, without launching anything, for larger ones.  The library
+ * calls no cudaMalloc/cudaFree and no allocating routine on this path.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call on a device shares the one array and
+ * overwrites it (nothing in it needs to start at zero): calls that can
+ * overlap on the GPU -- on different streams without ordering between them --
+ * race on it and must be serialised by the caller.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                   const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq,
+                   int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                   fa_stream_t stream);
+
+/*
  * fp32 variants for small problems (fp32 in, fp32 out, fp32 arithmetic on the
  * CUDA cores).  Same arguments and semantics as fa_fwd / fa_bwd; d <= 256 and
  * d a multiple of 32.

@@ -24,7 +24,7 @@ def declared_functions():
 
 def test_header_declares_the_expected_entry_points():
     assert declared_functions() == sorted([
-        "fa_fwd", "fa_bwd", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
+        "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
         "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
 
 
