@@ -390,9 +390,10 @@ struct DkvCfg {
   static constexpr int NBAR = 1 + 2 * ST + 2 + 2 + 1 + 1;  // kv_full, q_full/q_empty, sp_full[2], ds_full[2], acc_done, drain
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  static constexpr int NWARPS = 6;
+  // two P^T/dS^T warpgroups take alternate steps (one per TMEM slot)
+  static constexpr int NWARPS = 10;
   static constexpr int NTHREADS = 32 * NWARPS;
-  static constexpr int TMA_WARP = 4, MMA_WARP = 5;
+  static constexpr int TMA_WARP = 8, MMA_WARP = 9;
   // TMEM: dK [0, DV), dV [DV, 2DV), slot u: S^T at 2DV + u*2BM, dP^T at +BM
   static constexpr int COL_DK = 0, COL_DV = DV, COL_SLOT = 2 * DV;
   static constexpr int TMEM_USED = 2 * DV + 4 * BM;
@@ -561,8 +562,9 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------ P^T / dS^T warpgroup (thread = key row)
-    const int r = threadIdx.x;  // 0..127 == TMEM lane == key within the tile
+    // ------------------------------------------------ P^T / dS^T warpgroups (thread = key row)
+    const int wg = warp / 4;           // handles the steps of TMEM slot wg
+    const int r = threadIdx.x % 128;   // TMEM lane == key within the tile
     const int key = k0 + r;
     // queries that see this key: [kq_lo, kq_hi]
     const int kq_lo = (p.mask.wr < 0) ? -0x3fffffff : key - delta - p.mask.wr;
@@ -570,7 +572,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int it = 0; it < n_steps; ++it) {
+    for (int it = wg; it < n_steps; it += 2) {
       const int u = it & 1, s = it % ST;
       ok = mbar_wait(&sp_full[u], (it >> 1) & 1, abort_flag, &g_status, p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
@@ -619,13 +621,13 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
     }
-    // epilogue: dK * scale, dV -> bf16 -> shared (the K and V buffers) -> TMA store
+    // epilogue: warpgroup 0 stages dK * scale, warpgroup 1 stages dV, as bf16 in
+    // the K and V buffers; one thread then issues the TMA stores
     if (ok) {
-#pragma unroll 1
-      for (int w = 0; w < 2; ++w) {
-        const uint32_t col = (w == 0) ? C::COL_DK : C::COL_DV;
-        const uint32_t stage = (w == 0) ? sK : sV;
-        const float sc = (w == 0) ? p.scale : 1.f;
+      {
+        const uint32_t col = (wg == 0) ? C::COL_DK : C::COL_DV;
+        const uint32_t stage = (wg == 0) ? sK : sV;
+        const float sc = (wg == 0) ? p.scale : 1.f;
 #pragma unroll 1
         for (int c = 0; c < DV / 64; ++c) {
           uint32_t ov[64];
@@ -649,8 +651,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       }
       fence_proxy_async_smem();
     }
-    named_bar_sync(1, 128);
-    if (r == 0 && *abort_flag == 0) {
+    named_bar_sync(1, 256);
+    if (threadIdx.x == 0 && *abort_flag == 0) {
       for (int c = 0; c < DV / 64; ++c) {
         const int x = (dslice * (DV / 64) + c) * 64;
         tma_store_4d(&tm_dk, sK + c * C::KCHUNK, x, hk, k0, b);

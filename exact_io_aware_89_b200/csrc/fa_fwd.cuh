@@ -323,14 +323,19 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       l = l * alpha + (rs0 + rs1);
 #pragma unroll
       for (int cc = 0; cc < BN / 64; ++cc) tmem_st_x32(lane_base + col_s + cc * 32, &pk[cc * 32]);
-      if (it > 0 && __any_sync(0xffffffffu, grow)) {
-        if constexpr (NQT == 1) {
-          // O must hold PV of the previous key tile before it is rescaled
+      if constexpr (NQT == 1) {
+        // PV of the previous key tile must be complete before O is rescaled.
+        // The wait is taken at every step, not only when rescaling: a parity
+        // wait is only unambiguous while the barrier is at most one phase
+        // ahead of the waiter, and this keeps the waiter in lock step.
+        if (it > 0) {
           ok = mbar_wait(&o_done[0], (it - 1) & 1, abort_flag, &g_status, p.wait_limit_ns);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
         }
+      }
+      if (it > 0 && __any_sync(0xffffffffu, grow)) {
         const uint32_t col_o = C::COL_O + t * D;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
