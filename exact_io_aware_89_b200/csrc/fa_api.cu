@@ -68,7 +68,7 @@ using Dq128 = DqCfg<128, 2, 64, 2>;
 using Dq256 = DqCfg<256, 1, 64, 1>;
 // dK/dV: {d, accumulated d slice, query tile, Q/dO ring depth}
 using Dkv64 = DkvCfg<64, 64, 64, 4>;
-using Dkv128 = DkvCfg<128, 128, 64, 3>;
+using Dkv128 = DkvCfg<128, 128, 64, 4>;
 using Dkv256 = DkvCfg<256, 128, 64, 1>;
 
 constexpr int kMaxDevices = 64;
@@ -106,6 +106,18 @@ int check_common(const void* q, const void* k, const void* v, int B, int Nq, int
 
 int pad_rows(int Nq) { return (Nq + 255) / 256 * 256; }
 
+// Heads per scheduling chunk: at most as many as keep the streamed operands
+// of one chunk (bytes_per_head each) within a third of the B200's 126 MB L2,
+// then evened out so the last chunk is not a small tail.
+int head_chunk(int n_heads, long long bytes_per_head) {
+  constexpr long long kBudget = 42ll << 20;
+  long long c = bytes_per_head > 0 ? kBudget / bytes_per_head : n_heads;
+  if (c < 1) c = 1;
+  if (c > n_heads) c = n_heads;
+  const long long n_chunks = (n_heads + c - 1) / c;
+  return static_cast<int>((n_heads + n_chunks - 1) / n_chunks);
+}
+
 // ------------------------------------------------------------------ forward
 template <class C>
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
@@ -120,6 +132,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.scale_log2 = scale * kLog2e;
   p.mask = mask;
   p.n_qgroups = (Nq + C::NQT * C::BM - 1) / (C::NQT * C::BM);
+  p.head_chunk = head_chunk(B * Hq, 4ll * Nk * C::D);  // K and V of one head, bf16
   p.lse = lse;
   p.wait_limit_ns = kWaitLimitNs;
   auto kern = fa_fwd_kernel<C>;
@@ -160,6 +173,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.lse2 = ws + rows_pad;
   p.n_qgroups = (Nq + CQ::NQT * CQ::BM - 1) / (CQ::NQT * CQ::BM);
   p.n_kvtiles = (Nk + CKV::BN - 1) / CKV::BN;
+  p.head_chunk = head_chunk(B * Hq, 4ll * Nk * D);                  // K and V per query head
+  p.head_chunk_kv = head_chunk(B * Hkv, 4ll * Nq * D * (Hq / Hkv));  // Q and dO per key/value head
   p.wait_limit_ns = kWaitLimitNs;
   {
     CUtensorMap tq, tk, tv, tdo, tdq;

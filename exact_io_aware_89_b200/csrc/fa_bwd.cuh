@@ -91,6 +91,8 @@ struct BwdParams {
   const float* lse2;  // [B, Hq, Nq_pad]
   int n_qgroups;      // dq kernel: CTAs along the query axis
   int n_kvtiles;      // dkdv kernel: CTAs along the key axis
+  int head_chunk;     // dq kernel: heads per scheduling chunk
+  int head_chunk_kv;  // dkdv kernel: key/value heads per scheduling chunk
   unsigned long long wait_limit_ns;
 };
 
@@ -150,9 +152,10 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
                  sV = sbase + C::OFF_V;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  const int BH = p.B * p.Hq;
-  const int bh = blockIdx.x % BH;
-  const int g = p.n_qgroups - 1 - blockIdx.x / BH;
+  // heaviest query groups first within L2-sized chunks of heads
+  const ChunkedOrder order(blockIdx.x, p.B * p.Hq, p.n_qgroups, p.head_chunk);
+  const int bh = order.head;
+  const int g = p.n_qgroups - 1 - order.rank;
   const int b = bh / p.Hq, h = bh % p.Hq, hk = h / p.group;
   const int r0 = g * NQT * BM;
   const int r_last = min(p.Nq - 1, r0 + NQT * BM - 1);
@@ -218,26 +221,36 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
         tc_fence_after();
         return ok;
       };
+      // Descriptors are built once; each MMA adds a compile-time offset (in
+      // 16-byte units).  The issuing thread has to keep ahead of the tensor
+      // core, so it does little besides issuing.
+      const uint64_t dq_q = sdesc_sw128(sQ, 16, 1024), dq_do = sdesc_sw128(sdO, 16, 1024);
+      const uint64_t dq_k = sdesc_sw128(sK, 16, 1024), dq_v = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dq_kmn = sdesc_sw128(sK, C::KCHUNK, 1024);
       // S_t = Q_t K_s^T and dP_t = dO_t V_s^T
       auto issue_sdp = [&](int t, int s) {
         const uint32_t d_s = tmem + t * 2 * BN, d_dp = d_s + BN;
+        const uint64_t qa = dq_q + static_cast<uint64_t>((t * C::QTILE) >> 4);
+        const uint64_t da = dq_do + static_cast<uint64_t>((t * C::QTILE) >> 4);
+        const uint64_t kb = dq_k + static_cast<uint64_t>((s * C::KTILE) >> 4);
+        const uint64_t vb = dq_v + static_cast<uint64_t>((s * C::KTILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2), kb = (kk & 3) * 32;
-          const uint32_t qo = t * C::QTILE + ko * C::QCHUNK + kb;
-          const uint32_t ks = s * C::KTILE + ko * C::KCHUNK + kb;
-          mma_ss(d_s, sdesc_sw128(sQ + qo, 16, 1024), sdesc_sw128(sK + ks, 16, 1024), ID_S, kk > 0);
-          mma_ss(d_dp, sdesc_sw128(sdO + qo, 16, 1024), sdesc_sw128(sV + ks, 16, 1024), ID_S, kk > 0);
+          const uint32_t qo = ((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4;
+          const uint32_t ko = ((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4;
+          mma_ss(d_s, qa + qo, kb + ko, ID_S, kk > 0);
+          mma_ss(d_dp, da + qo, vb + ko, ID_S, kk > 0);
         }
       };
       // dQ_t (+)= dS_t K_s, dS from TMEM (bf16 over dP_t), K as MN-major B
       auto issue_dq = [&](int t, int s, bool acc) {
         const uint32_t d_dq = tmem + C::COL_DQ + t * D;
         const uint32_t a_ds = tmem + t * 2 * BN + BN;
+        const uint64_t kb = dq_kmn + static_cast<uint64_t>((s * C::KTILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(d_dq, a_ds + kk * 8, sdesc_sw128(sK + s * C::KTILE + kk * 2048, C::KCHUNK, 1024),
-                 ID_DQ, (acc || kk > 0) ? 1u : 0u);
+          mma_ts(d_dq, a_ds + kk * 8, kb + static_cast<uint64_t>(kk * 128), ID_DQ,
+                 (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = wait(q_full, 0) && wait(&kv_full[0], 0);
       if (ok) {
@@ -247,12 +260,16 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
         }
         for (int it = 0; it < n_kv && ok; ++it) {
           const int s = it % KST, s1 = (it + 1) % KST;
+          const bool more = it + 1 < n_kv;
           for (int t = 0; t < NQT && ok; ++t) {
             if (!(ok = wait(&ds_full[t], it & 1))) break;
+            // with two or more stages the next key tile's wait shares this
+            // wait point; with one stage it has to follow this tile's release
+            if (KST > 1 && t == 0 && more && !(ok = wait(&kv_full[s1], ((it + 1) / KST) & 1))) break;
             issue_dq(t, s, it > 0);
             if (t == NQT - 1) tc_commit(&kv_empty[s]);
-            if (it + 1 < n_kv) {
-              if (t == 0 && !(ok = wait(&kv_full[s1], ((it + 1) / KST) & 1))) break;
+            if (more) {
+              if (KST == 1 && t == 0 && !(ok = wait(&kv_full[s1], ((it + 1) / KST) & 1))) break;
               issue_sdp(t, s1);
               tc_commit(&sp_full[t]);
             }
@@ -427,10 +444,11 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sSt = sbase + C::OFF_ST;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // ---- work unit: key tile j (heaviest first for causal), (b, hk), d slice
-  const int BHk = p.B * p.Hkv;
-  const int j = blockIdx.x / BHk;
-  const int bhk = blockIdx.x % BHk;
+  // ---- work unit: (b, hk), key tile j, d slice: the heaviest key tiles (the
+  // earliest, for causal) first within L2-sized chunks of head groups
+  const ChunkedOrder order(blockIdx.x, p.B * p.Hkv, p.n_kvtiles, p.head_chunk_kv);
+  const int bhk = order.head;
+  const int j = order.rank;
   const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
   const int dslice = blockIdx.y;  // which DV-wide slice of d
   const int k0 = j * BN;
@@ -510,30 +528,33 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
         tc_fence_after();
         return ok;
       };
+      // Descriptors built once; each MMA adds a compile-time offset.
+      const uint64_t dk_k = sdesc_sw128(sK, 16, 1024), dk_v = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dk_st = sdesc_sw128(sSt, 16, 1024);                // Q / dO, K-major B
+      const uint64_t dk_stmn = sdesc_sw128(sSt + dslice * (DV / 64) * C::QCHUNK, C::QCHUNK, 1024);
       // slot u: S^T = K Q^T, dP^T = V dO^T (M = keys, N = queries)
       auto issue_sdp = [&](int u, int s) {
         const uint32_t d_s = tmem + C::COL_SLOT + u * 2 * BM, d_dp = d_s + BM;
-        const uint32_t st = sSt + s * C::STAGE;
+        const uint64_t qb = dk_st + static_cast<uint64_t>((s * C::STAGE) >> 4);
+        const uint64_t dob = qb + static_cast<uint64_t>(C::QTILE >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2), kb = (kk & 3) * 32;
-          const uint32_t kofs = ko * C::KCHUNK + kb, qofs = ko * C::QCHUNK + kb;
-          mma_ss(d_s, sdesc_sw128(sK + kofs, 16, 1024), sdesc_sw128(st + qofs, 16, 1024), ID_S, kk > 0);
-          mma_ss(d_dp, sdesc_sw128(sV + kofs, 16, 1024), sdesc_sw128(st + C::QTILE + qofs, 16, 1024),
-                 ID_S, kk > 0);
+          const uint32_t kofs = ((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4;
+          const uint32_t qofs = ((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4;
+          mma_ss(d_s, dk_k + kofs, qb + qofs, ID_S, kk > 0);
+          mma_ss(d_dp, dk_v + kofs, dob + qofs, ID_S, kk > 0);
         }
       };
       // dV += P^T dO, dK += dS^T Q (A from TMEM, B MN-major over this CTA's d slice)
       auto issue_acc = [&](int u, int s, bool acc) {
         const uint32_t a_p = tmem + C::COL_SLOT + u * 2 * BM, a_ds = a_p + BM;
-        const uint32_t st = sSt + s * C::STAGE + dslice * (DV / 64) * C::QCHUNK;
+        const uint64_t qb = dk_stmn + static_cast<uint64_t>((s * C::STAGE) >> 4);
+        const uint64_t dob = qb + static_cast<uint64_t>(C::QTILE >> 4);
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t acc_k = (acc || kk > 0) ? 1u : 0u;
-          mma_ts(tmem + C::COL_DV, a_p + kk * 8,
-                 sdesc_sw128(st + C::QTILE + kk * 2048, C::QCHUNK, 1024), ID_ACC, acc_k);
-          mma_ts(tmem + C::COL_DK, a_ds + kk * 8, sdesc_sw128(st + kk * 2048, C::QCHUNK, 1024), ID_ACC,
-                 acc_k);
+          mma_ts(tmem + C::COL_DV, a_p + kk * 8, dob + static_cast<uint64_t>(kk * 128), ID_ACC, acc_k);
+          mma_ts(tmem + C::COL_DK, a_ds + kk * 8, qb + static_cast<uint64_t>(kk * 128), ID_ACC, acc_k);
         }
       };
       bool ok = wait(kv_full, 0);
@@ -544,12 +565,14 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       }
       for (int it = 0; it < n_steps && ok; ++it) {
         const int u = it & 1, s = it % ST;
+        const int nx = it + LA;
         if (!(ok = wait(&ds_full[u], (it >> 1) & 1))) break;
+        // with a deep enough ring the next step's operands share this wait point
+        if (nx < n_steps && LA < ST && !(ok = wait(&q_full[nx % ST], (nx / ST) & 1))) break;
         issue_acc(u, s, it > 0);
         tc_commit(&q_empty[s]);
-        const int nx = it + LA;
         if (nx < n_steps) {
-          if (!(ok = wait(&q_full[nx % ST], (nx / ST) & 1))) break;
+          if (LA >= ST && !(ok = wait(&q_full[nx % ST], (nx / ST) & 1))) break;
           issue_sdp(nx & 1, nx % ST);
           tc_commit(&sp_full[nx & 1]);
         }
@@ -587,30 +610,45 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       const float* Dv = lse2 + BM;
       const int q0 = step_q0(it);
       const bool need_mask = (q0 < kq_lo) || (q0 + BM - 1 > kq_hi);
-#pragma unroll 1
-      for (int cc = 0; cc < BM / 32; ++cc) {
-        uint32_t sv[32], dv[32];
-        tmem_ld_x32(lane_base + col_s + cc * 32, sv);
-        tmem_ld_x32(lane_base + col_dp + cc * 32, dv);
-        tmem_ld_wait_x32(sv);
-        tmem_ld_wait_x32(dv);
-        uint32_t pp[16], dd[16];
+      // all of this step's S^T and dP^T columns come in with one wait
+      uint32_t sv[BM], dv[BM];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float x0 = __uint_as_float(sv[c]), x1 = __uint_as_float(sv[c + 1]);
-          if (need_mask) {
-            const int qi = q0 + cc * 32 + c;
-            if (qi < kq_lo || qi > kq_hi) x0 = -INFINITY;
-            if (qi + 1 < kq_lo || qi + 1 > kq_hi) x1 = -INFINITY;
-          }
-          const float p0 = ex2_approx(fmaf(x0, sl2, -lse2[cc * 32 + c]));
-          const float p1 = ex2_approx(fmaf(x1, sl2, -lse2[cc * 32 + c + 1]));
-          pp[c / 2] = pack_bf16x2(p0, p1);
-          dd[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - Dv[cc * 32 + c]),
-                                  p1 * (__uint_as_float(dv[c + 1]) - Dv[cc * 32 + c + 1]));
+      for (int cc = 0; cc < BM / 32; ++cc) {
+        tmem_ld_x32(lane_base + col_s + cc * 32, &sv[cc * 32]);
+        tmem_ld_x32(lane_base + col_dp + cc * 32, &dv[cc * 32]);
+      }
+#pragma unroll
+      for (int cc = 0; cc < BM / 32; ++cc) {
+        tmem_ld_wait_x32(&sv[cc * 32]);
+        tmem_ld_wait_x32(&dv[cc * 32]);
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < BM; ++c) {
+          const int qi = q0 + c;
+          if (qi < kq_lo || qi > kq_hi) sv[c] = __float_as_uint(-INFINITY);
         }
-        tmem_st_x16(lane_base + col_s + cc * 16, pp);
-        tmem_st_x16(lane_base + col_dp + cc * 16, dd);
+      }
+      const float4* lse4 = reinterpret_cast<const float4*>(lse2);
+      const float4* d4 = reinterpret_cast<const float4*>(Dv);
+      uint32_t pp[BM / 2], dd[BM / 2];
+#pragma unroll
+      for (int c = 0; c < BM; c += 4) {
+        const float4 l4 = lse4[c / 4], D4 = d4[c / 4];
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -l4.x));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -l4.y));
+        const float p2 = ex2_approx(fmaf(__uint_as_float(sv[c + 2]), sl2, -l4.z));
+        const float p3 = ex2_approx(fmaf(__uint_as_float(sv[c + 3]), sl2, -l4.w));
+        pp[c / 2] = pack_bf16x2(p0, p1);
+        pp[c / 2 + 1] = pack_bf16x2(p2, p3);
+        dd[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - D4.x), p1 * (__uint_as_float(dv[c + 1]) - D4.y));
+        dd[c / 2 + 1] =
+            pack_bf16x2(p2 * (__uint_as_float(dv[c + 2]) - D4.z), p3 * (__uint_as_float(dv[c + 3]) - D4.w));
+      }
+#pragma unroll
+      for (int cc = 0; cc < BM / 32; ++cc) {
+        tmem_st_x16(lane_base + col_s + cc * 16, &pp[cc * 16]);
+        tmem_st_x16(lane_base + col_dp + cc * 16, &dd[cc * 16]);
       }
       tmem_st_wait();
       tc_fence_before();

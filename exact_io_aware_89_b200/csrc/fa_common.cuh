@@ -34,6 +34,28 @@ struct MaskSpec {
   }
 };
 
+// Maps a linear CTA index to (head, work index within the head), where the
+// work index is ordered heaviest first.  Heads are taken in chunks of
+// `chunk` (sized on the host so one chunk's K/V fits comfortably in L2);
+// inside a chunk the order is heaviest-first across all its heads, which
+// balances causal work like a longest-first schedule, while the CTAs resident
+// together only touch one chunk's K/V.
+struct ChunkedOrder {
+  int head, rank;  // rank 0 = heaviest work unit of the head
+  __device__ __forceinline__ ChunkedOrder(int L, int n_heads, int per_head, int chunk) {
+    const int full = n_heads / chunk;
+    const int span = chunk * per_head;
+    int c = L / span, idx = L - c * span, ce = chunk;
+    if (c >= full) {  // the last, partial chunk
+      c = full;
+      idx = L - full * span;
+      ce = n_heads - full * chunk;
+    }
+    rank = idx / ce;
+    head = c * chunk + idx % ce;
+  }
+};
+
 // Byte offset, inside one 128-byte-swizzled [rows][64 x bf16] chunk, of the
 // 16-byte unit `u` (0..7) of row `r`: the unit index is XORed with r mod 8.
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t u) {

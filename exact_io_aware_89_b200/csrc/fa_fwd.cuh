@@ -36,6 +36,7 @@ struct FwdParams {
   float scale_log2;               // softmax scale * log2(e)
   MaskSpec mask;
   int n_qgroups;                  // CTAs along the query axis
+  int head_chunk;                 // heads per scheduling chunk (see ChunkedOrder)
   float* lse;                     // [B, Hq, Nq]
   unsigned long long wait_limit_ns;
 };
@@ -53,6 +54,8 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + NQT * QTILE;
   static constexpr int OFF_V = OFF_K + KST * KTILE;
   static constexpr int OFF_BAR = OFF_V + KST * KTILE;
+  // bar_q, k_full[KST] (with NQT == 2 it signals K and V of the tile together),
+  // k_empty[KST], v_full[KST], v_empty[KST], s_full[2], p_full[2], o_done[2], drain
   static constexpr int NBAR = 1 + 4 * KST + 6 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KiB
@@ -97,10 +100,11 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- work unit: (query group g, batch b, head h); heaviest groups first
-  const int BH = p.B * p.Hq;
-  const int bh = blockIdx.x % BH;
-  const int g = p.n_qgroups - 1 - blockIdx.x / BH;
+  // ---- work unit: (batch b, head h, query group g), heaviest (latest, for
+  // causal) query groups first within L2-sized chunks of heads
+  const ChunkedOrder order(blockIdx.x, p.B * p.Hq, p.n_qgroups, p.head_chunk);
+  const int bh = order.head;
+  const int g = p.n_qgroups - 1 - order.rank;
   const int b = bh / p.Hq, h = bh % p.Hq, hk = h / p.group;
   const int r0 = g * NQT * BM;
   const int r_last = min(p.Nq - 1, r0 + NQT * BM - 1);
@@ -151,18 +155,31 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       for (int it = 0; it < n_kv; ++it) {
         const int s = it % KST, use = it / KST;
         const int krow = (j_begin + it) * BN;
-        if (use > 0 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
-          break;
-        mbar_expect_tx(&k_full[s], C::KTILE);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[s], c * 64, hk, krow, b);
-        ++nk;
-        if (use > 0 && !mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
-          break;
-        mbar_expect_tx(&v_full[s], C::KTILE);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[s], c * 64, hk, krow, b);
-        ++nv;
+        if constexpr (NQT == 2) {
+          // K_j and V_j share a stage and its full barrier; the stage is free
+          // once the last PV of the previous tile in it has completed
+          if (use > 0 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
+            break;
+          mbar_expect_tx(&k_full[s], 2 * C::KTILE);
+          for (int c = 0; c < C::NCHUNK; ++c) {
+            tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[s], c * 64, hk, krow, b);
+            tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &k_full[s], c * 64, hk, krow, b);
+          }
+          ++nk;
+        } else {
+          if (use > 0 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
+            break;
+          mbar_expect_tx(&k_full[s], C::KTILE);
+          for (int c = 0; c < C::NCHUNK; ++c)
+            tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[s], c * 64, hk, krow, b);
+          ++nk;
+          if (use > 0 && !mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
+            break;
+          mbar_expect_tx(&v_full[s], C::KTILE);
+          for (int c = 0; c < C::NCHUNK; ++c)
+            tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[s], c * 64, hk, krow, b);
+          ++nv;
+        }
       }
       // every copy issued must land before the CTA may exit
       mbar_drain(bar_q, 0, p.wait_limit_ns);
@@ -176,6 +193,13 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     if (lane == 0 && n_kv > 0) {
       constexpr uint32_t ID_QK = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
+      // Descriptors are built once; every MMA only adds a compile-time offset
+      // (in 16-byte units) to the start-address field.  The issuing thread
+      // must stay ahead of the tensor core, so it does as little as possible
+      // between MMAs and checks barriers at as few points as it can.
+      const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(sV, C::KCHUNK, 1024);
       auto wait = [&](uint64_t* bar, uint32_t par) {
         const bool ok = mbar_wait(bar, par, abort_flag, &g_status, p.wait_limit_ns);
         tc_fence_after();
@@ -184,47 +208,53 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       // S[slot] = Q_t K_s^T
       auto issue_s = [&](int slot, int t, int s) {
         const uint32_t d_tmem = tmem + C::COL_S + slot * BN;
+        const uint64_t qa = dq0 + static_cast<uint64_t>((t * C::QTILE) >> 4);
+        const uint64_t kb = dk0 + static_cast<uint64_t>((s * C::KTILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2), kb = (kk & 3) * 32;
-          mma_ss(d_tmem, sdesc_sw128(sQ + t * C::QTILE + ko * C::QCHUNK + kb, 16, 1024),
-                 sdesc_sw128(sK + s * C::KTILE + ko * C::KCHUNK + kb, 16, 1024), ID_QK, kk > 0);
+          const uint32_t oq = ((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4;
+          const uint32_t ok_ = ((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4;
+          mma_ss(d_tmem, qa + oq, kb + ok_, ID_QK, kk > 0);
         }
       };
       // O_t (+)= P[slot] V_s
       auto issue_pv = [&](int slot, int t, int s, bool acc) {
         const uint32_t d_tmem = tmem + C::COL_O + t * D;
+        const uint32_t a_tmem = tmem + C::COL_S + slot * BN;
+        const uint64_t vb = dv0 + static_cast<uint64_t>((s * C::KTILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(d_tmem, tmem + C::COL_S + slot * BN + kk * 8,
-                 sdesc_sw128(sV + s * C::KTILE + kk * 2048, C::KCHUNK, 1024), ID_PV,
+          mma_ts(d_tmem, a_tmem + kk * 8, vb + static_cast<uint64_t>(kk * 128), ID_PV,
                  (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
       if (ok) {
         if constexpr (NQT == 2) {
+          // per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1); the two Q
+          // tiles' softmax warpgroups alternate with the tensor core
           issue_s(0, 0, 0);
           tc_commit(&s_full[0]);
           issue_s(1, 1, 0);
           tc_commit(&s_full[1]);
-          tc_commit(&k_empty[0]);
           for (int it = 0; it < n_kv && ok; ++it) {
-            const int s = it % KST;
-            const int s1 = (it + 1) % KST;
-            if (!(ok = wait(&v_full[s], (it / KST) & 1))) break;
-            for (int t = 0; t < 2 && ok; ++t) {
-              if (!(ok = wait(&p_full[t], it & 1))) break;
-              issue_pv(t, t, s, it > 0);
-              tc_commit(&o_done[t]);
-              if (t == 1) tc_commit(&v_empty[s]);
-              if (it + 1 < n_kv) {
-                if (t == 0 && !(ok = wait(&k_full[s1], ((it + 1) / KST) & 1))) break;
-                issue_s(t, t, s1);
-                tc_commit(&s_full[t]);
-                if (t == 1) tc_commit(&k_empty[s1]);
-              }
+            const int s = it % KST, s1 = (it + 1) % KST;
+            const bool more = it + 1 < n_kv;
+            if (!(ok = wait(&p_full[0], it & 1))) break;
+            if (more && !(ok = wait(&k_full[s1], ((it + 1) / KST) & 1))) break;
+            issue_pv(0, 0, s, it > 0);
+            if (more) {
+              issue_s(0, 0, s1);
+              tc_commit(&s_full[0]);
+            }
+            if (!(ok = wait(&p_full[1], it & 1))) break;
+            issue_pv(1, 1, s, it > 0);
+            tc_commit(&k_empty[s]);  // K_j and V_j are no longer read
+            if (more) {
+              issue_s(1, 1, s1);
+              tc_commit(&s_full[1]);
             }
           }
+          if (ok) tc_commit(&o_done[0]);
         } else {
           // one Q tile: S slots alternate between consecutive key tiles
           issue_s(0, 0, 0);
@@ -239,8 +269,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
           }
           for (int it = 0; it < n_kv && ok; ++it) {
             const int slot = it & 1, s = it % KST;
-            if (!(ok = wait(&v_full[s], (it / KST) & 1))) break;
             if (!(ok = wait(&p_full[slot], (it >> 1) & 1))) break;
+            if (!(ok = wait(&v_full[s], (it / KST) & 1))) break;
             issue_pv(slot, 0, s, it > 0);
             tc_commit(&o_done[0]);
             tc_commit(&v_empty[s]);
@@ -353,8 +383,10 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
     // ---- epilogue: O / l -> bf16 -> shared (reusing this tile's Q buffer) -> TMA store
     if (ok && n_kv > 0) {
-      ok = mbar_wait(&o_done[NQT == 2 ? t : 0], (n_kv - 1) & 1, abort_flag, &g_status,
-                     p.wait_limit_ns);
+      // NQT == 2: one commit after the last PV of both tiles (phase 0);
+      // NQT == 1: one commit per PV, the last one is phase n_kv - 1
+      ok = mbar_wait(&o_done[0], NQT == 2 ? 0u : static_cast<uint32_t>((n_kv - 1) & 1), abort_flag,
+                     &g_status, p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
     }
