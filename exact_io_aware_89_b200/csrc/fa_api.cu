@@ -62,9 +62,10 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 using Fwd64 = FwdCfg<64, 2, 128, 3>;
 using Fwd128 = FwdCfg<128, 2, 128, 2>;
 using Fwd256 = FwdCfg<256, 1, 64, 2>;
-// dQ: {d, Q tiles per CTA, key tile, K/V ring depth}
-using Dq64 = DqCfg<64, 2, 64, 3>;
-using Dq128 = DqCfg<128, 2, 64, 2>;
+// dQ: one 128-row query tile per CTA with 128-key tiles {d, K ring, V ring};
+// d = 256 keeps 64-key tiles {d, Q tiles per CTA, key tile, K/V ring depth}
+using Dq64 = Dq2Cfg<64, 4, 3>;
+using Dq128 = Dq2Cfg<128, 3, 2>;
 using Dq256 = DqCfg<256, 1, 64, 1>;
 // dK/dV: {d, accumulated d slice, query tile, Q/dO ring depth}
 using Dkv64 = DkvCfg<64, 64, 64, 4>;
@@ -182,11 +183,18 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         !encode_bnhd(&tv, v, B, Nk, Hkv, D, CQ::BN) || !encode_bnhd(&tdo, dO, B, Nq, Hq, D, CQ::BM) ||
         !encode_bnhd(&tdq, dq, B, Nq, Hq, D, CQ::BM))
       return FA_ERR_CUDA;
-    auto kern = fa_bwd_dq_kernel<CQ>;
-    if (smem_attr_once(kern, CQ::SMEM_BYTES, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
     const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
-    TraceScope tr(FA_KERNEL_BWD_DQ, stream);
-    kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
+    if constexpr (CQ::ONE_TILE) {
+      auto kern = fa_bwd_dq2_kernel<CQ>;
+      if (smem_attr_once(kern, CQ::SMEM_BYTES, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
+      TraceScope tr(FA_KERNEL_BWD_DQ, stream);
+      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
+    } else {
+      auto kern = fa_bwd_dq_kernel<CQ>;
+      if (smem_attr_once(kern, CQ::SMEM_BYTES, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
+      TraceScope tr(FA_KERNEL_BWD_DQ, stream);
+      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
+    }
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
   {

@@ -103,6 +103,7 @@ template <int D_, int NQT_, int BN_, int KST_>
 struct DqCfg {
   static constexpr int D = D_, NQT = NQT_, BN = BN_, KST = KST_;
   static constexpr int BM = 128;
+  static constexpr bool ONE_TILE = false;
   static constexpr int NCHUNK = D / 64;
   static constexpr int QCHUNK = BM * 128;
   static constexpr int KCHUNK = BN * 128;
@@ -370,6 +371,306 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     if (r == 0 && *abort_flag == 0 && r0 + t * BM < p.Nq) {
       for (int c = 0; c < C::NCHUNK; ++c)
         tma_store_4d(&tm_dq, stage + c * C::QCHUNK, c * 64, h, r0 + t * BM, b);
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == C::MMA_WARP) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// =====================================================================
+// 2b. dQ, one 128-row query tile per CTA, 128-key tiles (d <= 128)
+// =====================================================================
+// S = Q K_j^T and dP = dO V_j^T land in TMEM (N = 128, so the shared-memory
+// operand traffic matches the tensor core).  Both warpgroups read them (each
+// owns 64 of the 128 key columns of every row) and release them at once, so
+// S/dP of the next key tile are computed while dS of this one is formed.  dS
+// (bf16) goes to its own TMEM columns and feeds dQ += dS K_j as the A operand.
+// K is needed first (S) and last (dQ), V only for dP, so K gets the deeper
+// ring: each tile's loads are issued two steps ahead of their use.
+template <int D_, int KS_, int VS_>
+struct Dq2Cfg {
+  static constexpr int D = D_, KS = KS_, VS = VS_;
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int NQT = 1;
+  static constexpr bool ONE_TILE = true;
+  // the next key tile's K stage must be free before this tile's dQ is issued
+  static_assert(KS >= 2 && VS >= 2, "needs at least two K and two V stages");
+  static constexpr int NCHUNK = D / 64;
+  static constexpr int QCHUNK = BM * 128;
+  static constexpr int KCHUNK = BN * 128;
+  static constexpr int QTILE = NCHUNK * QCHUNK;
+  static constexpr int KTILE = NCHUNK * KCHUNK;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = OFF_Q + QTILE;
+  static constexpr int OFF_K = OFF_DO + QTILE;                // K stages [KS]
+  static constexpr int OFF_V = OFF_K + KS * KTILE;            // V stages [VS]
+  static constexpr int OFF_BAR = OFF_V + VS * KTILE;
+  // q_full, k_full/k_empty[KS], v_full/v_empty[VS], sp_full, sp_free, ds_full, ds_free, dq_done, drain
+  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 6;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int NWARPS = 10;
+  static constexpr int NTHREADS = 32 * NWARPS;
+  static constexpr int TMA_WARP = 8, MMA_WARP = 9;
+  // TMEM: S, dP (fp32), dQ (fp32), dS (bf16 pairs: 64 columns)
+  static constexpr int COL_S = 0, COL_DP = BN, COL_DQ = 2 * BN, COL_DS = 2 * BN + D;
+  static constexpr int TMEM_USED = COL_DS + BN / 2;
+  static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
+  static_assert(TMEM_USED <= 512, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::NTHREADS, 1)
+    fa_bwd_dq2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                      const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+  constexpr int D = C::D, BN = C::BN, KS = C::KS, VS = C::VS, BM = C::BM;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + KS;
+  uint64_t* v_full = k_empty + KS;
+  uint64_t* v_empty = v_full + VS;
+  uint64_t* sp_full = v_empty + VS;
+  uint64_t* sp_free = sp_full + 1;
+  uint64_t* ds_full = sp_free + 1;
+  uint64_t* ds_free = ds_full + 1;
+  uint64_t* dq_done = ds_free + 1;
+  uint64_t* bar_drain = dq_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  const uint32_t sQ = sbase + C::OFF_Q, sdO = sbase + C::OFF_DO, sK = sbase + C::OFF_K,
+                 sV = sbase + C::OFF_V;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  const ChunkedOrder order(blockIdx.x, p.B * p.Hq, p.n_qgroups, p.head_chunk);
+  const int bh = order.head;
+  const int g = p.n_qgroups - 1 - order.rank;  // query tile, latest first
+  const int b = bh / p.Hq, h = bh % p.Hq, hk = h / p.group;
+  const int r0 = g * BM;
+  const int r_last = min(p.Nq - 1, r0 + BM - 1);
+  const int key_lo = p.mask.lo(r0), key_hi = p.mask.hi(r_last);
+  const int j_begin = key_lo / BN;
+  const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    mbar_init(sp_full, 1);
+    mbar_init(sp_free, 256);
+    mbar_init(ds_full, 256);
+    mbar_init(ds_free, 1);
+    mbar_init(dq_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::TMA_WARP) {
+    if (lane == 0 && n_kv > 0) {
+      mbar_expect_tx(q_full, 2 * C::QTILE);
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        tma_load_4d(sQ + c * C::QCHUNK, &tm_q, q_full, c * 64, h, r0, b);
+        tma_load_4d(sdO + c * C::QCHUNK, &tm_do, q_full, c * 64, h, r0, b);
+      }
+      int nk = 0, nv = 0;
+      for (int it = 0; it < n_kv; ++it) {
+        const int sk = it % KS, uk = it / KS, sv = it % VS, uv = it / VS;
+        const int krow = (j_begin + it) * BN;
+        if (uk > 0 && !mbar_wait(&k_empty[sk], (uk - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
+          break;
+        mbar_expect_tx(&k_full[sk], C::KTILE);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sK + sk * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[sk], c * 64, hk, krow, b);
+        ++nk;
+        if (uv > 0 && !mbar_wait(&v_empty[sv], (uv - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
+          break;
+        mbar_expect_tx(&v_full[sv], C::KTILE);
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sV + sv * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[sv], c * 64, hk, krow, b);
+        ++nv;
+      }
+      mbar_drain(q_full, 0, p.wait_limit_ns);
+      for (int s = 0; s < KS; ++s)
+        if (nk > s) mbar_drain(&k_full[s], ((nk - 1 - s) / KS) & 1, p.wait_limit_ns);
+      for (int s = 0; s < VS; ++s)
+        if (nv > s) mbar_drain(&v_full[s], ((nv - 1 - s) / VS) & 1, p.wait_limit_ns);
+    }
+  } else if (warp == C::MMA_WARP) {
+    if (lane == 0 && n_kv > 0) {
+      constexpr uint32_t ID_S = idesc_bf16_f32(128, BN, false, false);
+      constexpr uint32_t ID_DQ = idesc_bf16_f32(128, D, false, true);
+      auto wait = [&](uint64_t* bar, uint32_t par) {
+        const bool ok = mbar_wait(bar, par, abort_flag, &g_status, p.wait_limit_ns);
+        tc_fence_after();
+        return ok;
+      };
+      const uint64_t dq_q = sdesc_sw128(sQ, 16, 1024), dq_do = sdesc_sw128(sdO, 16, 1024);
+      const uint64_t dq_k = sdesc_sw128(sK, 16, 1024), dq_v = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dq_kmn = sdesc_sw128(sK, C::KCHUNK, 1024);
+      // S = Q K^T, dP = dO V^T for key tile it
+      auto issue_sdp = [&](int it) {
+        const uint64_t kb = dq_k + static_cast<uint64_t>(((it % KS) * C::KTILE) >> 4);
+        const uint64_t vb = dq_v + static_cast<uint64_t>(((it % VS) * C::KTILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t qo = ((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4;
+          const uint32_t ko = ((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + C::COL_S, dq_q + qo, kb + ko, ID_S, kk > 0);
+          mma_ss(tmem + C::COL_DP, dq_do + qo, vb + ko, ID_S, kk > 0);
+        }
+      };
+      // dQ (+)= dS K: dS from TMEM, K as MN-major B
+      auto issue_dq = [&](int it) {
+        const uint64_t kb = dq_kmn + static_cast<uint64_t>(((it % KS) * C::KTILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + C::COL_DQ, tmem + C::COL_DS + kk * 8, kb + static_cast<uint64_t>(kk * 128), ID_DQ,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait(q_full, 0) && wait(&k_full[0], 0) && wait(&v_full[0], 0);
+      if (ok) {
+        issue_sdp(0);
+        tc_commit(sp_full);
+        tc_commit(&v_empty[0]);
+        for (int it = 0; it < n_kv && ok; ++it) {
+          if (it + 1 < n_kv) {
+            const int nx = it + 1;
+            // the next key tile's S/dP as soon as both warpgroups have read this one's
+            if (!(ok = wait(sp_free, it & 1))) break;
+            if (!(ok = wait(&k_full[nx % KS], (nx / KS) & 1))) break;
+            if (!(ok = wait(&v_full[nx % VS], (nx / VS) & 1))) break;
+            issue_sdp(nx);
+            tc_commit(sp_full);
+            tc_commit(&v_empty[nx % VS]);
+          }
+          if (!(ok = wait(ds_full, it & 1))) break;
+          issue_dq(it);
+          tc_commit(ds_free);
+          tc_commit(&k_empty[it % KS]);
+        }
+        if (ok) tc_commit(dq_done);
+      }
+    }
+    if (lane == 0) {
+      tc_commit(bar_drain);
+      mbar_drain(bar_drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------- dS warpgroups (thread = query row)
+    const int wg = warp / 4;          // key columns [64 wg, 64 wg + 64) of every tile
+    const int r = threadIdx.x % BM;   // row == TMEM lane
+    const int row = r0 + r;
+    const int lo = p.mask.lo(row), hi = p.mask.hi(row);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    const size_t srow = (static_cast<size_t>(b) * p.Hq + h) * p.Nq_pad + row;  // row < Nq_pad
+    const float lse2 = p.lse2[srow];
+    const float Drow = p.D[srow];
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < n_kv; ++it) {
+      ok = mbar_wait(sp_full, it & 1, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[64], dv[64];
+      tmem_ld_x32(lane_base + C::COL_S + wg * 64, sv);
+      tmem_ld_x32(lane_base + C::COL_S + wg * 64 + 32, sv + 32);
+      tmem_ld_x32(lane_base + C::COL_DP + wg * 64, dv);
+      tmem_ld_x32(lane_base + C::COL_DP + wg * 64 + 32, dv + 32);
+      tmem_ld_wait_x32(sv);
+      tmem_ld_wait_x32(sv + 32);
+      tmem_ld_wait_x32(dv);
+      tmem_ld_wait_x32(dv + 32);
+      tc_fence_before();
+      mbar_arrive(sp_free);  // S/dP may now be overwritten by the next key tile
+      const int k0 = (j_begin + it) * BN + wg * 64;
+      if (k0 < lo || k0 + 63 > hi) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int key = k0 + c;
+          if (key < lo || key > hi) sv[c] = __float_as_uint(-INFINITY);
+        }
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse2));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse2));
+        pk[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - Drow), p1 * (__uint_as_float(dv[c + 1]) - Drow));
+      }
+      // the previous key tile's dQ MMA must be done reading dS
+      if (it > 0) {
+        ok = mbar_wait(ds_free, (it - 1) & 1, abort_flag, &g_status, p.wait_limit_ns);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      tmem_st_x32(lane_base + C::COL_DS + wg * 32, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    if (ok && n_kv > 0) {
+      ok = mbar_wait(dq_done, 0, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+    // epilogue: dQ * scale -> bf16 -> shared (the Q buffer) -> TMA store;
+    // warpgroup wg stages the 64-column chunks wg, wg + 2, ...
+    if (ok) {
+#pragma unroll 1
+      for (int c = wg; c < C::NCHUNK; c += 2) {
+        uint32_t ov[64];
+        if (n_kv > 0) {
+          tmem_ld_x32(lane_base + C::COL_DQ + c * 64, ov);
+          tmem_ld_x32(lane_base + C::COL_DQ + c * 64 + 32, ov + 32);
+          tmem_ld_wait_x32(ov);
+          tmem_ld_wait_x32(ov + 32);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) ov[i] = 0u;
+        }
+        const float sc = p.scale;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float* f = reinterpret_cast<const float*>(ov + 8 * u);
+          st_shared_v4(sQ + c * C::QCHUNK + sw128_offset(r, u), pack_bf16x2(f[0] * sc, f[1] * sc),
+                       pack_bf16x2(f[2] * sc, f[3] * sc), pack_bf16x2(f[4] * sc, f[5] * sc),
+                       pack_bf16x2(f[6] * sc, f[7] * sc));
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(1, 256);
+    if (threadIdx.x == 0 && *abort_flag == 0 && r0 < p.Nq) {
+      for (int c = 0; c < C::NCHUNK; ++c) tma_store_4d(&tm_dq, sQ + c * C::QCHUNK, c * 64, h, r0, b);
       tma_store_commit();
       tma_store_wait_all();
     }
