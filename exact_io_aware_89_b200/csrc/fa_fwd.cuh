@@ -59,10 +59,21 @@ struct FwdCfg {
   static constexpr int NBAR = 1 + 4 * KST + 6 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KiB
-  static constexpr int NWARPS = 4 * NQT + 2;
+  // softmax warpgroups first, then one producer warpgroup (TMA warp, MMA
+  // warp, two idle warps) so registers can move to the softmax warpgroups
+  static constexpr int NWARPS = 4 * NQT + 4;
   static constexpr int NTHREADS = 32 * NWARPS;
   static constexpr int TMA_WARP = 4 * NQT;
   static constexpr int MMA_WARP = 4 * NQT + 1;
+  // registers per thread: at launch (65536 / NTHREADS, rounded down to 8),
+  // producer share, softmax share; the shares add up to the launch total
+  static constexpr int REG_LAUNCH = (65536 / NTHREADS) / 8 * 8;
+  static constexpr int REG_PRODUCER = 80;
+  static constexpr int REG_MATH =
+      ((NTHREADS * REG_LAUNCH - 128 * REG_PRODUCER) / (128 * NQT)) / 8 * 8 > 248
+          ? 248
+          : ((NTHREADS * REG_LAUNCH - 128 * REG_PRODUCER) / (128 * NQT)) / 8 * 8;
+  static_assert(NQT * 128 * REG_MATH + 128 * REG_PRODUCER <= NTHREADS * REG_LAUNCH, "register split");
   static constexpr int COL_S = 0;        // S slot s: columns [s*BN, s*BN+BN); its P: first BN/2
   static constexpr int COL_O = 2 * BN;   // O of Q tile t: columns [COL_O + t*D, +D)
   static constexpr int TMEM_USED = 2 * BN + NQT * D;
@@ -146,6 +157,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 
   if (warp == C::TMA_WARP) {
     // ------------------------------------------------------------ producer
+    setmaxnreg_dec<C::REG_PRODUCER>();
     if (lane == 0 && n_kv > 0) {
       mbar_expect_tx(bar_q, NQT * C::QTILE);
       for (int t = 0; t < NQT; ++t)
@@ -190,6 +202,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
+    setmaxnreg_dec<C::REG_PRODUCER>();
     if (lane == 0 && n_kv > 0) {
       constexpr uint32_t ID_QK = idesc_bf16_f32(128, BN, false, false);
       constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
@@ -290,8 +303,9 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       mbar_drain(bar_drain, 0, p.wait_limit_ns);
     }
     __syncwarp();
-  } else {
+  } else if (warp < C::TMA_WARP) {
     // ------------------------------------------------------------ softmax
+    setmaxnreg_inc<C::REG_MATH>();
     const int t = warp / 4;          // Q tile of this warpgroup
     const int r = threadIdx.x % BM;  // row within the tile == TMEM lane
     const int row = r0 + t * BM + r;
@@ -428,6 +442,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Nq + row] =
           (l > 0.f) ? (mb + log2f(l)) * kLn2 : -INFINITY;
     }
+  } else {
+    setmaxnreg_dec<C::REG_PRODUCER>();  // idle members of the producer warpgroup
   }
 
   tc_fence_before();

@@ -90,6 +90,18 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint6
   return true;
 }
 
+// Register reallocation between warpgroups (all four warps of a warpgroup
+// execute the same one).  The shares must add up to the block's launch
+// allocation (threads x registers per thread at launch).
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // named barrier over `nthreads` threads (a multiple of 32)
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
