@@ -62,6 +62,43 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t u) {
   return r * 128u + ((u ^ (r & 7u)) << 4);
 }
 
+// 2^x for a pair of arguments on the FMA pipe (the MUFU unit alone would
+// bound the softmax).  x is clamped to [-126, inf) and split as x = j + f with
+// j = round(x), f in [-1/2, 1/2] (Cody and Waite's range reduction; adding
+// 1.5 * 2^23 leaves j in the low mantissa bits); 2^f comes from a degree-3
+// polynomial and 2^j is added into the exponent field, the bit-level trick of
+// Schraudolph's fast exponential (Neural Computation, 1999).  The polynomial is the minimax fit, in relative error,
+// of 2^f on [-1/2, 1/2] (Remez exchange; max relative error 7.5e-5, well
+// under the 2^-9 rounding of P to bf16).  Arguments below -125 (possible only
+// for scores far below the row max) give a value below 2^-125 instead of ~0
+// (a subnormal at the clamp); a row sum is at least 1, so that is far below
+// fp32 resolution.  Masked (-inf)
+// scores must not come here: they take ex2_approx, which returns exact 0.
+constexpr float kExp2C0 = 0.99992806f;
+constexpr float kExp2C1 = 0.69326097f;
+constexpr float kExp2C2 = 0.24261113f;
+constexpr float kExp2C3 = 0.05517167f;
+
+__device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& lo, float& hi) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  float xl, xh;
+  f2_unpack(x2, xl, xh);
+  const uint64_t x = f2_pack(fmaxf(xl, -126.0f), fmaxf(xh, -126.0f));
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));    // kRound + j
+  const uint64_t j = f2_add(t, f2_pack(-kRound, -kRound));  // j, exact
+  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);   // x - j
+  uint64_t p = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  float pl, ph, tl, th;
+  f2_unpack(p, pl, ph);
+  f2_unpack(t, tl, th);
+  // the low 9 bits of t's pattern hold j (two's complement); shifted to the
+  // exponent field they add j to p's exponent
+  lo = __uint_as_float(__float_as_uint(pl) + (__float_as_uint(tl) << 23));
+  hi = __uint_as_float(__float_as_uint(ph) + (__float_as_uint(th) << 23));
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),

@@ -22,6 +22,11 @@
 // S/PV while the other tile's softmax runs.  For d = 256 (one Q tile) the two
 // S slots alternate between consecutive key tiles instead.
 //
+// In tiles without masked keys, NPOLY of every 8 pairs of exponentials are
+// computed on the FMA pipe (exp2_poly_pair) rather than the MUFU unit, which
+// would otherwise bound the softmax; tiles with masked keys use MUFU ex2 only,
+// which returns exact zeros for -inf.
+//
 // The running max is only moved (and O rescaled) when the tile max exceeds
 // it by more than 2^8 in the exp2 domain; otherwise the old reference is kept.
 // Every P stays <= 2^8, the result is the same exact softmax (the reference
@@ -41,9 +46,12 @@ struct FwdParams {
   unsigned long long wait_limit_ns;
 };
 
-template <int D_, int NQT_, int BN_, int KST_>
+template <int D_, int NQT_, int BN_, int KST_, int NPOLY_ = 2>
 struct FwdCfg {
   static constexpr int D = D_, NQT = NQT_, BN = BN_, KST = KST_;
+  // of every 8 score pairs of an unmasked tile, NPOLY take exp2 on the FMA
+  // pipe (exp2_poly_pair), the rest on the MUFU unit
+  static constexpr int NPOLY = NPOLY_;
   static constexpr int BM = 128;
   static constexpr int NCHUNK = D / 64;      // 128-byte swizzle chunks across d
   static constexpr int QCHUNK = BM * 128;    // bytes of one 64-column chunk of a Q tile
@@ -66,9 +74,13 @@ struct FwdCfg {
   static constexpr int TMA_WARP = 4 * NQT;
   static constexpr int MMA_WARP = 4 * NQT + 1;
   // registers per thread: at launch (65536 / NTHREADS, rounded down to 8),
-  // producer share, softmax share; the shares add up to the launch total
+  // producer share, softmax share; the shares add up to the launch total.
+  // The MMA thread keeps only base descriptors live (FwdIssueS / FwdIssuePV),
+  // so the producer warpgroup gets by with 40 and the softmax warpgroups get
+  // 232 (two Q tiles): with more registers their exp / pack stream schedules
+  // with more instruction-level parallelism.
   static constexpr int REG_LAUNCH = (65536 / NTHREADS) / 8 * 8;
-  static constexpr int REG_PRODUCER = 80;
+  static constexpr int REG_PRODUCER = 40;
   static constexpr int REG_MATH =
       ((NTHREADS * REG_LAUNCH - 128 * REG_PRODUCER) / (128 * NQT)) / 8 * 8 > 248
           ? 248
@@ -82,6 +94,31 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(D % 64 == 0 && BN % 64 == 0, "tile shapes");
   static_assert(NQT == 1 || NQT == 2, "one or two Q tiles per CTA");
+};
+
+// Unrolled MMA sequences with compile-time descriptor offsets (mma_ss_at /
+// mma_ts_at): S = Q K^T over d in steps of 16, and O (+)= P V over the key
+// tile in steps of 16.
+template <class C, int KK = 0>
+struct FwdIssueS {
+  static __device__ __forceinline__ void run(uint32_t d_tmem, uint64_t qa, uint64_t kb, uint32_t id) {
+    if constexpr (KK < C::D / 16) {
+      constexpr uint32_t oq = ((KK >> 2) * C::QCHUNK + (KK & 3) * 32) >> 4;
+      constexpr uint32_t ok = ((KK >> 2) * C::KCHUNK + (KK & 3) * 32) >> 4;
+      mma_ss_at<oq, ok>(d_tmem, qa, kb, id, KK > 0 ? 1u : 0u);
+      FwdIssueS<C, KK + 1>::run(d_tmem, qa, kb, id);
+    }
+  }
+};
+template <class C, int KK = 0>
+struct FwdIssuePV {
+  static __device__ __forceinline__ void run(uint32_t d_tmem, uint32_t a_tmem, uint64_t vb, uint32_t id,
+                                             bool acc) {
+    if constexpr (KK < C::BN / 16) {
+      mma_ts_at<KK * 8, KK * 128>(d_tmem, a_tmem, vb, id, (acc || KK > 0) ? 1u : 0u);
+      FwdIssuePV<C, KK + 1>::run(d_tmem, a_tmem, vb, id, acc);
+    }
+  }
 };
 
 template <class C>
@@ -220,25 +257,13 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       };
       // S[slot] = Q_t K_s^T
       auto issue_s = [&](int slot, int t, int s) {
-        const uint32_t d_tmem = tmem + C::COL_S + slot * BN;
-        const uint64_t qa = dq0 + static_cast<uint64_t>((t * C::QTILE) >> 4);
-        const uint64_t kb = dk0 + static_cast<uint64_t>((s * C::KTILE) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oq = ((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4;
-          const uint32_t ok_ = ((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4;
-          mma_ss(d_tmem, qa + oq, kb + ok_, ID_QK, kk > 0);
-        }
+        FwdIssueS<C>::run(tmem + C::COL_S + slot * BN, dq0 + static_cast<uint64_t>((t * C::QTILE) >> 4),
+                          dk0 + static_cast<uint64_t>((s * C::KTILE) >> 4), ID_QK);
       };
       // O_t (+)= P[slot] V_s
       auto issue_pv = [&](int slot, int t, int s, bool acc) {
-        const uint32_t d_tmem = tmem + C::COL_O + t * D;
-        const uint32_t a_tmem = tmem + C::COL_S + slot * BN;
-        const uint64_t vb = dv0 + static_cast<uint64_t>((s * C::KTILE) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, vb + static_cast<uint64_t>(kk * 128), ID_PV,
-                 (acc || kk > 0) ? 1u : 0u);
+        FwdIssuePV<C>::run(tmem + C::COL_O + t * D, tmem + C::COL_S + slot * BN,
+                           dv0 + static_cast<uint64_t>((s * C::KTILE) >> 4), ID_PV, acc);
       };
       bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
       if (ok) {
@@ -330,22 +355,24 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       for (int cc = 0; cc < BN / 32; ++cc) tmem_ld_wait_x32(&sv[cc * 32]);
       float* sc = reinterpret_cast<float*>(sv);
       const int k0 = (j_begin + it) * BN;
-      if (k0 < lo || k0 + BN - 1 > hi) {
+      const bool edge = k0 < lo || k0 + BN - 1 > hi;
+      if (edge) {
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
           const int key = k0 + c;
           if (key < lo || key > hi) sc[c] = -INFINITY;
         }
       }
-      float mx0 = sc[0], mx1 = sc[1], mx2 = sc[2], mx3 = sc[3];
+      float mx0 = fmaxf(sc[0], sc[1]), mx1 = fmaxf(sc[2], sc[3]);
+      float mx2 = fmaxf(sc[4], sc[5]), mx3 = fmaxf(sc[6], sc[7]);
 #pragma unroll
-      for (int c = 4; c < BN; c += 4) {
-        mx0 = fmaxf(mx0, sc[c]);
-        mx1 = fmaxf(mx1, sc[c + 1]);
-        mx2 = fmaxf(mx2, sc[c + 2]);
-        mx3 = fmaxf(mx3, sc[c + 3]);
+      for (int c = 8; c < BN; c += 8) {
+        mx0 = fmax3(mx0, sc[c], sc[c + 1]);
+        mx1 = fmax3(mx1, sc[c + 2], sc[c + 3]);
+        mx2 = fmax3(mx2, sc[c + 4], sc[c + 5]);
+        mx3 = fmax3(mx3, sc[c + 6], sc[c + 7]);
       }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_tile = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
       const float m_new = fmaxf(m_ref, m_tile);
       const bool grow = m_new > m_ref + 8.0f;
       float alpha = 1.f;
@@ -355,15 +382,42 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       }
       const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
       uint32_t pk[BN / 2];
-      float rs0 = 0.f, rs1 = 0.f;
+      const uint64_t scale2 = f2_pack(sl2, sl2), shift2 = f2_pack(-mb, -mb);
+      uint64_t acc0 = 0, acc1 = 0;  // running row sums, two pairs of fp32 lanes
+      if (edge) {  // masked scores are -inf: MUFU ex2 only, which gives exact zeros
 #pragma unroll
-      for (int c = 0; c < BN; c += 2) {
-        const float p0 = ex2_approx(fmaf(sc[c], sl2, -mb));
-        const float p1 = ex2_approx(fmaf(sc[c + 1], sl2, -mb));
-        rs0 += p0;
-        rs1 += p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < BN; c += 2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(sc[c], sc[c + 1]), scale2, shift2), x0, x1);
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          pk[c / 2] = pack_bf16x2(p0, p1);
+          if ((c / 2) & 1)
+            acc1 = f2_add(acc1, f2_pack(p0, p1));
+          else
+            acc0 = f2_add(acc0, f2_pack(p0, p1));
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < BN; c += 2) {
+          const uint64_t x2 = f2_fma(f2_pack(sc[c], sc[c + 1]), scale2, shift2);
+          float p0, p1;
+          if ((c / 2) % 8 < C::NPOLY) {
+            exp2_poly_pair(x2, p0, p1);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          pk[c / 2] = pack_bf16x2(p0, p1);
+          if ((c / 2) & 1)
+            acc1 = f2_add(acc1, f2_pack(p0, p1));
+          else
+            acc0 = f2_add(acc0, f2_pack(p0, p1));
+        }
       }
+      float rs0, rs1;
+      f2_unpack(f2_add(acc0, acc1), rs0, rs1);
       l = l * alpha + (rs0 + rs1);
 #pragma unroll
       for (int cc = 0; cc < BN / 64; ++cc) tmem_st_x32(lane_base + col_s + cc * 32, &pk[cc * 32]);
