@@ -59,8 +59,9 @@ struct TraceScope {
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 // fwd: {d, Q tiles per CTA, key tile, K/V ring depth}
-// {d, Q tiles per CTA, key tile, K/V ring depth, exp2 pairs of 8 on the FMA pipe}
-using Fwd64 = FwdCfg<64, 2, 128, 3, 2>;
+// {d, Q tiles per CTA, key tile, K/V ring depth, exp2 pairs of 8 on the FMA pipe,
+//  P handed over in two halves}
+using Fwd64 = FwdCfg<64, 2, 128, 3, 2, true>;
 using Fwd128 = FwdCfg<128, 2, 128, 2, 2>;
 using Fwd256 = FwdCfg<256, 1, 64, 2>;
 // dQ: one 128-row query tile per CTA with 128-key tiles {d, K ring, V ring};

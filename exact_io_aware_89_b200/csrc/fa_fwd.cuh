@@ -46,9 +46,13 @@ struct FwdParams {
   unsigned long long wait_limit_ns;
 };
 
-template <int D_, int NQT_, int BN_, int KST_, int NPOLY_ = 2>
+template <int D_, int NQT_, int BN_, int KST_, int NPOLY_ = 2, bool SPLITP_ = false>
 struct FwdCfg {
   static constexpr int D = D_, NQT = NQT_, BN = BN_, KST = KST_;
+  // NQT == 2 only: P reaches the tensor core in two key halves, so the first
+  // half's PV overlaps the softmax of the second (one more wait point per
+  // tile in the MMA thread; pays off when the PV is short, i.e. small d)
+  static constexpr bool SPLITP = SPLITP_ && NQT_ == 2;
   // of every 8 score pairs of an unmasked tile, NPOLY take exp2 on the FMA
   // pipe (exp2_poly_pair), the rest on the MUFU unit
   static constexpr int NPOLY = NPOLY_;
@@ -63,8 +67,10 @@ struct FwdCfg {
   static constexpr int OFF_V = OFF_K + KST * KTILE;
   static constexpr int OFF_BAR = OFF_V + KST * KTILE;
   // bar_q, k_full[KST] (with NQT == 2 it signals K and V of the tile together),
-  // k_empty[KST], v_full[KST], v_empty[KST], s_full[2], p_full[2], o_done[2], drain
-  static constexpr int NBAR = 1 + 4 * KST + 6 + 1;
+  // k_empty[KST], v_full[KST], v_empty[KST], s_full[2], p_full[4], o_done[2], drain
+  // (p_full: NQT == 2, [2t + half] for the key halves of Q tile t, [2t]
+  // alone without SPLITP; NQT == 1, [slot])
+  static constexpr int NBAR = 1 + 4 * KST + 8 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack to align the base to 1 KiB
   // softmax warpgroups first, then one producer warpgroup (TMA warp, MMA
@@ -110,16 +116,43 @@ struct FwdIssueS {
     }
   }
 };
-template <class C, int KK = 0>
+template <class C, int KK = 0, int KEND = C::BN / 16>
 struct FwdIssuePV {
   static __device__ __forceinline__ void run(uint32_t d_tmem, uint32_t a_tmem, uint64_t vb, uint32_t id,
                                              bool acc) {
-    if constexpr (KK < C::BN / 16) {
+    if constexpr (KK < KEND) {
       mma_ts_at<KK * 8, KK * 128>(d_tmem, a_tmem, vb, id, (acc || KK > 0) ? 1u : 0u);
-      FwdIssuePV<C, KK + 1>::run(d_tmem, a_tmem, vb, id, acc);
+      FwdIssuePV<C, KK + 1, KEND>::run(d_tmem, a_tmem, vb, id, acc);
     }
   }
 };
+
+// P for score columns [C0, C1) of one row: 2^(s * scale_log2 - mb) packed to
+// bf16 pairs into pk[C0/2 ..], row sums accumulated into two fp32 pairs.
+// EDGE: the tile has masked (-inf) scores, so MUFU ex2 only (exact zeros);
+// otherwise NPOLY of every 8 pairs use exp2_poly_pair.
+template <class C, int C0, int C1, bool EDGE>
+__device__ __forceinline__ void fwd_exp_cols(const float* sc, uint64_t scale2, uint64_t shift2,
+                                             uint32_t* pk, uint64_t& acc0, uint64_t& acc1) {
+#pragma unroll
+  for (int c = C0; c < C1; c += 2) {
+    const uint64_t x2 = f2_fma(f2_pack(sc[c], sc[c + 1]), scale2, shift2);
+    float p0, p1;
+    if (!EDGE && (c / 2) % 8 < C::NPOLY) {
+      exp2_poly_pair(x2, p0, p1);
+    } else {
+      float x0, x1;
+      f2_unpack(x2, x0, x1);
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    pk[c / 2] = pack_bf16x2(p0, p1);
+    if ((c / 2) & 1)
+      acc1 = f2_add(acc1, f2_pack(p0, p1));
+    else
+      acc0 = f2_add(acc0, f2_pack(p0, p1));
+  }
+}
 
 template <class C>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
@@ -138,8 +171,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   uint64_t* v_full = k_empty + KST;
   uint64_t* v_empty = v_full + KST;
   uint64_t* s_full = v_empty + KST;  // [2]
-  uint64_t* p_full = s_full + 2;     // [2]
-  uint64_t* o_done = p_full + 2;     // [2]
+  uint64_t* p_full = s_full + 2;     // [4]
+  uint64_t* o_done = p_full + 4;     // [2]
   uint64_t* bar_drain = o_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
@@ -170,9 +203,9 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], BM);
       mbar_init(&o_done[s], 1);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&p_full[i], BM);
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -260,16 +293,26 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
         FwdIssueS<C>::run(tmem + C::COL_S + slot * BN, dq0 + static_cast<uint64_t>((t * C::QTILE) >> 4),
                           dk0 + static_cast<uint64_t>((s * C::KTILE) >> 4), ID_QK);
       };
-      // O_t (+)= P[slot] V_s
+      // O_t (+)= P[slot] V_s, over the whole key tile or one half of it
       auto issue_pv = [&](int slot, int t, int s, bool acc) {
         FwdIssuePV<C>::run(tmem + C::COL_O + t * D, tmem + C::COL_S + slot * BN,
                            dv0 + static_cast<uint64_t>((s * C::KTILE) >> 4), ID_PV, acc);
+      };
+      auto issue_pv_lo = [&](int slot, int t, int s, bool acc) {
+        FwdIssuePV<C, 0, BN / 32>::run(tmem + C::COL_O + t * D, tmem + C::COL_S + slot * BN,
+                                       dv0 + static_cast<uint64_t>((s * C::KTILE) >> 4), ID_PV, acc);
+      };
+      auto issue_pv_hi = [&](int slot, int t, int s) {
+        FwdIssuePV<C, BN / 32, BN / 16>::run(tmem + C::COL_O + t * D, tmem + C::COL_S + slot * BN,
+                                             dv0 + static_cast<uint64_t>((s * C::KTILE) >> 4), ID_PV, true);
       };
       bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
       if (ok) {
         if constexpr (NQT == 2) {
           // per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1); the two Q
-          // tiles' softmax warpgroups alternate with the tensor core
+          // tiles' softmax warpgroups alternate with the tensor core.  With
+          // SPLITP, P arrives in two key halves, and the first half's PV
+          // runs while the softmax still computes the second.
           issue_s(0, 0, 0);
           tc_commit(&s_full[0]);
           issue_s(1, 1, 0);
@@ -277,15 +320,28 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
           for (int it = 0; it < n_kv && ok; ++it) {
             const int s = it % KST, s1 = (it + 1) % KST;
             const bool more = it + 1 < n_kv;
-            if (!(ok = wait(&p_full[0], it & 1))) break;
+            const uint32_t par = it & 1;
+            if (!(ok = wait(&p_full[0], par))) break;
             if (more && !(ok = wait(&k_full[s1], ((it + 1) / KST) & 1))) break;
-            issue_pv(0, 0, s, it > 0);
+            if constexpr (C::SPLITP) {
+              issue_pv_lo(0, 0, s, it > 0);
+              if (!(ok = wait(&p_full[1], par))) break;
+              issue_pv_hi(0, 0, s);
+            } else {
+              issue_pv(0, 0, s, it > 0);
+            }
             if (more) {
               issue_s(0, 0, s1);
               tc_commit(&s_full[0]);
             }
-            if (!(ok = wait(&p_full[1], it & 1))) break;
-            issue_pv(1, 1, s, it > 0);
+            if (!(ok = wait(&p_full[2], par))) break;
+            if constexpr (C::SPLITP) {
+              issue_pv_lo(1, 1, s, it > 0);
+              if (!(ok = wait(&p_full[3], par))) break;
+              issue_pv_hi(1, 1, s);
+            } else {
+              issue_pv(1, 1, s, it > 0);
+            }
             tc_commit(&k_empty[s]);  // K_j and V_j are no longer read
             if (more) {
               issue_s(1, 1, s1);
@@ -384,57 +440,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       uint32_t pk[BN / 2];
       const uint64_t scale2 = f2_pack(sl2, sl2), shift2 = f2_pack(-mb, -mb);
       uint64_t acc0 = 0, acc1 = 0;  // running row sums, two pairs of fp32 lanes
-      if (edge) {  // masked scores are -inf: MUFU ex2 only, which gives exact zeros
-#pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(sc[c], sc[c + 1]), scale2, shift2), x0, x1);
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          pk[c / 2] = pack_bf16x2(p0, p1);
-          if ((c / 2) & 1)
-            acc1 = f2_add(acc1, f2_pack(p0, p1));
-          else
-            acc0 = f2_add(acc0, f2_pack(p0, p1));
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          const uint64_t x2 = f2_fma(f2_pack(sc[c], sc[c + 1]), scale2, shift2);
-          float p0, p1;
-          if ((c / 2) % 8 < C::NPOLY) {
-            exp2_poly_pair(x2, p0, p1);
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
-          pk[c / 2] = pack_bf16x2(p0, p1);
-          if ((c / 2) & 1)
-            acc1 = f2_add(acc1, f2_pack(p0, p1));
-          else
-            acc0 = f2_add(acc0, f2_pack(p0, p1));
-        }
-      }
-      float rs0, rs1;
-      f2_unpack(f2_add(acc0, acc1), rs0, rs1);
-      l = l * alpha + (rs0 + rs1);
-#pragma unroll
-      for (int cc = 0; cc < BN / 64; ++cc) tmem_st_x32(lane_base + col_s + cc * 32, &pk[cc * 32]);
-      if constexpr (NQT == 1) {
-        // PV of the previous key tile must be complete before O is rescaled.
-        // The wait is taken at every step, not only when rescaling: a parity
-        // wait is only unambiguous while the barrier is at most one phase
-        // ahead of the waiter, and this keeps the waiter in lock step.
-        if (it > 0) {
-          ok = mbar_wait(&o_done[0], (it - 1) & 1, abort_flag, &g_status, p.wait_limit_ns);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
-        }
-      }
-      if (it > 0 && __any_sync(0xffffffffu, grow)) {
-        const uint32_t col_o = C::COL_O + t * D;
+      const uint32_t col_o = C::COL_O + t * D;
+      auto rescale_o = [&]() {
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t ov[32];
@@ -444,10 +451,59 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
           for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
           tmem_st_x32(lane_base + col_o + cc * 32, ov);
         }
+      };
+      if constexpr (C::SPLITP) {
+        // O of this tile is current (PV of the previous key tile completed
+        // before S of this one, which was committed after it): rescale it
+        // before the first half of P goes to the tensor core
+        if (it > 0 && __any_sync(0xffffffffu, grow)) rescale_o();
+        if (edge)
+          fwd_exp_cols<C, 0, BN / 2, true>(sc, scale2, shift2, pk, acc0, acc1);
+        else
+          fwd_exp_cols<C, 0, BN / 2, false>(sc, scale2, shift2, pk, acc0, acc1);
+#pragma unroll
+        for (int cc = 0; cc < BN / 128; ++cc) tmem_st_x32(lane_base + col_s + cc * 32, &pk[cc * 32]);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[2 * t]);
+        if (edge)
+          fwd_exp_cols<C, BN / 2, BN, true>(sc, scale2, shift2, pk, acc0, acc1);
+        else
+          fwd_exp_cols<C, BN / 2, BN, false>(sc, scale2, shift2, pk, acc0, acc1);
+#pragma unroll
+        for (int cc = BN / 128; cc < BN / 64; ++cc) tmem_st_x32(lane_base + col_s + cc * 32, &pk[cc * 32]);
+        float rs0, rs1;
+        f2_unpack(f2_add(acc0, acc1), rs0, rs1);
+        l = l * alpha + (rs0 + rs1);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[2 * t + 1]);
+      } else {
+        if (edge)
+          fwd_exp_cols<C, 0, BN, true>(sc, scale2, shift2, pk, acc0, acc1);
+        else
+          fwd_exp_cols<C, 0, BN, false>(sc, scale2, shift2, pk, acc0, acc1);
+        float rs0, rs1;
+        f2_unpack(f2_add(acc0, acc1), rs0, rs1);
+        l = l * alpha + (rs0 + rs1);
+#pragma unroll
+        for (int cc = 0; cc < BN / 64; ++cc) tmem_st_x32(lane_base + col_s + cc * 32, &pk[cc * 32]);
+        // NQT == 1: PV of the previous key tile must be complete before O is
+        // rescaled.  The wait is taken at every step, not only when
+        // rescaling: a parity wait is only unambiguous while the barrier is
+        // at most one phase ahead of the waiter, and this keeps the waiter in
+        // lock step.  (NQT == 2: that PV completed before S of this tile.)
+        if (NQT == 1 && it > 0) {
+          ok = mbar_wait(&o_done[0], (it - 1) & 1, abort_flag, &g_status, p.wait_limit_ns);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        if (it > 0 && __any_sync(0xffffffffu, grow)) rescale_o();
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[NQT == 2 ? 2 * t : slot]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[slot]);
     }
     // ---- epilogue: O / l -> bf16 -> shared (reusing this tile's Q buffer) -> TMA store
     if (ok && n_kv > 0) {
