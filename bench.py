@@ -47,6 +47,40 @@ WORKLOADS = {
 }
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch,
+# from the ncu capture summarised in the named profile file.  It is reported
+# only while the kernel sources hash to the ones that were profiled (a changed
+# kernel reports null until it is captured again).
+NCU_TRAFFIC = {
+    ("train", "bwd_dkdv"): dict(bytes=72.61e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
+    ("mid", "bwd_dkdv"): dict(bytes=377.65e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
+    ("mid", "bwd_dq"): dict(bytes=325.07e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
+    ("mid", "fwd"): dict(bytes=249.98e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
+}
+NCU_SOURCES_SHA256 = "239ab3f8074aa22e35940162d6829fd372368695f1c0024f11796d5d972b24ad"
+
+
+def sources_sha256():
+    """sha256 over the kernel sources (csrc/*.cu, *.cuh and include/fa.h)."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_89_b200", "csrc")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh")))
+    files.append(os.path.join(ROOT, "include", "fa.h"))
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(workload_key, kernel):
+    t = NCU_TRAFFIC.get((workload_key, kernel))
+    if t is None or sources_sha256() != NCU_SOURCES_SHA256:
+        return None, None
+    return t["bytes"], t["profile"]
+
+
 def fwd_flops(w):
     f = 4.0 * w["B"] * w["H"] * w["N"] * w["N"] * w["d"]
     return f / 2 if w["causal"] else f
@@ -154,6 +188,13 @@ def max_over_ranks(value, world):
                      device="cuda" if dist.get_backend() == "nccl" else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(flops_per_step, steps, t_ms_local, world):
+    """Whole-job TFLOP/s under weak scaling: every rank ran `steps` steps of
+    `flops_per_step` on its own batch; the job's time is the slowest rank's."""
+    t_max = max_over_ranks(t_ms_local, world)
+    return flops_per_step * steps * world / (t_max * 1e-3) / 1e12
 
 
 def barrier(world):
@@ -400,14 +441,10 @@ def run_ours(args, world, rank, local):
     peaks = load_peaks()
     w = WORKLOADS[args.workload]
     res = time_gpu(w, args.steps, args.warmup, world, rank, dev)
-    t_ms = sum(res["step_ms"])
-    t_max = max_over_ranks(t_ms, world)
     F = fwd_flops(w)
-    total = 3.5 * F * world * args.steps
-    value = total / (t_max * 1e-3) / 1e12
-    fwd_tf = F * world * args.steps / (max_over_ranks(sum(res["fwd_ms"]), world) * 1e-3) / 1e12
-    e2e_ms = max_over_ranks(sum(res["e2e_ms"]), world)
-    e2e_val = 3.5 * F * world * len(res["e2e_ms"]) / (e2e_ms * 1e-3) / 1e12
+    value = job_throughput(3.5 * F, args.steps, sum(res["step_ms"]), world)
+    fwd_tf = job_throughput(F, args.steps, sum(res["fwd_ms"]), world)
+    e2e_val = job_throughput(3.5 * F, len(res["e2e_ms"]), sum(res["e2e_ms"]), world)
     dom, per = roofline(w, res, peaks)
     launches = int(sum(res["trace_n"].values()))
 
@@ -417,10 +454,8 @@ def run_ours(args, world, rank, local):
         r2 = time_gpu(we, max(3, args.steps // 2), max(3, args.warmup), world, rank, dev,
                       with_e2e=False)
         F2 = fwd_flops(we)
-        tf2 = 3.5 * F2 * world * len(r2["step_ms"]) / (
-            max_over_ranks(sum(r2["step_ms"]), world) * 1e-3) / 1e12
-        ff2 = F2 * world * len(r2["fwd_ms"]) / (
-            max_over_ranks(sum(r2["fwd_ms"]), world) * 1e-3) / 1e12
+        tf2 = job_throughput(3.5 * F2, len(r2["step_ms"]), sum(r2["step_ms"]), world)
+        ff2 = job_throughput(F2, len(r2["fwd_ms"]), sum(r2["fwd_ms"]), world)
         d2, per2 = roofline(we, r2, peaks)
         extra.append({"workload": we["name"], "fwd_bwd_tflops": round(tf2, 2),
                       "fwd_tflops": round(ff2, 2),
@@ -437,6 +472,7 @@ def run_ours(args, world, rank, local):
         cpu = {"value": round(tf_c, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": "%d of %d heads, full N, fwd+bwd, %.1f s" % (heads, w["B"] * w["H"], secs)}
     dk = per.get(dom, {}) if dom else {}
+    traffic, traffic_profile = ncu_traffic(args.workload, dom)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -452,7 +488,7 @@ def run_ours(args, world, rank, local):
         "fwd_pct_dense_peak": round(100 * fwd_tf / (world * DENSE_PEAK_TFLOPS), 2),
         "roofline": {"kernel": dom, "bound": dk.get("bound"), "achieved": dk.get("achieved"),
                      "peak": dk.get("peak"), "unit": dk.get("unit"), "frac": dk.get("frac"),
-                     "traffic": None,
+                     "traffic": traffic, "traffic_profile": traffic_profile,
                      "peak_source": "%s, %s" % (peaks["source"],
                                                 "sustained" if dk.get("bound") == "tensor" else "copy")},
         "kernels": per,

@@ -1,0 +1,105 @@
+"""Host-side logic of bench.py, on the CPU: the FLOP accounting, the roofline
+bookkeeping, the ncu-traffic gate, and the multi-process path (two gloo ranks:
+max over ranks, weak-scaling throughput, barrier, reference arm on rank 0 only).
+"""
+import os
+import socket
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_flop_accounting_matches_the_metric():
+    w = bench.WORKLOADS["train"]
+    F = bench.fwd_flops(w)
+    assert F == 4 * 2 * 16 * 2048 * 2048 * 128 / 2
+    alg = bench.kernel_algorithmic(w)
+    tensor = sum(work for kind, (bound, work) in alg.items() if bound == "tensor")
+    assert tensor == pytest.approx(3.5 * F)  # forward + 2.5x for the backward
+    assert alg["bwd_prep"][0] == "hbm"
+
+
+def test_roofline_picks_the_longest_kernel_and_uses_the_measured_peak():
+    w = bench.WORKLOADS["train"]
+    F = bench.fwd_flops(w)
+    res = {"trace_ms": {"fwd": 1.0, "bwd_dkdv": 3.0, "bwd_dq": 2.0, "bwd_prep": 0.5},
+           "trace_n": {"fwd": 10, "bwd_dkdv": 10, "bwd_dq": 10, "bwd_prep": 10}}
+    peaks = dict(hbm_gbs=6000.0, bf16=1600.0, bf16_sustained=1400.0, source="test")
+    dom, per = bench.roofline(w, res, peaks)
+    assert dom == "bwd_dkdv"
+    assert per["bwd_dkdv"]["achieved"] == pytest.approx(2 * F / 0.3e-3 / 1e12, rel=1e-3)
+    assert per["bwd_dkdv"]["peak"] == 1400.0
+    assert per["bwd_dkdv"]["frac"] == pytest.approx(per["bwd_dkdv"]["achieved"] / 1400.0, abs=1e-4)
+    assert sum(p["share"] for p in per.values()) == pytest.approx(1.0, abs=1e-3)
+    assert per["bwd_prep"]["unit"] == "GB/s"
+
+
+def test_ncu_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
+    monkeypatch.setattr(bench, "NCU_SOURCES_SHA256", bench.sources_sha256())
+    b, prof = bench.ncu_traffic("train", "bwd_dkdv")
+    assert b > 0 and os.path.exists(os.path.join(ROOT, prof))
+    monkeypatch.setattr(bench, "NCU_SOURCES_SHA256", "0" * 64)
+    assert bench.ncu_traffic("train", "bwd_dkdv") == (None, None)
+    monkeypatch.setattr(bench, "NCU_SOURCES_SHA256", bench.sources_sha256())
+    assert bench.ncu_traffic("train", "no_such_kernel") == (None, None)
+
+
+def test_profiles_named_in_the_traffic_table_exist():
+    for (wl, kern), t in bench.NCU_TRAFFIC.items():
+        assert wl in bench.WORKLOADS
+        assert os.path.exists(os.path.join(ROOT, t["profile"])), t["profile"]
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # rank r's loop took (r + 1) * 10 ms for 5 steps of 1e12 FLOP each
+        t_local = (rank + 1) * 10.0
+        tmax = bench.max_over_ranks(t_local, world)
+        tf = bench.job_throughput(1e12, 5, t_local, world)
+        bench.barrier(world)
+        q.put((rank, tmax, tf))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_on_max_time_and_job_throughput():
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    world, port = 2, _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, tmax, tf in out:
+        assert tmax == 20.0                      # the slowest rank's time
+        assert tf == pytest.approx(1e12 * 5 * 2 / 20e-3 / 1e12)  # all ranks' work / max time
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    called = []
+    monkeypatch.setattr(bench, "oracle_sample", lambda *a, **k: called.append(1) or (1.0, 1, 1.0, 1))
+
+    class A:
+        workload, steps, warmup = "train", 3, 3
+    bench.run_reference(A(), world=2, rank=1)
+    assert called == [] and capsys.readouterr().out == ""
