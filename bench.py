@@ -434,6 +434,117 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ sweep
+
+def sweep_workloads():
+    """The sequence-length sweep (N in 512..16k, d in {64, 128}, hidden 2048 so
+    H = 2048 / d, batch 16384 / N, causal and not), then the GQA + window and
+    the d = 256 workloads."""
+    from seeded_inputs import config_seed, sweep_seed
+    out = []
+    for d in (64, 128):
+        for N in (512, 1024, 2048, 4096, 8192, 16384):
+            for causal in (False, True):
+                out.append(dict(name="sweep N=%d d=%d %s" % (N, d, "causal" if causal else "non-causal"),
+                                B=16384 // N, N=N, H=2048 // d, Hkv=2048 // d, d=d, causal=causal,
+                                window=(-1, -1), seed=sweep_seed(N, d)))
+    out.append(dict(name="GQA + window B=1 Hq=32 Hkv=8 N=8192 d=128 causal window (4096, 0)",
+                    B=1, N=8192, H=32, Hkv=8, d=128, causal=True, window=(4096, 0), seed=config_seed(4)))
+    out.append(dict(name="long wide d=256 B=1 H=16 N=16384 causal", B=1, N=16384, H=16, Hkv=16, d=256,
+                    causal=True, window=(-1, -1), seed=config_seed(5) + 50))
+    return out
+
+
+def visible_pairs(w):
+    """Number of visible (query, key) pairs per (batch, head) under the mask."""
+    N = w["N"]
+    wl, wr = w["window"]
+    wr = 0 if w["causal"] else wr
+    i = range(N)
+    hi = [N - 1 if wr < 0 else min(N - 1, r + wr) for r in i]
+    lo = [0 if wl < 0 else max(0, r - wl) for r in i]
+    return sum(max(0, h - l + 1) for h, l in zip(hi, lo))
+
+
+def time_modes(w, steps, warmup, dev):
+    """Median ms of fa_fwd alone, fa_bwd alone and fa_fwd + fa_bwd (L2 flushed
+    before every timed call, CUDA events on the launching stream)."""
+    import torch
+    import exact_io_aware_89_b200 as fa
+    x, _ = make_device_inputs(w, 0, dev)
+    q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+    B, N, H, Hkv, d = w["B"], w["N"], w["H"], w["Hkv"], w["d"]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(16, fa.fa_bwd_workspace_size(B, N, H, d)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sp = torch.cuda.current_stream().cuda_stream
+    scale = 1.0 / math.sqrt(d)
+    c, (wl, wr) = int(w["causal"]), w["window"]
+
+    def fwd():
+        st = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                       B, N, N, H, Hkv, d, scale, c, wl, wr, sp)
+        if st:
+            raise fa.FAError("fa_fwd", st)
+
+    def bwd():
+        st = fa.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                       do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, N, H, Hkv,
+                       d, scale, c, wl, wr, ws.data_ptr(), ws.numel(), sp)
+        if st:
+            raise fa.FAError("fa_bwd", st)
+
+    def both():
+        fwd()
+        bwd()
+
+    out = {}
+    for mode, fn in (("fwd", fwd), ("bwd", bwd), ("fwd_bwd", both)):
+        for _ in range(warmup):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record()
+            fn()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        out[mode] = statistics.median(a.elapsed_time(b) for a, b in ev)
+    if fa.fa_get_device_status(None) != 0:
+        raise RuntimeError("device status reports a timed-out wait")
+    del flush, x
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_sweep(args, local):
+    """One JSON line per workload of the sweep: fwd, bwd and fwd+bwd timed
+    separately, TFLOP/s by the metric's formula (forward 4 B H N^2 d, halved
+    when causal; backward 2.5x; fwd+bwd 3.5x), and, for a window, also by the
+    visible pairs (4 B H pairs d)."""
+    import torch
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    for w in sweep_workloads():
+        t = time_modes(w, args.steps, args.warmup, dev)
+        F = fwd_flops(w)
+        line = {"sweep": w["name"], "B": w["B"], "H": w["H"], "Hkv": w["Hkv"], "N": w["N"], "d": w["d"],
+                "causal": w["causal"], "window": list(w["window"]),
+                "ms": {m: round(v, 4) for m, v in t.items()},
+                "tflops": {"fwd": round(F / t["fwd"] / 1e9, 1), "bwd": round(2.5 * F / t["bwd"] / 1e9, 1),
+                           "fwd_bwd": round(3.5 * F / t["fwd_bwd"] / 1e9, 1)}}
+        line["pct_dense_peak"] = {m: round(100 * v / DENSE_PEAK_TFLOPS, 2) for m, v in line["tflops"].items()}
+        if w["window"] != (-1, -1):
+            Fv = 4.0 * w["B"] * w["H"] * visible_pairs(w) * w["d"]
+            line["tflops_visible_pairs"] = {"fwd": round(Fv / t["fwd"] / 1e9, 1),
+                                            "bwd": round(2.5 * Fv / t["bwd"] / 1e9, 1),
+                                            "fwd_bwd": round(3.5 * Fv / t["fwd_bwd"] / 1e9, 1)}
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank, local):
     import torch
     dev = torch.device("cuda", local)
@@ -513,10 +624,18 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-budget", type=float, default=15.0,
                     help="seconds of oracle time for the CPU baseline sample")
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the benchmark line: the sequence-length sweep and the GQA/window "
+                         "and d=256 workloads, fwd / bwd / fwd+bwd timed separately, one JSON line each")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     world, rank, local = dist_setup(args)
+    if args.sweep:
+        if world > 1:
+            raise SystemExit("--sweep runs on one GPU")
+        run_sweep(args, local)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)  # rank 0 alone; no process group
         return

@@ -103,3 +103,26 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
         workload, steps, warmup = "train", 3, 3
     bench.run_reference(A(), world=2, rank=1)
     assert called == [] and capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("N,causal,window", [(7, False, (-1, -1)), (7, True, (-1, -1)), (9, True, (3, 0)),
+                                              (9, False, (2, 1)), (5, False, (0, 0))])
+def test_visible_pairs_counts_the_mask(N, causal, window):
+    # brute force over the visibility rule (Nq = Nk: no bottom-right offset)
+    wl, wr = window
+    wr = 0 if causal else wr
+    n = sum(1 for i in range(N) for j in range(N)
+            if (wr < 0 or j <= i + wr) and (wl < 0 or j >= i - wl))
+    assert bench.visible_pairs(dict(N=N, causal=causal, window=window)) == n
+
+
+def test_sweep_covers_the_sequence_length_grid():
+    ws = bench.sweep_workloads()
+    grid = {(w["N"], w["d"], w["causal"]) for w in ws if w["window"] == (-1, -1) and w["d"] in (64, 128)}
+    for N in (512, 1024, 2048, 4096, 8192, 16384):
+        for d in (64, 128):
+            for c in (False, True):
+                assert (N, d, c) in grid
+    for w in ws:
+        if w["name"].startswith("sweep"):
+            assert w["B"] * w["N"] == 16384 and w["H"] * w["d"] == 2048
