@@ -159,11 +159,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   const int Nq_pad = pad_rows(Nq);
   const long long rows_pad = static_cast<long long>(B) * Hq * Nq_pad;
   {
-    const long long blocks = (rows_pad * 32 + 255) / 256;
+    constexpr int G = D / 8;  // lanes per row (16-byte loads)
+    constexpr int RPG = 4;    // rows per lane group
+    const long long blocks = (rows_pad * G / RPG + 255) / 256;
     TraceScope tr(FA_KERNEL_BWD_PREP, stream);
-    fa_bwd_prep_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+    fa_bwd_prep_bf16_kernel<G, RPG><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, ws, B, Nq,
-        Hq, D, Nq_pad);
+        Hq, Nq_pad);
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
   BwdParams p;

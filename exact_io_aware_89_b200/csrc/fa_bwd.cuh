@@ -10,7 +10,7 @@
 //   dV_j  = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j
 //
 // Three launches on the caller's stream:
-//   1. fa_bwd_prep_kernel : D_i and lse2_i = LSE_i * log2(e) into the workspace
+//   1. fa_bwd_prep_*      : D_i and lse2_i = LSE_i * log2(e) into the workspace
 //                           (rows padded to a multiple of 256; padding rows get
 //                           lse2 = +inf so every P there is exactly 0).
 //   2. fa_bwd_dq_kernel   : query-stationary.  Per key tile: S = Q K^T and
@@ -33,18 +33,8 @@ namespace fa {
 // =====================================================================
 // 1. preprocess: D = rowsum(dO * O), lse2 = LSE * log2(e)
 // =====================================================================
-template <typename T>
-__device__ __forceinline__ float load_as_float(const T* p);
-template <>
-__device__ __forceinline__ float load_as_float<float>(const float* p) {
-  return *p;
-}
-template <>
-__device__ __forceinline__ float load_as_float<__nv_bfloat16>(const __nv_bfloat16* p) {
-  return __bfloat162float(*p);
-}
-
-// one warp per (b, i, h) row; ws layout: D [B, Hq, Nq_pad] then lse2 [B, Hq, Nq_pad]
+// fp32 inputs (the fp32 entry points): one warp per (b, i, h) row; ws layout:
+// D [B, Hq, Nq_pad] then lse2 [B, Hq, Nq_pad]
 template <typename T>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const T* __restrict__ o,
                                                           const T* __restrict__ dout,
@@ -70,7 +60,7 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const T* __restrict__ 
   }
   const size_t base = ((static_cast<size_t>(b) * Nq + i) * Hq + h) * d;
   float acc = 0.f;
-  for (int c = lane; c < d; c += 32) acc += load_as_float(o + base + c) * load_as_float(dout + base + c);
+  for (int c = lane; c < d; c += 32) acc += static_cast<float>(o[base + c]) * static_cast<float>(dout[base + c]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) {
@@ -78,6 +68,70 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const T* __restrict__ 
     const float L = lse[(static_cast<size_t>(b) * Hq + h) * Nq + i];
     // a row with no visible key (LSE = -inf) has P = 0 everywhere
     *L2p = (L == -INFINITY) ? INFINITY : L * kLog2e;
+  }
+}
+
+// bf16: G = d / 8 lanes per row, each loading 8 elements of O and of dO with
+// one 16-byte load; the G partial dot products are added with shuffles inside
+// the lane group (groups are aligned within the warp, G divides 32).  Each
+// lane group handles RPG rows, with all their loads issued before any use, so
+// that enough bytes are in flight to approach HBM bandwidth.  Same outputs
+// and layout as fa_bwd_prep_kernel; rows_pad must be a multiple of
+// RPG * 256 / G (it is a multiple of 256).
+template <int G, int RPG>
+__global__ void __launch_bounds__(256) fa_bwd_prep_bf16_kernel(const __nv_bfloat16* __restrict__ o,
+                                                               const __nv_bfloat16* __restrict__ dout,
+                                                               const float* __restrict__ lse,
+                                                               float* __restrict__ ws, int B, int Nq,
+                                                               int Hq, int Nq_pad) {
+  static_assert(G == 8 || G == 16 || G == 32, "d = 64, 128 or 256");
+  constexpr int D = G * 8;
+  constexpr int GROUPS = 256 / G;  // lane groups per block
+  const int grp = threadIdx.x / G;
+  const int sub = threadIdx.x % G;
+  const long long rows_pad = static_cast<long long>(B) * Hq * Nq_pad;
+  uint4 ov[RPG], gv[RPG];
+  long long row[RPG];
+  bool live[RPG];
+#pragma unroll
+  for (int k = 0; k < RPG; ++k) {
+    row[k] = (static_cast<long long>(blockIdx.x) * RPG + k) * GROUPS + grp;
+    const int i = static_cast<int>(row[k] % Nq_pad);
+    const long long bh = row[k] / Nq_pad;
+    live[k] = row[k] < rows_pad && i < Nq;
+    if (live[k]) {
+      const size_t base = ((static_cast<size_t>(bh / Hq) * Nq + i) * Hq + bh % Hq) * D + sub * 8;
+      ov[k] = __ldg(reinterpret_cast<const uint4*>(o + base));
+      gv[k] = __ldg(reinterpret_cast<const uint4*>(dout + base));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < RPG; ++k) {
+    float acc = 0.f;
+    if (live[k]) {
+      const uint32_t* op = reinterpret_cast<const uint32_t*>(&ov[k]);
+      const uint32_t* gp = reinterpret_cast<const uint32_t*>(&gv[k]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        // a bf16 is the top half of an fp32
+        acc = fmaf(__uint_as_float(op[u] << 16), __uint_as_float(gp[u] << 16), acc);
+        acc = fmaf(__uint_as_float(op[u] & 0xFFFF0000u), __uint_as_float(gp[u] & 0xFFFF0000u), acc);
+      }
+    }
+#pragma unroll
+    for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (sub == 0 && row[k] < rows_pad) {
+      const int i = static_cast<int>(row[k] % Nq_pad);
+      if (i >= Nq) {  // padding row: D = 0 and lse2 = +inf, so every P there is 0
+        ws[row[k]] = 0.f;
+        ws[rows_pad + row[k]] = INFINITY;
+      } else {
+        ws[row[k]] = acc;
+        const float L = lse[(row[k] / Nq_pad) * Nq + i];
+        // a row with no visible key (LSE = -inf) has P = 0 everywhere
+        ws[rows_pad + row[k]] = (L == -INFINITY) ? INFINITY : L * kLog2e;
+      }
+    }
   }
 }
 
