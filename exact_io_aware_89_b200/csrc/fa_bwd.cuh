@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       for (int c = 0; c < C::NCHUNK; ++c)
         tma_store_4d(&tm_dq, stage + c * C::QCHUNK, c * 64, h, r0 + t * BM, b);
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read();
     }
   }
 
@@ -726,7 +726,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     if (threadIdx.x == 0 && *abort_flag == 0 && r0 < p.Nq) {
       for (int c = 0; c < C::NCHUNK; ++c) tma_store_4d(&tm_dq, sQ + c * C::QCHUNK, c * 64, h, r0, b);
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read();
     }
   }
 
@@ -1052,7 +1052,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
         tma_store_4d(&tm_dv, sV + c * C::KCHUNK, x, hk, k0, b);
       }
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read();
     }
   }
 

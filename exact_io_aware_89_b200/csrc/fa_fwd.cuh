@@ -193,7 +193,28 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int j_begin = key_lo / BN;
   const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
 
-  if (threadIdx.x == 0) {
+  // Copies of key tile `it` into ring stage it % KST (K and V on one barrier
+  // with two Q tiles, on their own barriers with one)
+  auto load_k = [&](int it) {
+    const int s = it % KST, krow = (j_begin + it) * BN;
+    uint64_t* bar = &k_full[s];
+    mbar_expect_tx(bar, (NQT == 2 ? 2 : 1) * C::KTILE);
+    for (int c = 0; c < C::NCHUNK; ++c) {
+      tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, bar, c * 64, hk, krow, b);
+      if (NQT == 2) tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, bar, c * 64, hk, krow, b);
+    }
+  };
+  auto load_v = [&](int it) {  // NQT == 1 only
+    const int s = it % KST, krow = (j_begin + it) * BN;
+    mbar_expect_tx(&v_full[s], C::KTILE);
+    for (int c = 0; c < C::NCHUNK; ++c)
+      tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[s], c * 64, hk, krow, b);
+  };
+  // The TMA thread sets up the barriers and issues Q and the first KST key
+  // tiles (no stage to wait for yet) before the block-wide sync, so the
+  // copies overlap the TMEM allocation and the sync.
+  const int n_pre = min(n_kv, KST);
+  if (warp == C::TMA_WARP && lane == 0) {
     mbar_init(bar_q, 1);
     for (int s = 0; s < KST; ++s) {
       mbar_init(&k_full[s], 1);
@@ -209,16 +230,21 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    if (n_kv > 0) {
+      mbar_expect_tx(bar_q, NQT * C::QTILE);
+      for (int t = 0; t < NQT; ++t)
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_load_4d(sQ + t * C::QTILE + c * C::QCHUNK, &tm_q, bar_q, c * 64, h, r0 + t * BM, b);
+      for (int it = 0; it < n_pre; ++it) {
+        load_k(it);
+        if (NQT == 1) load_v(it);
+      }
+    }
+    tma_prefetch_desc(&tm_o);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
-  }
-  if (warp == C::TMA_WARP && lane == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_o);
   }
   tc_fence_before();
   __syncthreads();
@@ -229,37 +255,18 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     // ------------------------------------------------------------ producer
     setmaxnreg_dec<C::REG_PRODUCER>();
     if (lane == 0 && n_kv > 0) {
-      mbar_expect_tx(bar_q, NQT * C::QTILE);
-      for (int t = 0; t < NQT; ++t)
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sQ + t * C::QTILE + c * C::QCHUNK, &tm_q, bar_q, c * 64, h, r0 + t * BM, b);
-      int nk = 0, nv = 0;
-      for (int it = 0; it < n_kv; ++it) {
+      // Q and key tiles 0 .. n_pre-1 were issued before the block-wide sync
+      int nk = n_pre, nv = NQT == 1 ? n_pre : 0;
+      for (int it = n_pre; it < n_kv; ++it) {
         const int s = it % KST, use = it / KST;
-        const int krow = (j_begin + it) * BN;
-        if constexpr (NQT == 2) {
-          // K_j and V_j share a stage and its full barrier; the stage is free
-          // once the last PV of the previous tile in it has completed
-          if (use > 0 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
-            break;
-          mbar_expect_tx(&k_full[s], 2 * C::KTILE);
-          for (int c = 0; c < C::NCHUNK; ++c) {
-            tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[s], c * 64, hk, krow, b);
-            tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &k_full[s], c * 64, hk, krow, b);
-          }
-          ++nk;
-        } else {
-          if (use > 0 && !mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
-            break;
-          mbar_expect_tx(&k_full[s], C::KTILE);
-          for (int c = 0; c < C::NCHUNK; ++c)
-            tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[s], c * 64, hk, krow, b);
-          ++nk;
-          if (use > 0 && !mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
-            break;
-          mbar_expect_tx(&v_full[s], C::KTILE);
-          for (int c = 0; c < C::NCHUNK; ++c)
-            tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[s], c * 64, hk, krow, b);
+        // the stage is free once the last MMA reading the tile held there
+        // before has completed (NQT == 2: K_j and V_j share the stage)
+        if (!mbar_wait(&k_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns)) break;
+        load_k(it);
+        ++nk;
+        if constexpr (NQT == 1) {
+          if (!mbar_wait(&v_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns)) break;
+          load_v(it);
           ++nv;
         }
       }
@@ -545,7 +552,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       for (int c = 0; c < C::NCHUNK; ++c)
         tma_store_4d(&tm_o, sQt + c * C::QCHUNK, c * 64, h, r0 + t * BM, b);
       tma_store_commit();
-      tma_store_wait_all();
+      tma_store_wait_read();
     }
     if (!aborted && row < p.Nq) {
       const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;

@@ -142,8 +142,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 __device__ __forceinline__ void tma_store_commit() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-__device__ __forceinline__ void tma_store_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+// Waits until every committed bulk store has finished reading its shared
+// memory source (the global writes complete on their own; a kernel's writes
+// are visible once it has finished).  Enough before shared memory is reused
+// or the CTA exits.
+__device__ __forceinline__ void tma_store_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 // generic-proxy smem writes -> visible to the async proxy (TMA store, MMA)
 __device__ __forceinline__ void fence_proxy_async_smem() {
