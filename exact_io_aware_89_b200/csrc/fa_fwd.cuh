@@ -340,6 +340,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
             if (more) {
               issue_s(0, 0, s1);
               tc_commit(&s_full[0]);
+            } else {
+              tc_commit(&o_done[0]);  // tile 0's epilogue may start
             }
             if (!(ok = wait(&p_full[2], par))) break;
             if constexpr (C::SPLITP) {
@@ -353,9 +355,10 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
             if (more) {
               issue_s(1, 1, s1);
               tc_commit(&s_full[1]);
+            } else {
+              tc_commit(&o_done[1]);
             }
           }
-          if (ok) tc_commit(&o_done[0]);
         } else {
           // one Q tile: S slots alternate between consecutive key tiles
           issue_s(0, 0, 0);
@@ -514,9 +517,10 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
     // ---- epilogue: O / l -> bf16 -> shared (reusing this tile's Q buffer) -> TMA store
     if (ok && n_kv > 0) {
-      // NQT == 2: one commit after the last PV of both tiles (phase 0);
+      // NQT == 2: one commit per tile after its last PV (phase 0), so each
+      // tile's epilogue starts as soon as its own O is final;
       // NQT == 1: one commit per PV, the last one is phase n_kv - 1
-      ok = mbar_wait(&o_done[0], NQT == 2 ? 0u : static_cast<uint32_t>((n_kv - 1) & 1), abort_flag,
+      ok = mbar_wait(&o_done[NQT == 2 ? t : 0], NQT == 2 ? 0u : static_cast<uint32_t>((n_kv - 1) & 1), abort_flag,
                      &g_status, p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
