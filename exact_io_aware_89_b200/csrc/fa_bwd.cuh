@@ -517,7 +517,23 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int j_begin = key_lo / BN;
   const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
 
-  if (threadIdx.x == 0) {
+  // copies of K or V of key tile `it` into their rings
+  auto load_k = [&](int it) {
+    const int sk = it % KS, krow = (j_begin + it) * BN;
+    mbar_expect_tx(&k_full[sk], C::KTILE);
+    for (int c = 0; c < C::NCHUNK; ++c)
+      tma_load_4d(sK + sk * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[sk], c * 64, hk, krow, b);
+  };
+  auto load_v = [&](int it) {
+    const int sv = it % VS, krow = (j_begin + it) * BN;
+    mbar_expect_tx(&v_full[sv], C::KTILE);
+    for (int c = 0; c < C::NCHUNK; ++c)
+      tma_load_4d(sV + sv * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[sv], c * 64, hk, krow, b);
+  };
+  // The TMA thread sets up the barriers and issues Q, dO and the first ring
+  // stages (nothing to wait for yet) before the block-wide sync.
+  const int n_pre_k = min(n_kv, KS), n_pre_v = min(n_kv, VS);
+  if (warp == C::TMA_WARP && lane == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < KS; ++s) {
       mbar_init(&k_full[s], 1);
@@ -535,6 +551,15 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    if (n_kv > 0) {
+      mbar_expect_tx(q_full, 2 * C::QTILE);
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        tma_load_4d(sQ + c * C::QCHUNK, &tm_q, q_full, c * 64, h, r0, b);
+        tma_load_4d(sdO + c * C::QCHUNK, &tm_do, q_full, c * 64, h, r0, b);
+      }
+      for (int it = 0; it < n_pre_k; ++it) load_k(it);
+      for (int it = 0; it < n_pre_v; ++it) load_v(it);
+    }
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
@@ -547,27 +572,20 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 
   if (warp == C::TMA_WARP) {
     if (lane == 0 && n_kv > 0) {
-      mbar_expect_tx(q_full, 2 * C::QTILE);
-      for (int c = 0; c < C::NCHUNK; ++c) {
-        tma_load_4d(sQ + c * C::QCHUNK, &tm_q, q_full, c * 64, h, r0, b);
-        tma_load_4d(sdO + c * C::QCHUNK, &tm_do, q_full, c * 64, h, r0, b);
-      }
-      int nk = 0, nv = 0;
+      int nk = n_pre_k, nv = n_pre_v;
       for (int it = 0; it < n_kv; ++it) {
-        const int sk = it % KS, uk = it / KS, sv = it % VS, uv = it / VS;
-        const int krow = (j_begin + it) * BN;
-        if (uk > 0 && !mbar_wait(&k_empty[sk], (uk - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
-          break;
-        mbar_expect_tx(&k_full[sk], C::KTILE);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sK + sk * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[sk], c * 64, hk, krow, b);
-        ++nk;
-        if (uv > 0 && !mbar_wait(&v_empty[sv], (uv - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
-          break;
-        mbar_expect_tx(&v_full[sv], C::KTILE);
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sV + sv * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[sv], c * 64, hk, krow, b);
-        ++nv;
+        if (it >= n_pre_k) {
+          const int sk = it % KS, uk = it / KS;
+          if (!mbar_wait(&k_empty[sk], (uk - 1) & 1, abort_flag, &g_status, p.wait_limit_ns)) break;
+          load_k(it);
+          ++nk;
+        }
+        if (it >= n_pre_v) {
+          const int sv = it % VS, uv = it / VS;
+          if (!mbar_wait(&v_empty[sv], (uv - 1) & 1, abort_flag, &g_status, p.wait_limit_ns)) break;
+          load_v(it);
+          ++nv;
+        }
       }
       mbar_drain(q_full, 0, p.wait_limit_ns);
       for (int s = 0; s < KS; ++s)
@@ -818,7 +836,28 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int n_qt = (q_hi >= q_lo) ? (q_hi / BM - i_begin + 1) : 0;
   const int n_steps = n_qt * p.group;  // (query head in group) x (query tile)
 
-  if (threadIdx.x == 0) {
+  auto step_head = [&](int step) { return hk * p.group + step / n_qt; };
+  auto step_q0 = [&](int step) { return (i_begin + step % n_qt) * BM; };
+  // copies of step `it` (Q, dO and their lse2 / D rows) into stage it % ST
+  auto load_step = [&](int it) {
+    const int s = it % ST;
+    const int hq = step_head(it), q0 = step_q0(it);
+    const uint32_t st = sSt + s * C::STAGE;
+    mbar_expect_tx(&q_full[s], C::STAGE + C::SSTAGE);
+    for (int c = 0; c < C::NCHUNK; ++c) {
+      tma_load_4d(st + c * C::QCHUNK, &tm_q, &q_full[s], c * 64, hq, q0, b);
+      tma_load_4d(st + C::QTILE + c * C::QCHUNK, &tm_do, &q_full[s], c * 64, hq, q0, b);
+    }
+    const size_t srow = (static_cast<size_t>(b) * p.Hq + hq) * p.Nq_pad + q0;
+    const uint32_t stat = sbase + C::OFF_STAT + s * C::SSTAGE;
+    bulk_load(stat, p.lse2 + srow, BM * 4, &q_full[s]);
+    bulk_load(stat + BM * 4, p.D + srow, BM * 4, &q_full[s]);
+  };
+  // The TMA thread sets up the barriers and issues K, V and the first ST
+  // steps (no stage to wait for yet) before the block-wide sync, so the
+  // copies overlap the TMEM allocation and the sync.
+  const int n_pre = min(n_steps, ST);
+  if (warp == C::TMA_WARP && lane == 0) {
     mbar_init(kv_full, 1);
     for (int s = 0; s < ST; ++s) {
       mbar_init(&q_full[s], 1);
@@ -832,6 +871,14 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    if (n_steps > 0) {
+      mbar_expect_tx(kv_full, 2 * C::KTILE);
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        tma_load_4d(sK + c * C::KCHUNK, &tm_k, kv_full, c * 64, hk, k0, b);
+        tma_load_4d(sV + c * C::KCHUNK, &tm_v, kv_full, c * 64, hk, k0, b);
+      }
+      for (int it = 0; it < n_pre; ++it) load_step(it);
+    }
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
@@ -842,32 +889,13 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  auto step_head = [&](int step) { return hk * p.group + step / n_qt; };
-  auto step_q0 = [&](int step) { return (i_begin + step % n_qt) * BM; };
-
   if (warp == C::TMA_WARP) {
     if (lane == 0 && n_steps > 0) {
-      mbar_expect_tx(kv_full, 2 * C::KTILE);
-      for (int c = 0; c < C::NCHUNK; ++c) {
-        tma_load_4d(sK + c * C::KCHUNK, &tm_k, kv_full, c * 64, hk, k0, b);
-        tma_load_4d(sV + c * C::KCHUNK, &tm_v, kv_full, c * 64, hk, k0, b);
-      }
-      int n_issued = 0;
-      for (int it = 0; it < n_steps; ++it) {
+      int n_issued = n_pre;
+      for (int it = n_pre; it < n_steps; ++it) {
         const int s = it % ST, use = it / ST;
-        if (use > 0 && !mbar_wait(&q_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
-          break;
-        const int hq = step_head(it), q0 = step_q0(it);
-        const uint32_t st = sSt + s * C::STAGE;
-        mbar_expect_tx(&q_full[s], C::STAGE + C::SSTAGE);
-        for (int c = 0; c < C::NCHUNK; ++c) {
-          tma_load_4d(st + c * C::QCHUNK, &tm_q, &q_full[s], c * 64, hq, q0, b);
-          tma_load_4d(st + C::QTILE + c * C::QCHUNK, &tm_do, &q_full[s], c * 64, hq, q0, b);
-        }
-        const size_t srow = (static_cast<size_t>(b) * p.Hq + hq) * p.Nq_pad + q0;
-        const uint32_t stat = sbase + C::OFF_STAT + s * C::SSTAGE;
-        bulk_load(stat, p.lse2 + srow, BM * 4, &q_full[s]);
-        bulk_load(stat + BM * 4, p.D + srow, BM * 4, &q_full[s]);
+        if (!mbar_wait(&q_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns)) break;
+        load_step(it);
         ++n_issued;
       }
       mbar_drain(kv_full, 0, p.wait_limit_ns);
