@@ -52,12 +52,12 @@ WORKLOADS = {
 # only while the kernel sources hash to the ones that were profiled (a changed
 # kernel reports null until it is captured again).
 NCU_TRAFFIC = {
-    ("train", "bwd_dkdv"): dict(bytes=72.61e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
-    ("mid", "bwd_dkdv"): dict(bytes=377.65e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
-    ("mid", "bwd_dq"): dict(bytes=325.07e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
-    ("mid", "fwd"): dict(bytes=249.98e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
+    ("train", "bwd_dkdv"): dict(bytes=72.68e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
+    ("mid", "bwd_dkdv"): dict(bytes=378.44e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
+    ("mid", "bwd_dq"): dict(bytes=326.29e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
+    ("mid", "fwd"): dict(bytes=252.54e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
 }
-NCU_SOURCES_SHA256 = "239ab3f8074aa22e35940162d6829fd372368695f1c0024f11796d5d972b24ad"
+NCU_SOURCES_SHA256 = "f62d04c24b51c15fc18228ee502c792a8957027481233d600f21f5c487b1683f"
 
 
 def sources_sha256():
