@@ -10,8 +10,8 @@ causal) that the throughput target names is measured alongside it under
 forward+backward = 3.5x forward.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
-on the launching stream with a 256 MiB write between steps to flush L2
-(outside the events); barrier + synchronize around the loop; with N > 1
+on the launching stream, with L2 flushed between steps outside the events (a
+256 MiB write, then a 256 MiB read so the lines left in L2 are clean); barrier + synchronize around the loop; with N > 1
 processes (torchrun) every rank runs its own batch (weak scaling, no
 collective on the data path) and the time is the max over ranks.  Rank 0
 prints one JSON line.
@@ -95,6 +95,23 @@ def load_peaks():
                     bf16_sustained=float(p["bf16_tflops_sustained"]), source="measured")
     except Exception:
         return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class L2Flush:
+    """Evicts the step's inputs from the 126 MB L2 between timed calls: a
+    256 MiB write, then a 256 MiB read of another buffer.  The read leaves L2
+    holding clean lines, as it would after ordinary work; after the write
+    alone, L2 is full of dirty lines whose write-back (about 15 us of HBM
+    time) would land inside the next timed call."""
+
+    def __init__(self, dev):
+        import torch
+        self.dirty = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.clean = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.dirty.zero_()
+        self.clean.sum()
 
 
 # ------------------------------------------------------------------ clocks
@@ -223,7 +240,7 @@ def time_gpu(w, steps, warmup, world, rank, dev, with_e2e=True, with_trace=True)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(max(16, fa.fa_bwd_workspace_size(B, N, H, d)), dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
     scale = 1.0 / math.sqrt(d)
@@ -262,7 +279,7 @@ def time_gpu(w, steps, warmup, world, rank, dev, with_e2e=True, with_trace=True)
     torch.cuda.synchronize()
     with ClockSampler(dev) as clocks:
         for i in range(steps):
-            flush.zero_()
+            flush()
             ev[i][0].record(stream)
             step(q, k, v, do)
             ev[i][1].record(stream)
@@ -277,7 +294,7 @@ def time_gpu(w, steps, warmup, world, rank, dev, with_e2e=True, with_trace=True)
     fev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(steps)]
     for i in range(steps):
-        flush.zero_()
+        flush()
         fev[i][0].record(stream)
         fwd_only()
         fev[i][1].record(stream)
@@ -478,7 +495,7 @@ def time_modes(w, steps, warmup, dev):
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(max(16, fa.fa_bwd_workspace_size(B, N, H, d)), dtype=torch.uint8, device=dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     sp = torch.cuda.current_stream().cuda_stream
     scale = 1.0 / math.sqrt(d)
     c, (wl, wr) = int(w["causal"]), w["window"]
@@ -507,7 +524,7 @@ def time_modes(w, steps, warmup, dev):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(steps)]
         for i in range(steps):
-            flush.zero_()
+            flush()
             ev[i][0].record()
             fn()
             ev[i][1].record()
@@ -543,6 +560,118 @@ def run_sweep(args, local):
                                             "bwd": round(2.5 * Fv / t["bwd"] / 1e9, 1),
                                             "fwd_bwd": round(3.5 * Fv / t["fwd_bwd"] / 1e9, 1)}
         print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ decode (split-KV)
+
+def decode_workloads():
+    """Decoding steps with a KV cache (few query rows, many cached keys,
+    causal bottom-right): GQA shapes of common model families, long context,
+    MHA, and a 4-token speculative step."""
+    return [
+        dict(name="decode GQA B=8 Hq=32 Hkv=8 Nq=1 Nk=32768 d=128", B=8, Nq=1, Nk=32768, Hq=32, Hkv=8, d=128),
+        dict(name="decode GQA B=1 Hq=32 Hkv=8 Nq=1 Nk=131072 d=128", B=1, Nq=1, Nk=131072, Hq=32, Hkv=8, d=128),
+        dict(name="decode GQA B=64 Hq=64 Hkv=8 Nq=1 Nk=8192 d=128", B=64, Nq=1, Nk=8192, Hq=64, Hkv=8, d=128),
+        dict(name="decode MHA B=16 H=32 Nq=1 Nk=8192 d=128", B=16, Nq=1, Nk=8192, Hq=32, Hkv=32, d=128),
+        dict(name="decode GQA B=8 Hq=32 Hkv=8 Nq=4 Nk=32768 d=128 (speculative)", B=8, Nq=4, Nk=32768,
+             Hq=32, Hkv=8, d=128),
+        dict(name="decode GQA B=8 Hq=16 Hkv=2 Nq=1 Nk=32768 d=64", B=8, Nq=1, Nk=32768, Hq=16, Hkv=2, d=64),
+        dict(name="decode GQA B=4 Hq=16 Hkv=4 Nq=1 Nk=32768 d=256", B=4, Nq=1, Nk=32768, Hq=16, Hkv=4, d=256),
+    ]
+
+
+def decode_bytes(w):
+    """Algorithmic HBM bytes of one decoding step (causal, so every cached key
+    is visible): read K, V, Q; write O (bf16) and LSE (fp32)."""
+    kv = 2 * w["B"] * w["Nk"] * w["Hkv"] * w["d"] * 2
+    qo = 2 * w["B"] * w["Nq"] * w["Hq"] * w["d"] * 2
+    return kv + qo + 4 * w["B"] * w["Hq"] * w["Nq"]
+
+
+def run_decode(args, local):
+    """One JSON line per decoding workload: fa_fwd_splitkv (the library's split
+    count) timed with CUDA events on the launching stream, L2 flushed before
+    every call, median over the steps; algorithmic bytes / time against the
+    measured HBM copy bandwidth; fa_fwd on the same inputs for comparison."""
+    import torch
+    import exact_io_aware_89_b200 as fa
+    from seeded_inputs import make_inputs
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    flush = L2Flush(dev)
+    sp = torch.cuda.current_stream().cuda_stream
+    for n, w in enumerate(decode_workloads()):
+        B, Nq, Nk, Hq, Hkv, d = w["B"], w["Nq"], w["Nk"], w["Hq"], w["Hkv"], w["d"]
+        inp = make_inputs(B, Nq, Nk, Hq, Hkv, d, 4000 + n, with_dout=False)
+        q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
+        del inp
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+        scale = 1.0 / math.sqrt(d)
+        wsb = fa.fa_fwd_splitkv_workspace_size(B, Nq, Nk, Hq, Hkv, d, 1, -1, -1, 0)
+        ws = torch.empty(max(16, wsb), dtype=torch.uint8, device=dev)
+
+        def split():
+            st = fa.fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                   lse.data_ptr(), B, Nq, Nk, Hq, Hkv, d, scale, 1, -1, -1, 0,
+                                   ws.data_ptr(), ws.numel(), sp)
+            if st:
+                raise fa.FAError("fa_fwd_splitkv", st)
+
+        def plain():
+            st = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           B, Nq, Nk, Hq, Hkv, d, scale, 1, -1, -1, sp)
+            if st:
+                raise fa.FAError("fa_fwd", st)
+
+        def timed(fn, trace=False):
+            for _ in range(args.warmup):
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            if trace:
+                fa.fa_trace_enable(1)
+                fa.fa_trace_read()
+            torch.cuda.synchronize()
+            with ClockSampler(dev) as clocks:
+                for i in range(args.steps):
+                    flush()
+                    ev[i][0].record()
+                    fn()
+                    ev[i][1].record()
+                torch.cuda.synchronize()
+            tr = fa.fa_trace_read() if trace else None
+            if trace:
+                fa.fa_trace_enable(0)
+            return statistics.median(a.elapsed_time(b) for a, b in ev), tr, clocks.summary()
+
+        t_split, (tms, tn), clk = timed(split, trace=True)
+        t_plain, _, _ = timed(plain)
+        if fa.fa_get_device_status(None) != 0:
+            raise RuntimeError("device status reports a timed-out wait")
+        nbytes = decode_bytes(w)
+        gbs = nbytes / (t_split * 1e-3) / 1e9
+        main_ms = tms["decode"] / max(1, tn["decode"])
+        G = Hq // Hkv
+        qpt = min(Nq, 128 // G)
+        units = B * Hkv * (-(-Nq // qpt))
+        n_splits = (wsb - 8 * units) // (4 * (d + 1)) // (units * qpt * G) if wsb else 1
+        line = {"decode": w["name"], "B": B, "Nq": Nq, "Nk": Nk, "Hq": Hq, "Hkv": Hkv, "d": d,
+                "causal": True, "ms": round(t_split, 4), "fa_fwd_ms": round(t_plain, 4),
+                "speedup_vs_fa_fwd": round(t_plain / t_split, 2),
+                "n_splits": n_splits, "workspace_bytes": wsb,
+                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                             "algorithmic_bytes": nbytes,
+                             "kernel_ms": round(main_ms, 4),
+                             "kernel_frac": round(nbytes / (main_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                             "peak_source": peaks["source"] + ", copy"},
+                "clocks": clk}
+        print(json.dumps(line), flush=True)
+        del q, k, v, o, lse, ws
+        torch.cuda.empty_cache()
+    del flush
 
 
 def run_ours(args, world, rank, local):
@@ -593,7 +722,8 @@ def run_ours(args, world, rank, local):
         "config": {"workload": w["name"], "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
                    "causal": w["causal"], "global_batch": w["B"] * world,
                    "parallelism": "dp%d" % world,
-                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+                   "l2": "flushed between steps outside the timed events (256 MiB write, then a "
+                         "256 MiB read so the evicted lines are clean)"},
         "fwd_tflops": round(fwd_tf, 3),
         "fwd_bwd_pct_dense_peak": round(100 * value / (world * DENSE_PEAK_TFLOPS), 2),
         "fwd_pct_dense_peak": round(100 * fwd_tf / (world * DENSE_PEAK_TFLOPS), 2),
@@ -624,6 +754,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-budget", type=float, default=15.0,
                     help="seconds of oracle time for the CPU baseline sample")
+    ap.add_argument("--decode", action="store_true",
+                    help="instead of the benchmark line: the KV-cache decoding workloads through "
+                         "fa_fwd_splitkv, one JSON line each")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the benchmark line: the sequence-length sweep and the GQA/window "
                          "and d=256 workloads, fwd / bwd / fwd+bwd timed separately, one JSON line each")
@@ -631,10 +764,10 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     world, rank, local = dist_setup(args)
-    if args.sweep:
+    if args.sweep or args.decode:
         if world > 1:
-            raise SystemExit("--sweep runs on one GPU")
-        run_sweep(args, local)
+            raise SystemExit("--sweep and --decode run on one GPU")
+        (run_sweep if args.sweep else run_decode)(args, local)
         return
     if args.impl == "reference":
         run_reference(args, world, rank)  # rank 0 alone; no process group

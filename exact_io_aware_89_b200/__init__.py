@@ -3,12 +3,14 @@
 The C ABI (include/fa.h) is the product boundary; this module only marshals
 arguments to it.  Two layers:
 
-* ``fa_fwd``, ``fa_bwd``, ``fa_fwd_f32``, ``fa_bwd_f32``, ``fa_bwd_workspace_size``,
+* ``fa_fwd``, ``fa_bwd``, ``fa_fwd_splitkv``, ``fa_fwd_f32``, ``fa_bwd_f32``,
+  ``fa_bwd_workspace_size``, ``fa_fwd_splitkv_workspace_size``,
   ``fa_get_device_status``, ``fa_status_string``: the C entry points under the
   same names, taking raw device pointers (ints) and sizes, returning the
   status code.
-* ``attention_forward`` / ``attention_backward``: the same calls on torch CUDA
-  tensors (torch only allocates the outputs and supplies the current stream).
+* ``attention_forward`` / ``attention_backward`` / ``attention_forward_splitkv``:
+  the same calls on torch CUDA tensors (torch only allocates the outputs and
+  the workspace and supplies the current stream).
 
 There is no fallback: if libfa.so cannot be loaded or built, importing the
 tensor API raises, and every computation runs in the library's CUDA kernels.
@@ -20,8 +22,9 @@ import os
 __all__ = [
     "FAError", "load_library", "library_path",
     "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
+    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size",
     "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
-    "KERNEL_KINDS", "attention_forward", "attention_backward",
+    "KERNEL_KINDS", "attention_forward", "attention_backward", "attention_forward_splitkv",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -64,12 +67,15 @@ def load_library():
     lib.fa_bwd_f32.argtypes = lib.fa_bwd.argtypes
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_size.restype = sz
+    lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, i, vp, sz, vp]
+    lib.fa_fwd_splitkv_workspace_size.argtypes = [i, i, i, i, i, i, i, i, i, i]
+    lib.fa_fwd_splitkv_workspace_size.restype = sz
     lib.fa_get_device_status.argtypes = [vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_trace_enable.argtypes = [i]
     lib.fa_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
-    for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32",
+    for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv",
                  "fa_get_device_status",
                  "fa_trace_enable", "fa_trace_read"):
         getattr(lib, name).restype = i
@@ -98,6 +104,18 @@ def fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale
                                          scale, causal, win_l, win_r, stream)
 
 
+def fa_fwd_splitkv(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, n_splits,
+                   workspace, workspace_bytes, stream):
+    """Forward for few query rows over a long key range, split across CTAs."""
+    return load_library().fa_fwd_splitkv(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal,
+                                         win_l, win_r, n_splits, workspace, workspace_bytes, stream)
+
+
+def fa_fwd_splitkv_workspace_size(B, Nq, Nk, Hq, Hkv, d, causal, win_l, win_r, n_splits):
+    return load_library().fa_fwd_splitkv_workspace_size(B, Nq, Nk, Hq, Hkv, d, causal, win_l,
+                                                        win_r, n_splits)
+
+
 def fa_fwd_f32(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, stream):
     return load_library().fa_fwd_f32(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal,
                                      win_l, win_r, stream)
@@ -122,7 +140,7 @@ def fa_status_string(status):
     return load_library().fa_status_string(int(status)).decode()
 
 
-KERNEL_KINDS = ("fwd", "bwd_prep", "bwd_dq", "bwd_dkdv", "f32")
+KERNEL_KINDS = ("fwd", "bwd_prep", "bwd_dq", "bwd_dkdv", "f32", "decode")
 
 
 def fa_trace_enable(on):
@@ -186,6 +204,35 @@ def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), out=No
     fn = fa_fwd if q.dtype == torch.bfloat16 else fa_fwd_f32
     _check(fn.__name__, fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                            B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, _stream()))
+    return o, lse
+
+
+def attention_forward_splitkv(q, k, v, scale=None, causal=False, window=(-1, -1), n_splits=0,
+                              out=None, lse=None, workspace=None):
+    """O, LSE = attention(q, k, v) through fa_fwd_splitkv (bf16 only).
+
+    Meant for few query rows against many keys (decoding with a KV cache):
+    the keys are split across CTAs and the splits merged by their LSE.
+    ``n_splits`` 0 lets the library choose.  ``workspace``: optional uint8
+    CUDA tensor of at least ``fa_fwd_splitkv_workspace_size(...)`` bytes,
+    allocated here if omitted and needed.
+    """
+    import torch
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    if q.dtype != torch.bfloat16:
+        raise ValueError("fa_fwd_splitkv takes bf16 tensors")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    wsb = fa_fwd_splitkv_workspace_size(B, Nq, Nk, Hq, Hkv, d, c, wl, wr, int(n_splits))
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
+    _check("fa_fwd_splitkv",
+           fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                          B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, int(n_splits),
+                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                          _stream()))
     return o, lse
 
 

@@ -2,11 +2,13 @@
 // validation, TMA descriptor encoding and kernel launches on the caller's
 // stream.  No device memory is allocated here and nothing runs on the CPU
 // besides the checks.
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 #include <vector>
 
 #include "fa_bwd.cuh"
+#include "fa_decode.cuh"
 #include "fa_f32.cuh"
 #include "fa_fwd.cuh"
 #include "fa_host.cuh"
@@ -73,6 +75,12 @@ using Dq256 = DqCfg<256, 1, 64, 1>;
 using Dkv64 = DkvCfg<64, 64, 64, 4>;
 using Dkv128 = DkvCfg<128, 128, 64, 4>;
 using Dkv256 = DkvCfg<256, 128, 64, 1>;
+
+// split-KV decode: {d, key tile, K/V ring depth, TMEM lanes per copy of the packed rows}
+template <int RCP> using Dec64 = DecCfg<64, 128, 6, RCP>;
+template <int RCP> using Dec128 = DecCfg<128, 128, 3, RCP>;
+template <int RCP> using Dec256 = DecCfg<256, 64, 2, RCP>;
+constexpr int kMaxDecodeSplits = 4096;
 
 constexpr int kMaxDevices = 64;
 
@@ -223,6 +231,125 @@ size_t workspace_bytes(int B, int Nq, int Hq) {
          sizeof(float);
 }
 
+// ------------------------------------------------------------ split-KV decode
+// Row packing and key split of one fa_fwd_splitkv call.
+struct DecodePlan {
+  int group, qpt, n_qtiles, rt, rcp, key_tile, n_splits;
+  long long units;  // (batch, kv head, query tile) units
+};
+
+int decode_key_tile(int d) { return d == 256 ? 64 : 128; }
+
+// Key tiles visible to query tile qt (rows qt * qpt .. +qpt-1).
+int decode_tiles(const MaskSpec& m, int Nq, int qpt, int qt, int bn) {
+  const int i0 = qt * qpt, i1 = (qt + 1) * qpt - 1 < Nq - 1 ? (qt + 1) * qpt - 1 : Nq - 1;
+  const int lo = m.lo(i0), hi = m.hi(i1);
+  return hi >= lo ? hi / bn - lo / bn + 1 : 0;
+}
+
+// n_splits <= 0: one wave of CTAs.  With fewer (batch, kv head, query tile)
+// units than SMs, each unit's visible key tiles are split so that about one
+// CTA per SM streams its share of K and V, keeping at least 4 key tiles per
+// split so the copy ring fills; otherwise no split.
+int plan_decode(int B, int Nq, int Hq, int Hkv, int d, const MaskSpec& m, int n_splits, int sm_count,
+                DecodePlan* pl) {
+  pl->group = Hq / Hkv;
+  if (pl->group > 128) return FA_ERR_UNSUPPORTED;
+  pl->qpt = 128 / pl->group < Nq ? 128 / pl->group : Nq;
+  pl->n_qtiles = (Nq + pl->qpt - 1) / pl->qpt;
+  pl->rt = pl->qpt * pl->group;
+  pl->rcp = pl->rt <= 32 ? 32 : pl->rt <= 64 ? 64 : 128;
+  pl->key_tile = decode_key_tile(d);
+  pl->units = static_cast<long long>(B) * Hkv * pl->n_qtiles;
+  if (n_splits > kMaxDecodeSplits) return FA_ERR_INVALID_ARG;
+  if (n_splits > 0) {
+    pl->n_splits = n_splits;
+  } else {
+    if (sm_count < 1) return FA_ERR_CUDA;
+    int tiles = decode_tiles(m, Nq, pl->qpt, 0, pl->key_tile);
+    const int t_last = decode_tiles(m, Nq, pl->qpt, pl->n_qtiles - 1, pl->key_tile);
+    if (t_last > tiles) tiles = t_last;
+    long long n = pl->units >= sm_count ? 1 : sm_count / pl->units;
+    const long long cap = tiles / 4 > 1 ? tiles / 4 : 1;
+    if (n > cap) n = cap;
+    pl->n_splits = static_cast<int>(n);
+  }
+  if (pl->units * pl->n_splits > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+int current_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// Workspace of a split call: the partial O rows (fp32), their LSE, then one
+// 8-byte counter per unit (16-byte aligned).
+size_t decode_counters_offset(const DecodePlan& pl, int d) {
+  const size_t rows = static_cast<size_t>(pl.units) * pl.n_splits * pl.rt;
+  return (rows * d * sizeof(float) + rows * sizeof(float) + 15) / 16 * 16;
+}
+
+size_t decode_workspace_bytes(const DecodePlan& pl, int d) {
+  if (pl.n_splits <= 1) return 0;
+  return decode_counters_offset(pl, d) + static_cast<size_t>(pl.units) * sizeof(unsigned long long);
+}
+
+// Tag of one split call, so counters left by an earlier call read as zero.
+unsigned int next_decode_tag() {
+  static std::atomic<unsigned int> counter{0};
+  unsigned int t = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (t == 0) t = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+  return t;
+}
+
+template <class C>
+int launch_decode_cfg(const void* q, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                      long long grid, cudaStream_t stream) {
+  static int attr_done[kMaxDevices] = {0};
+  auto kern = fa_decode_kernel<C>;
+  if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
+  TraceScope tr(FA_KERNEL_DECODE, stream);
+  kern<<<static_cast<unsigned>(grid), C::NTHREADS, C::SMEM_BYTES, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), tk, tv, p);
+  return launch_status();
+}
+
+template <int D, template <int> class Cfg>
+int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+                  int Nk, int Hq, int Hkv, float scale, const MaskSpec& mask, const DecodePlan& pl,
+                  void* workspace, cudaStream_t stream) {
+  CUtensorMap tk, tv;
+  const int bn = Cfg<32>::BN;
+  if (!encode_bnhd(&tk, k, B, Nk, Hkv, D, bn) || !encode_bnhd(&tv, v, B, Nk, Hkv, D, bn)) return FA_ERR_CUDA;
+  DecodeParams p;
+  p.B = B; p.Nq = Nq; p.Nk = Nk; p.Hq = Hq; p.Hkv = Hkv; p.group = pl.group;
+  p.qpt = pl.qpt;
+  p.n_qtiles = pl.n_qtiles;
+  p.n_splits = pl.n_splits;
+  p.scale_log2 = scale * kLog2e;
+  p.mask = mask;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  const size_t rows = static_cast<size_t>(pl.units) * pl.n_splits * pl.rt;
+  const bool split = pl.n_splits > 1;
+  p.part_o = split ? static_cast<float*>(workspace) : nullptr;
+  p.part_lse = split ? static_cast<float*>(workspace) + rows * D : nullptr;
+  p.counters = split ? reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) +
+                                                             decode_counters_offset(pl, D))
+                     : nullptr;
+  p.tag = next_decode_tag();
+  p.wait_limit_ns = kWaitLimitNs;
+  const long long grid = pl.units * pl.n_splits;
+  switch (pl.rcp) {
+    case 32: return launch_decode_cfg<Cfg<32>>(q, tk, tv, p, grid, stream);
+    case 64: return launch_decode_cfg<Cfg<64>>(q, tk, tv, p, grid, stream);
+    default: return launch_decode_cfg<Cfg<128>>(q, tk, tv, p, grid, stream);
+  }
+}
+
 }  // namespace
 
 // ------------------------------------------------- allocation-free backward
@@ -325,6 +452,41 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
       return launch_bwd<Dq128, Dkv128>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
     default:
       return launch_bwd<Dq256, Dkv256>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+  }
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int Nq, int Nk, int Hq, int Hkv, int d, int causal,
+                                      int win_l, int win_r, int n_splits) {
+  if (B < 1 || Nq < 1 || Nk < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return 0;
+  if (d != 64 && d != 128 && d != 256) return 0;
+  DecodePlan pl;
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  if (plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(), &pl) != FA_OK)
+    return 0;
+  return decode_workspace_bytes(pl, d);
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+                   int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                   int n_splits, void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  DecodePlan pl;
+  st = plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(), &pl);
+  if (st != FA_OK) return st;
+  const size_t need = decode_workspace_bytes(pl, d);
+  if (need > 0 && (!aligned16(workspace) || workspace_bytes_ < need)) return FA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64:
+      return launch_decode<64, Dec64>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, workspace, s);
+    case 128:
+      return launch_decode<128, Dec128>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, workspace, s);
+    default:
+      return launch_decode<256, Dec256>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, workspace, s);
   }
 }
 

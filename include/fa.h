@@ -127,6 +127,38 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
                    fa_stream_t stream);
 
 /*
+ * Forward pass for few query rows against a long key/value sequence
+ * (decoding with a KV cache; hysenlabs page, changelog v2.2), bf16, with the
+ * arguments, masks, GQA mapping and outputs of fa_fwd: o and lse hold the same
+ * attention result (up to fp32 summation order).  The key range is split
+ * across CTAs, each CTA handling the Hq/Hkv query heads of one key/value head
+ * together (K and V are read from HBM once per key/value head, not once per
+ * query head).  One kernel launch: the last CTA of each (batch, key/value
+ * head, query tile) to finish merges the splits' partial outputs through
+ * their log-sum-exp, in split order, so results are deterministic.
+ *   n_splits : key splits per (batch, key/value head, query tile); 0 lets the
+ *              library choose from the current device's SM count (the same
+ *              choice fa_fwd_splitkv_workspace_size makes with that device
+ *              current); at most 4096
+ *   workspace: device buffer of at least fa_fwd_splitkv_workspace_size() bytes,
+ *              16-byte aligned, owned by the caller, contents ignored (each
+ *              call tags the per-unit counters it keeps there and leaves them
+ *              at zero; CUDA graph replays are fine); may be NULL when that
+ *              size is 0 (no split).  Calls that can overlap on the GPU must
+ *              not share a workspace.
+ * Requires Hq / Hkv <= 128 (else FA_ERR_UNSUPPORTED) and d in {64, 128, 256}.
+ * Any Nq is accepted; query rows are packed into 128-row tiles of
+ * floor(128 / (Hq/Hkv)) queries, so it pays off while Nq * Hq / Hkv is small.
+ * Returns FA_OK or an fa_status code (FA_ERR_WORKSPACE: workspace missing or
+ * too small).
+ */
+size_t fa_fwd_splitkv_workspace_size(int B, int Nq, int Nk, int Hq, int Hkv, int d, int causal,
+                                     int win_l, int win_r, int n_splits);
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+                   int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                   int n_splits, void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fp32 variants for small problems (fp32 in, fp32 out, fp32 arithmetic on the
  * CUDA cores).  Same arguments and semantics as fa_fwd / fa_bwd; d <= 256 and
  * d a multiple of 32.
@@ -165,7 +197,8 @@ enum fa_kernel_kind {
   FA_KERNEL_BWD_DQ = 2,   /* backward dQ, bf16 (tcgen05) */
   FA_KERNEL_BWD_DKDV = 3, /* backward dK/dV, bf16 (tcgen05) */
   FA_KERNEL_F32 = 4,      /* any fp32-path kernel */
-  FA_KERNEL_KINDS = 5
+  FA_KERNEL_DECODE = 5,   /* fa_fwd_splitkv, bf16 (tcgen05) */
+  FA_KERNEL_KINDS = 6
 };
 int fa_trace_enable(int on);
 int fa_trace_read(double* ms, long long* launches);

@@ -129,6 +129,38 @@ def attn_bwd(q, k, v, dout, scale=None, causal=False, window=(-1, -1), nthreads=
     return dq, dk, dv
 
 
+def merge_partials(o_parts, lse_parts):
+    """Merge attention results computed over disjoint key subsets.
+
+    o_parts[s] [B, Nq, Hq, d] and lse_parts[s] [B, Hq, Nq] are the outputs of
+    attention restricted to the s-th subset (O normalised over that subset,
+    LSE its natural log-sum-exp; -inf and O = 0 for a subset with no visible
+    key).  The blockwise softmax rule (abeam.tech FlashAttention summary,
+    "computing softmax blockwise correctly"), applied to whole subsets:
+    with l_s = exp(lse_s) the subset's row sum relative to a common
+    reference, the full row sum is sum_s l_s and the full output the l_s
+    weighted mean of the O_s.  In log form, relative to m = max_s lse_s:
+        lse = m + ln sum_s exp(lse_s - m),   O = sum_s exp(lse_s - lse) O_s.
+    Rows with every lse_s = -inf give lse = -inf and O = 0.  fp64 numpy."""
+    lse_parts = [np.asarray(x, dtype=np.float64) for x in lse_parts]
+    o_parts = [np.asarray(x, dtype=np.float64) for x in o_parts]
+    if not lse_parts or len(lse_parts) != len(o_parts):
+        raise ValueError("need matching, non-empty lists of partial results")
+    ls = np.stack(lse_parts)                       # [S, B, Hq, Nq]
+    m = ls.max(axis=0)
+    finite = np.isfinite(m)
+    m_safe = np.where(finite, m, 0.0)
+    with np.errstate(invalid="ignore"):
+        w = np.where(np.isneginf(ls), 0.0, np.exp(ls - m_safe))
+    total = w.sum(axis=0)
+    lse = np.where(finite, m_safe + np.log(np.where(finite, total, 1.0)), -np.inf)
+    wn = np.where(finite, w / np.where(finite, total, 1.0), 0.0)   # [S, B, Hq, Nq]
+    o = np.zeros_like(o_parts[0])
+    for s, op in enumerate(o_parts):
+        o += np.transpose(wn[s], (0, 2, 1))[..., None] * op     # weights as [B, Nq, Hq, 1]
+    return o, lse
+
+
 def _rows(rows):
     r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).ravel())
     return r, r.ctypes.data_as(ctypes.POINTER(ctypes.c_int))

@@ -25,7 +25,16 @@ def declared_functions():
 def test_header_declares_the_expected_entry_points():
     assert declared_functions() == sorted([
         "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
+        "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size",
         "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
+
+
+def test_kernel_kinds_match_the_header():
+    header = open(HEADER).read()
+    kinds = re.findall(r"\bFA_KERNEL_([A-Z0-9_]+)\s*=\s*(\d+)", header)
+    named = {int(v): n.lower() for n, v in kinds if n != "KINDS"}
+    n_kinds = int(dict(kinds)["KINDS"])
+    assert [named[i] for i in range(n_kinds)] == list(fa.KERNEL_KINDS)
 
 
 def test_library_exports_every_declared_symbol():
@@ -113,3 +122,52 @@ def test_f32_head_dim_limits():
     for d in (16, 48, 288):
         assert fa.fa_fwd_f32(a["q"], a["k"], a["v"], a["o"], a["lse"], 1, 8, 8, 1, 1, d, 0.1, 0, -1,
                              -1, None) == UNSUPPORTED
+
+
+# ------------------------------------------------------------ split-KV forward
+
+def _splitkv(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=2, Nq=1, Nk=1000, Hq=8, Hkv=2, d=128,
+             scale=0.125, causal=0, win_l=-1, win_r=-1, n_splits=4, ws=0, wsb=0, stream=None)
+    a.update(kw)
+    return fa.fa_fwd_splitkv(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Nq"], a["Nk"],
+                             a["Hq"], a["Hkv"], a["d"], a["scale"], a["causal"], a["win_l"],
+                             a["win_r"], a["n_splits"], a["ws"], a["wsb"], a["stream"])
+
+
+def test_splitkv_workspace_size():
+    # rows of one query tile = queries per tile * group; the partial O rows
+    # (fp32, d wide) of every (batch, kv head, query tile, split), then their
+    # LSE, then (16-byte aligned) one 8-byte counter per unit
+    def expect(units, splits, rows, d):
+        n = units * splits * rows
+        return (n * d * 4 + n * 4 + 15) // 16 * 16 + 8 * units
+    ws = fa.fa_fwd_splitkv_workspace_size
+    assert ws(2, 1, 1000, 8, 2, 128, 0, -1, -1, 4) == expect(2 * 2, 4, 4, 128)
+    # group 4: 32 queries per tile, 40 queries -> 2 tiles of 128 packed rows
+    assert ws(1, 40, 4096, 8, 2, 64, 1, -1, -1, 3) == expect(1 * 2 * 2, 3, 128, 64)
+    # MQA with 32 query heads: up to 4 queries per tile, here both of the 2
+    assert ws(3, 2, 512, 32, 1, 256, 0, 100, 0, 2) == expect(3 * 1 * 1, 2, 64, 256)
+    assert ws(2, 1, 1000, 8, 2, 128, 0, -1, -1, 1) == 0          # no split, no workspace
+    assert ws(1, 1, 1000, 256, 1, 128, 0, -1, -1, 4) == 0        # group > 128: unsupported
+    assert ws(1, 1, 1000, 8, 2, 96, 0, -1, -1, 4) == 0           # head dim
+    assert ws(1, 1, 1000, 6, 4, 128, 0, -1, -1, 4) == 0          # Hq % Hkv
+    assert ws(1, 1, 1000, 8, 2, 128, 0, -1, -1, 5000) == 0       # too many splits
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=0), dict(k=MISALIGNED), dict(o=0), dict(lse=MISALIGNED), dict(B=0), dict(Nk=0),
+    dict(Hq=6, Hkv=4), dict(scale=float("nan")), dict(n_splits=5000),
+])
+def test_splitkv_rejects_invalid_arguments(kw):
+    assert _splitkv(**kw) == INVALID
+
+
+def test_splitkv_rejects_unsupported_and_missing_workspace():
+    assert _splitkv(d=96) == UNSUPPORTED
+    assert _splitkv(Hq=256, Hkv=1) == UNSUPPORTED
+    need = fa.fa_fwd_splitkv_workspace_size(2, 1, 1000, 8, 2, 128, 0, -1, -1, 4)
+    assert need > 0
+    assert _splitkv(ws=0, wsb=need) == WORKSPACE
+    assert _splitkv(ws=FAKE, wsb=need - 4) == WORKSPACE
+    assert _splitkv(ws=MISALIGNED, wsb=need) == WORKSPACE

@@ -310,3 +310,61 @@ def test_selected_rows_equal_full_functions(causal, wl, wr):
     dk_r, dv_r = oracle.attn_dkdv_rows(q, k, v, do, krows, nthreads=3, **kw)
     np.testing.assert_allclose(dk_r, dk[:, krows], rtol=1e-13, atol=1e-13)
     np.testing.assert_allclose(dv_r, dv[:, krows], rtol=1e-13, atol=1e-13)
+
+
+# ------------------------------------------------- merging partial results
+
+def _subset_result(q, k, v, idx, scale):
+    """Attention restricted to the keys in idx (non-causal); an empty subset
+    gives O = 0 and LSE = -inf."""
+    B, Nq, Hq, d = q.shape
+    if len(idx) == 0:
+        return np.zeros((B, Nq, Hq, d)), np.full((B, Hq, Nq), -np.inf)
+    return oracle.attn_fwd(q, k[:, idx], v[:, idx], scale=scale)
+
+
+@pytest.mark.parametrize("n_parts", [1, 2, 4, 7])
+def test_merge_of_key_subsets_equals_attention_over_all_keys(n_parts):
+    """Splitting the keys into disjoint subsets (contiguous or scattered, one
+    possibly empty), attending over each and merging gives attention over all
+    keys: the merge is pinned to the two-pass definition."""
+    rng = np.random.default_rng(40 + n_parts)
+    B, Nq, Nk, Hq, Hkv, d = 2, 5, 23, 4, 2, 8
+    q = rng.standard_normal((B, Nq, Hq, d))
+    k = rng.standard_normal((B, Nk, Hkv, d))
+    v = rng.standard_normal((B, Nk, Hkv, d))
+    scale = 0.7
+    labels = rng.integers(0, n_parts, Nk)
+    if n_parts > 2:
+        labels[labels == n_parts - 1] = 0          # the last subset is empty
+    parts = [_subset_result(q, k, v, np.flatnonzero(labels == s), scale) for s in range(n_parts)]
+    o, lse = oracle.merge_partials([p[0] for p in parts], [p[1] for p in parts])
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, scale=scale)
+    assert np.abs(o - o_ref).max() < 1e-12
+    assert np.abs(lse - lse_ref).max() < 1e-12
+
+
+def test_merge_of_contiguous_splits_is_order_free():
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((1, 3, 2, 4))
+    k = rng.standard_normal((1, 40, 2, 4))
+    v = rng.standard_normal((1, 40, 2, 4))
+    cuts = [0, 9, 10, 31, 40]
+    parts = [_subset_result(q, k, v, np.arange(a, b), 0.5) for a, b in zip(cuts, cuts[1:])]
+    o1, l1 = oracle.merge_partials([p[0] for p in parts], [p[1] for p in parts])
+    o2, l2 = oracle.merge_partials([p[0] for p in parts[::-1]], [p[1] for p in parts[::-1]])
+    assert np.abs(o1 - o2).max() < 1e-14 and np.abs(l1 - l2).max() < 1e-14
+
+
+def test_merge_rows_without_keys():
+    """A row whose every subset is empty stays empty (LSE -inf, O 0); a row
+    with one non-empty subset gets exactly that subset's result."""
+    o_a = np.ones((1, 2, 1, 3))
+    o_b = np.full((1, 2, 1, 3), 2.0)
+    lse_a = np.array([[[-np.inf, 0.25]]])
+    lse_b = np.array([[[-np.inf, -np.inf]]])
+    o_b[:, 1] = 0.0
+    o_a[:, 0] = 0.0
+    o, lse = oracle.merge_partials([o_a, o_b], [lse_a, lse_b])
+    assert np.isneginf(lse[0, 0, 0]) and np.all(o[0, 0] == 0.0)
+    assert lse[0, 0, 1] == 0.25 and np.all(o[0, 1] == 1.0)
