@@ -52,12 +52,13 @@ WORKLOADS = {
 # only while the kernel sources hash to the ones that were profiled (a changed
 # kernel reports null until it is captured again).
 NCU_TRAFFIC = {
-    ("train", "bwd_dkdv"): dict(bytes=72.68e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
-    ("mid", "bwd_dkdv"): dict(bytes=378.44e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
-    ("mid", "bwd_dq"): dict(bytes=326.29e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
-    ("mid", "fwd"): dict(bytes=252.54e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
+    ("train", "bwd_dkdv"): dict(bytes=72.78e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
+    ("mid", "bwd_dkdv"): dict(bytes=377.91e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
+    ("mid", "bwd_dq"): dict(bytes=325.89e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
+    ("mid", "fwd"): dict(bytes=250.95e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
+    ("decode0", "decode"): dict(bytes=1078.09e6, profile="profiles/decode_B8Hq32Hkv8Nq1Nk32768d128.md"),
 }
-NCU_SOURCES_SHA256 = "f62d04c24b51c15fc18228ee502c792a8957027481233d600f21f5c487b1683f"
+NCU_SOURCES_SHA256 = "ae64b5eee6d39decc6046491fcc8746f3eb2753cb7e38359a75c5e36e87b7c11"
 
 
 def sources_sha256():
@@ -602,6 +603,8 @@ def run_decode(args, local):
     flush = L2Flush(dev)
     sp = torch.cuda.current_stream().cuda_stream
     for n, w in enumerate(decode_workloads()):
+        if args.decode_case is not None and n != args.decode_case:
+            continue
         B, Nq, Nk, Hq, Hkv, d = w["B"], w["Nq"], w["Nk"], w["Hq"], w["Hkv"], w["d"]
         inp = make_inputs(B, Nq, Nk, Hq, Hkv, d, 4000 + n, with_dout=False)
         q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
@@ -664,6 +667,8 @@ def run_decode(args, local):
                 "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                              "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                              "algorithmic_bytes": nbytes,
+                             "traffic": ncu_traffic("decode%d" % n, "decode")[0],
+                             "traffic_profile": ncu_traffic("decode%d" % n, "decode")[1],
                              "kernel_ms": round(main_ms, 4),
                              "kernel_frac": round(nbytes / (main_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                              "peak_source": peaks["source"] + ", copy"},
@@ -757,6 +762,8 @@ def main(argv=None):
     ap.add_argument("--decode", action="store_true",
                     help="instead of the benchmark line: the KV-cache decoding workloads through "
                          "fa_fwd_splitkv, one JSON line each")
+    ap.add_argument("--decode-case", type=int, default=None,
+                    help="with --decode: only this workload (index into the list)")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the benchmark line: the sequence-length sweep and the GQA/window "
                          "and d=256 workloads, fwd / bwd / fwd+bwd timed separately, one JSON line each")

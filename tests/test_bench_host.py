@@ -49,9 +49,20 @@ def test_ncu_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
 
 
 def test_profiles_named_in_the_traffic_table_exist():
+    n_decode = len(bench.decode_workloads())
     for (wl, kern), t in bench.NCU_TRAFFIC.items():
-        assert wl in bench.WORKLOADS
+        if wl.startswith("decode"):
+            assert kern == "decode" and 0 <= int(wl[len("decode"):]) < n_decode
+        else:
+            assert wl in bench.WORKLOADS
         assert os.path.exists(os.path.join(ROOT, t["profile"])), t["profile"]
+
+
+def test_decode_bytes_count_kv_once():
+    w = bench.decode_workloads()[0]
+    kv = 2 * w["B"] * w["Nk"] * w["Hkv"] * w["d"] * 2
+    assert bench.decode_bytes(w) == kv + 2 * w["B"] * w["Nq"] * w["Hq"] * w["d"] * 2 + \
+        4 * w["B"] * w["Hq"] * w["Nq"]
 
 
 def _free_port():
