@@ -578,13 +578,29 @@ def decode_workloads():
              Hq=32, Hkv=8, d=128),
         dict(name="decode GQA B=8 Hq=16 Hkv=2 Nq=1 Nk=32768 d=64", B=8, Nq=1, Nk=32768, Hq=16, Hkv=2, d=64),
         dict(name="decode GQA B=4 Hq=16 Hkv=4 Nq=1 Nk=32768 d=256", B=4, Nq=1, Nk=32768, Hq=16, Hkv=4, d=256),
+        dict(name="decode GQA B=16 Hq=32 Hkv=8 Nq=1 d=128, KV cache of 32768 keys with ragged lengths "
+                   "(seeded uniform), one new key/value appended in place", B=16, Nq=1, Nk=32768, Hq=32,
+             Hkv=8, d=128, ragged=True),
     ]
+
+
+def decode_lengths(w):
+    """Cached keys per sequence of a ragged decoding workload (seeded)."""
+    import numpy as np
+    rng = np.random.default_rng(4321)
+    return rng.integers(1, w["Nk"], w["B"]).tolist()
 
 
 def decode_bytes(w):
     """Algorithmic HBM bytes of one decoding step (causal, so every cached key
-    is visible): read K, V, Q; write O (bf16) and LSE (fp32)."""
-    kv = 2 * w["B"] * w["Nk"] * w["Hkv"] * w["d"] * 2
+    is visible): read K, V, Q; write O (bf16) and LSE (fp32).  With ragged
+    lengths, K and V of each sequence's own keys (its cached ones plus the
+    new one), and the new key/value read once and written into the cache."""
+    row = w["Hkv"] * w["d"] * 2
+    if w.get("ragged"):
+        kv = 2 * row * sum(min(w["Nk"], n + 1) for n in decode_lengths(w)) + 2 * 2 * w["B"] * row
+    else:
+        kv = 2 * w["B"] * w["Nk"] * row
     qo = 2 * w["B"] * w["Nq"] * w["Hq"] * w["d"] * 2
     return kv + qo + 4 * w["B"] * w["Hq"] * w["Nq"]
 
@@ -609,13 +625,27 @@ def run_decode(args, local):
         inp = make_inputs(B, Nq, Nk, Hq, Hkv, d, 4000 + n, with_dout=False)
         q, k, v = (inp[x].to(dev) for x in ("q", "k", "v"))
         del inp
+        ragged = bool(w.get("ragged"))
+        if ragged:
+            lens = torch.tensor(decode_lengths(w), dtype=torch.int32, device=dev)
+            new = make_inputs(B, 1, 1, Hkv, Hkv, d, 5000 + n, with_dout=False)
+            k_new, v_new = new["k"].to(dev), new["v"].to(dev)
         o = torch.empty_like(q)
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
         scale = 1.0 / math.sqrt(d)
-        wsb = fa.fa_fwd_splitkv_workspace_size(B, Nq, Nk, Hq, Hkv, d, 1, -1, -1, 0)
+        wsb = (fa.fa_fwd_kvcache_workspace_size(B, Nq, Nk, Hq, Hkv, d, 1, -1, -1, 0, 1) if ragged else
+               fa.fa_fwd_splitkv_workspace_size(B, Nq, Nk, Hq, Hkv, d, 1, -1, -1, 0))
         ws = torch.empty(max(16, wsb), dtype=torch.uint8, device=dev)
 
         def split():
+            if ragged:
+                st = fa.fa_fwd_kvcache(q.data_ptr(), k.data_ptr(), v.data_ptr(), k_new.data_ptr(),
+                                       v_new.data_ptr(), lens.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                       B, Nq, Nk, 1, Hq, Hkv, d, scale, 1, -1, -1, 0, ws.data_ptr(),
+                                       ws.numel(), sp)
+                if st:
+                    raise fa.FAError("fa_fwd_kvcache", st)
+                return
             st = fa.fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                    lse.data_ptr(), B, Nq, Nk, Hq, Hkv, d, scale, 1, -1, -1, 0,
                                    ws.data_ptr(), ws.numel(), sp)
@@ -650,7 +680,7 @@ def run_decode(args, local):
             return statistics.median(a.elapsed_time(b) for a, b in ev), tr, clocks.summary()
 
         t_split, (tms, tn), clk = timed(split, trace=True)
-        t_plain, _, _ = timed(plain)
+        t_plain = None if ragged else timed(plain)[0]
         if fa.fa_get_device_status(None) != 0:
             raise RuntimeError("device status reports a timed-out wait")
         nbytes = decode_bytes(w)
@@ -661,8 +691,9 @@ def run_decode(args, local):
         units = B * Hkv * (-(-Nq // qpt))
         n_splits = (wsb - 8 * units) // (4 * (d + 1)) // (units * qpt * G) if wsb else 1
         line = {"decode": w["name"], "B": B, "Nq": Nq, "Nk": Nk, "Hq": Hq, "Hkv": Hkv, "d": d,
-                "causal": True, "ms": round(t_split, 4), "fa_fwd_ms": round(t_plain, 4),
-                "speedup_vs_fa_fwd": round(t_plain / t_split, 2),
+                "causal": True, "ms": round(t_split, 4),
+                "fa_fwd_ms": None if t_plain is None else round(t_plain, 4),
+                "speedup_vs_fa_fwd": None if t_plain is None else round(t_plain / t_split, 2),
                 "n_splits": n_splits, "workspace_bytes": wsb,
                 "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                              "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
@@ -673,6 +704,15 @@ def run_decode(args, local):
                              "kernel_frac": round(nbytes / (main_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                              "peak_source": peaks["source"] + ", copy"},
                 "clocks": clk}
+        if ragged:
+            lens_h = decode_lengths(w)
+            line["cache_lengths"] = {"min": min(lens_h), "max": max(lens_h),
+                                     "mean": round(sum(lens_h) / B, 1)}
+            line["append_kernel_ms"] = round(tms["kvcache_append"] / max(1, tn["kvcache_append"]), 4)
+            # the whole call is two launches (append, then attention)
+            line["roofline"]["kernel_ms"] = round(main_ms + line["append_kernel_ms"], 4)
+            line["roofline"]["kernel_frac"] = round(
+                nbytes / (line["roofline"]["kernel_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
         print(json.dumps(line), flush=True)
         del q, k, v, o, lse, ws
         torch.cuda.empty_cache()

@@ -3,12 +3,13 @@
 The C ABI (include/fa.h) is the product boundary; this module only marshals
 arguments to it.  Two layers:
 
-* ``fa_fwd``, ``fa_bwd``, ``fa_fwd_splitkv``, ``fa_fwd_f32``, ``fa_bwd_f32``,
+* ``fa_fwd``, ``fa_bwd``, ``fa_fwd_splitkv``, ``fa_fwd_kvcache``, ``fa_fwd_f32``, ``fa_bwd_f32``,
   ``fa_bwd_workspace_size``, ``fa_fwd_splitkv_workspace_size``,
   ``fa_get_device_status``, ``fa_status_string``: the C entry points under the
   same names, taking raw device pointers (ints) and sizes, returning the
   status code.
-* ``attention_forward`` / ``attention_backward`` / ``attention_forward_splitkv``:
+* ``attention_forward`` / ``attention_backward`` / ``attention_forward_splitkv`` /
+  ``attention_forward_kvcache``:
   the same calls on torch CUDA tensors (torch only allocates the outputs and
   the workspace and supplies the current stream).
 
@@ -22,9 +23,11 @@ import os
 __all__ = [
     "FAError", "load_library", "library_path",
     "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
-    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size",
+    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
+    "fa_fwd_kvcache_workspace_size",
     "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
     "KERNEL_KINDS", "attention_forward", "attention_backward", "attention_forward_splitkv",
+    "attention_forward_kvcache",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,12 +73,16 @@ def load_library():
     lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, i, vp, sz, vp]
     lib.fa_fwd_splitkv_workspace_size.argtypes = [i, i, i, i, i, i, i, i, i, i]
     lib.fa_fwd_splitkv_workspace_size.restype = sz
+    lib.fa_fwd_kvcache_workspace_size.argtypes = [i, i, i, i, i, i, i, i, i, i, i]
+    lib.fa_fwd_kvcache_workspace_size.restype = sz
+    lib.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i,
+                                   i, vp, sz, vp]
     lib.fa_get_device_status.argtypes = [vp]
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_trace_enable.argtypes = [i]
     lib.fa_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
-    for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv",
+    for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache",
                  "fa_get_device_status",
                  "fa_trace_enable", "fa_trace_read"):
         getattr(lib, name).restype = i
@@ -111,6 +118,20 @@ def fa_fwd_splitkv(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l,
                                          win_l, win_r, n_splits, workspace, workspace_bytes, stream)
 
 
+def fa_fwd_kvcache(q, k_cache, v_cache, k_new, v_new, cache_seqlens, o, lse, B, Nq, Nk, n_new, Hq,
+                   Hkv, d, scale, causal, win_l, win_r, n_splits, workspace, workspace_bytes, stream):
+    """fa_fwd_splitkv over a key/value cache, appending n_new keys/values in place."""
+    return load_library().fa_fwd_kvcache(q, k_cache, v_cache, k_new, v_new, cache_seqlens, o, lse,
+                                         B, Nq, Nk, n_new, Hq, Hkv, d, scale, causal, win_l, win_r,
+                                         n_splits, workspace, workspace_bytes, stream)
+
+
+def fa_fwd_kvcache_workspace_size(B, Nq, Nk, Hq, Hkv, d, causal, win_l, win_r, n_splits,
+                                  with_seqlens):
+    return load_library().fa_fwd_kvcache_workspace_size(B, Nq, Nk, Hq, Hkv, d, causal, win_l,
+                                                        win_r, n_splits, int(bool(with_seqlens)))
+
+
 def fa_fwd_splitkv_workspace_size(B, Nq, Nk, Hq, Hkv, d, causal, win_l, win_r, n_splits):
     return load_library().fa_fwd_splitkv_workspace_size(B, Nq, Nk, Hq, Hkv, d, causal, win_l,
                                                         win_r, n_splits)
@@ -140,7 +161,7 @@ def fa_status_string(status):
     return load_library().fa_status_string(int(status)).decode()
 
 
-KERNEL_KINDS = ("fwd", "bwd_prep", "bwd_dq", "bwd_dkdv", "f32", "decode")
+KERNEL_KINDS = ("fwd", "bwd_prep", "bwd_dq", "bwd_dkdv", "f32", "decode", "kvcache_append")
 
 
 def fa_trace_enable(on):
@@ -233,6 +254,49 @@ def attention_forward_splitkv(q, k, v, scale=None, causal=False, window=(-1, -1)
                           B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, int(n_splits),
                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                           _stream()))
+    return o, lse
+
+
+def attention_forward_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache_seqlens=None,
+                              scale=None, causal=False, window=(-1, -1), n_splits=0, out=None,
+                              lse=None, workspace=None):
+    """O, LSE through fa_fwd_kvcache (bf16 only): k_new / v_new [B, n_new,
+    Hkv, d] are written into k_cache / v_cache [B, Nk, Hkv, d] in place at
+    rows cache_seqlens[b] .. + n_new - 1, then q [B, Nq, Hq, d] attends to
+    the first cache_seqlens[b] + n_new keys of each sequence.
+    ``cache_seqlens``: int32 CUDA tensor [B], or None for full caches (then no
+    k_new / v_new)."""
+    import torch
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k_cache, v_cache)
+    if q.dtype != torch.bfloat16:
+        raise ValueError("fa_fwd_kvcache takes bf16 tensors")
+    n_new = 0
+    if k_new is not None or v_new is not None:
+        if k_new is None or v_new is None or k_new.shape != v_new.shape:
+            raise ValueError("k_new and v_new must be given together, with equal shapes")
+        if k_new.dim() != 4 or k_new.shape[0] != B or k_new.shape[2:] != k_cache.shape[2:]:
+            raise ValueError("k_new must be [B, n_new, Hkv, d]")
+        if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.dtype != q.dtype:
+            raise ValueError("k_new / v_new must be contiguous bf16")
+        n_new = int(k_new.shape[1])
+    if cache_seqlens is not None:
+        if cache_seqlens.dtype != torch.int32 or not cache_seqlens.is_cuda or \
+                cache_seqlens.numel() != B or not cache_seqlens.is_contiguous():
+            raise ValueError("cache_seqlens must be a contiguous int32 CUDA tensor of B entries")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    wsb = fa_fwd_kvcache_workspace_size(B, Nq, Nk, Hq, Hkv, d, c, wl, wr, int(n_splits),
+                                        cache_seqlens is not None)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
+    ptr = lambda t: None if t is None else t.data_ptr()
+    _check("fa_fwd_kvcache",
+           fa_fwd_kvcache(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), ptr(k_new),
+                          ptr(v_new), ptr(cache_seqlens), o.data_ptr(), lse.data_ptr(), B, Nq, Nk,
+                          n_new, Hq, Hkv, d, scale, c, wl, wr, int(n_splits), workspace.data_ptr(),
+                          workspace.numel() * workspace.element_size(), _stream()))
     return o, lse
 
 

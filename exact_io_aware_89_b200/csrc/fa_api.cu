@@ -234,7 +234,7 @@ size_t workspace_bytes(int B, int Nq, int Hq) {
 // ------------------------------------------------------------ split-KV decode
 // Row packing and key split of one fa_fwd_splitkv call.
 struct DecodePlan {
-  int group, qpt, n_qtiles, rt, rcp, key_tile, n_splits;
+  int group, qpt, n_qtiles, rt, rcp, key_tile, n_splits, split_tiles;
   long long units;  // (batch, kv head, query tile) units
 };
 
@@ -247,12 +247,18 @@ int decode_tiles(const MaskSpec& m, int Nq, int qpt, int qt, int bn) {
   return hi >= lo ? hi / bn - lo / bn + 1 : 0;
 }
 
-// n_splits <= 0: one wave of CTAs.  With fewer (batch, kv head, query tile)
-// units than SMs, each unit's visible key tiles are split so that about one
-// CTA per SM streams its share of K and V, keeping at least 4 key tiles per
-// split so the copy ring fills; otherwise no split.
+// Key splits.  Every split of a unit takes `split_tiles` key tiles (the
+// last one the rest), so a unit with fewer visible tiles -- a shorter
+// sequence under per-sequence cache lengths -- uses fewer CTAs.
+// n_splits <= 0 lets the library choose: with fewer (batch, kv head, query
+// tile) units than SMs, the widest unit's tiles are split so that about one
+// wave of CTAs (one per SM) streams K and V, keeping at least 4 key tiles per
+// split so the copy ring fills.  With per-sequence lengths (ragged) the
+// target is 3 waves' worth at full length, so the longest sequences are cut
+// finely enough to balance (on 16 sequences of uniformly random length, 3
+// waves came within 1% of the best split count, 1 wave was 34% slower).
 int plan_decode(int B, int Nq, int Hq, int Hkv, int d, const MaskSpec& m, int n_splits, int sm_count,
-                DecodePlan* pl) {
+                bool ragged, DecodePlan* pl) {
   pl->group = Hq / Hkv;
   if (pl->group > 128) return FA_ERR_UNSUPPORTED;
   pl->qpt = 128 / pl->group < Nq ? 128 / pl->group : Nq;
@@ -262,18 +268,23 @@ int plan_decode(int B, int Nq, int Hq, int Hkv, int d, const MaskSpec& m, int n_
   pl->key_tile = decode_key_tile(d);
   pl->units = static_cast<long long>(B) * Hkv * pl->n_qtiles;
   if (n_splits > kMaxDecodeSplits) return FA_ERR_INVALID_ARG;
-  if (n_splits > 0) {
-    pl->n_splits = n_splits;
-  } else {
+  // the widest query tile's visible key tiles (at full capacity)
+  int tiles = 0;
+  for (int qt = 0; qt < pl->n_qtiles; ++qt) {
+    const int t = decode_tiles(m, Nq, pl->qpt, qt, pl->key_tile);
+    if (t > tiles) tiles = t;
+  }
+  long long n = n_splits;
+  if (n_splits <= 0) {
     if (sm_count < 1) return FA_ERR_CUDA;
-    int tiles = decode_tiles(m, Nq, pl->qpt, 0, pl->key_tile);
-    const int t_last = decode_tiles(m, Nq, pl->qpt, pl->n_qtiles - 1, pl->key_tile);
-    if (t_last > tiles) tiles = t_last;
-    long long n = pl->units >= sm_count ? 1 : sm_count / pl->units;
+    const long long target = ragged ? 3ll * sm_count : sm_count;
+    n = pl->units >= target ? 1 : (target + pl->units - 1) / pl->units;
+    if (!ragged && pl->units < target) n = target / pl->units;
     const long long cap = tiles / 4 > 1 ? tiles / 4 : 1;
     if (n > cap) n = cap;
-    pl->n_splits = static_cast<int>(n);
   }
+  pl->split_tiles = tiles > 0 ? static_cast<int>((tiles + n - 1) / n) : 1;
+  pl->n_splits = tiles > 0 ? (tiles + pl->split_tiles - 1) / pl->split_tiles : 1;
   if (pl->units * pl->n_splits > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
@@ -320,7 +331,7 @@ int launch_decode_cfg(const void* q, const CUtensorMap& tk, const CUtensorMap& t
 template <int D, template <int> class Cfg>
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
                   int Nk, int Hq, int Hkv, float scale, const MaskSpec& mask, const DecodePlan& pl,
-                  void* workspace, cudaStream_t stream) {
+                  const int* seqlens, int n_new, void* workspace, cudaStream_t stream) {
   CUtensorMap tk, tv;
   const int bn = Cfg<32>::BN;
   if (!encode_bnhd(&tk, k, B, Nk, Hkv, D, bn) || !encode_bnhd(&tv, v, B, Nk, Hkv, D, bn)) return FA_ERR_CUDA;
@@ -329,8 +340,11 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.qpt = pl.qpt;
   p.n_qtiles = pl.n_qtiles;
   p.n_splits = pl.n_splits;
+  p.split_tiles = pl.split_tiles;
   p.scale_log2 = scale * kLog2e;
   p.mask = mask;
+  p.seqlens = seqlens;
+  p.n_new = n_new;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   const size_t rows = static_cast<size_t>(pl.units) * pl.n_splits * pl.rt;
@@ -455,15 +469,26 @@ int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, c
   }
 }
 
-size_t fa_fwd_splitkv_workspace_size(int B, int Nq, int Nk, int Hq, int Hkv, int d, int causal,
-                                      int win_l, int win_r, int n_splits) {
+static size_t splitkv_workspace(int B, int Nq, int Nk, int Hq, int Hkv, int d, int causal, int win_l,
+                                int win_r, int n_splits, bool ragged) {
   if (B < 1 || Nq < 1 || Nk < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return 0;
   if (d != 64 && d != 128 && d != 256) return 0;
   DecodePlan pl;
   const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
-  if (plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(), &pl) != FA_OK)
+  if (plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(), ragged, &pl) !=
+      FA_OK)
     return 0;
   return decode_workspace_bytes(pl, d);
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int Nq, int Nk, int Hq, int Hkv, int d, int causal,
+                                      int win_l, int win_r, int n_splits) {
+  return splitkv_workspace(B, Nq, Nk, Hq, Hkv, d, causal, win_l, win_r, n_splits, false);
+}
+
+size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Nk, int Hq, int Hkv, int d, int causal,
+                                     int win_l, int win_r, int n_splits, int with_seqlens) {
+  return splitkv_workspace(B, Nq, Nk, Hq, Hkv, d, causal, win_l, win_r, n_splits, with_seqlens != 0);
 }
 
 int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
@@ -475,18 +500,61 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
   if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
   const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
   DecodePlan pl;
-  st = plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(), &pl);
+  st = plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(), false, &pl);
   if (st != FA_OK) return st;
   const size_t need = decode_workspace_bytes(pl, d);
   if (need > 0 && (!aligned16(workspace) || workspace_bytes_ < need)) return FA_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (d) {
     case 64:
-      return launch_decode<64, Dec64>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, workspace, s);
+      return launch_decode<64, Dec64>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, nullptr, 0, workspace, s);
     case 128:
-      return launch_decode<128, Dec128>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, workspace, s);
+      return launch_decode<128, Dec128>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, nullptr, 0, workspace, s);
     default:
-      return launch_decode<256, Dec256>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, workspace, s);
+      return launch_decode<256, Dec256>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, nullptr, 0, workspace, s);
+  }
+}
+
+int fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                   const int* cache_seqlens, void* o, float* lse, int B, int Nq, int Nk, int n_new,
+                   int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r, int n_splits,
+                   void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_common(q, k_cache, v_cache, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if (n_new < 0) return FA_ERR_INVALID_ARG;
+  if (n_new > 0 && (!aligned16(k_new) || !aligned16(v_new) || cache_seqlens == nullptr))
+    return FA_ERR_INVALID_ARG;
+  if (cache_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  DecodePlan pl;
+  st = plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(),
+                   cache_seqlens != nullptr, &pl);
+  if (st != FA_OK) return st;
+  const size_t need = decode_workspace_bytes(pl, d);
+  if (need > 0 && (!aligned16(workspace) || workspace_bytes_ < need)) return FA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (n_new > 0) {
+    const long long units = static_cast<long long>(B) * n_new * Hkv * (d / 8);
+    const long long blocks = (units + 255) / 256 < 4096 ? (units + 255) / 256 : 4096;
+    TraceScope tr(FA_KERNEL_KVCACHE_APPEND, s);
+    fa_kvcache_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache),
+        static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), cache_seqlens, B,
+        n_new, Nk, Hkv, d);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  switch (d) {
+    case 64:
+      return launch_decode<64, Dec64>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
+                                      cache_seqlens, n_new, workspace, s);
+    case 128:
+      return launch_decode<128, Dec128>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
+                                        cache_seqlens, n_new, workspace, s);
+    default:
+      return launch_decode<256, Dec256>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
+                                        cache_seqlens, n_new, workspace, s);
   }
 }
 

@@ -40,9 +40,13 @@ struct DecodeParams {
   int B, Nq, Nk, Hq, Hkv, group;  // group = Hq / Hkv
   int qpt;                        // query rows per tile; rows per tile RT = qpt * group <= 128
   int n_qtiles;                   // ceil(Nq / qpt)
-  int n_splits;                   // key splits per (batch, kv head, query tile)
+  int n_splits;                   // most key splits of a (batch, kv head, query tile) unit
+  int split_tiles;                // key tiles per split; a unit with n visible key tiles
+                                  // uses ceil(n / split_tiles) splits (at least 1)
   float scale_log2;
-  MaskSpec mask;
+  MaskSpec mask;                  // with Nk = the key capacity; per batch see below
+  const int* seqlens;             // [B] cached keys per sequence, or null (all Nk)
+  int n_new;                      // keys appended after seqlens[b] by this call
   __nv_bfloat16* o;               // [B, Nq, Hq, d]
   float* lse;                     // [B, Hq, Nq]
   float* part_o;                  // [units, n_splits, RT, d] normalised partial O (n_splits > 1)
@@ -179,12 +183,25 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int RT = p.qpt * G;
   const int i_first = qt * p.qpt;
   const int i_last = min(p.Nq - 1, i_first + p.qpt - 1);
-  const int key_lo = p.mask.lo(i_first), key_hi = p.mask.hi(i_last);
+  // keys of this sequence: the whole capacity, or its cached length plus the
+  // keys appended by this call (clamped to the capacity); the causal diagonal
+  // and the window are aligned to that length
+  MaskSpec mask = p.mask;
+  if (p.seqlens != nullptr) mask.Nk = max(0, min(p.Nk, __ldg(p.seqlens + b) + p.n_new));
+  const int key_lo = mask.lo(i_first), key_hi = mask.hi(i_last);
   const int j_all = key_lo / BN;
   const int n_all = (key_hi >= key_lo) ? (key_hi / BN - j_all + 1) : 0;
-  const int per_split = (n_all + p.n_splits - 1) / p.n_splits;
-  const int t_begin = min(n_all, split * per_split);
-  const int n_kv = min(n_all, t_begin + per_split) - t_begin;
+  // this unit's splits: a fixed number of key tiles each, so a sequence with
+  // fewer keys (ragged cache lengths) takes fewer CTAs; the others leave at once
+  int split_tiles = p.split_tiles;
+  int ns = max(1, (n_all + split_tiles - 1) / split_tiles);
+  if (ns > p.n_splits) {  // more tiles than the launch planned for: spread them over its splits
+    split_tiles = (n_all + p.n_splits - 1) / p.n_splits;
+    ns = max(1, (n_all + split_tiles - 1) / split_tiles);
+  }
+  if (split >= ns) return;
+  const int t_begin = split * split_tiles;
+  const int n_kv = min(n_all, t_begin + split_tiles) - t_begin;
   const int j_begin = j_all + t_begin;
 
   auto load_k = [&](int it) {
@@ -326,7 +343,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const int tl = warp * 32 + lane;              // TMEM lane = c * RCP + rr
     const int i = i_first + rr / G;
     const bool row_ok = rr < RT && i < p.Nq;
-    const int lo = row_ok ? p.mask.lo(i) : 1, hi = row_ok ? p.mask.hi(i) : 0;
+    const int lo = row_ok ? mask.lo(i) : 1, hi = row_ok ? mask.hi(i) : 0;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const float sl2 = p.scale_log2;
     if constexpr (NC > 1) {
@@ -446,7 +463,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const bool aborted = *abort_flag != 0;
     if (!aborted) {
       const long long unit = static_cast<long long>(bk) * p.n_qtiles + qt;
-      if (p.n_splits == 1) {
+      if (ns == 1) {
         constexpr int UPR = D / 8;
         for (int x = threadIdx.x; x < RT * UPR; x += BM) {
           const int r2 = x / UPR, col = (x % UPR) * 8;
@@ -490,23 +507,23 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
         // count merges all of them
         __threadfence();
         named_bar_sync(1, BM);
-        if (threadIdx.x == 0) *last_flag = decode_claim_last(p.counters + unit, p.tag, p.n_splits) ? 1 : 0;
+        if (threadIdx.x == 0) *last_flag = decode_claim_last(p.counters + unit, p.tag, ns) ? 1 : 0;
         named_bar_sync(1, BM);
-        if (*last_flag && p.n_splits * RT <= C::STAGE_FLOATS) {
+        if (*last_flag && ns * RT <= C::STAGE_FLOATS) {
           // the unit's partial LSEs (contiguous, [split][row]) into shared
           // memory in one parallel pass, then turned into merge weights
           __threadfence();
           const size_t ubase = static_cast<size_t>(unit) * p.n_splits * RT;  // split s, row r: ubase + s RT + r
-          const int nsr = p.n_splits * RT;
+          const int nsr = ns * RT;
           for (int x = threadIdx.x; x < nsr; x += BM) stage[x] = __ldcg(p.part_lse + ubase + x);
           named_bar_sync(1, BM);
           if (threadIdx.x < RT) {
             const int r2 = threadIdx.x;
             float mx = -INFINITY;
-            for (int s = 0; s < p.n_splits; ++s) mx = fmaxf(mx, stage[s * RT + r2]);
+            for (int s = 0; s < ns; ++s) mx = fmaxf(mx, stage[s * RT + r2]);
             float sum = 0.f;
             if (mx != -INFINITY) {
-              for (int s = 0; s < p.n_splits; ++s) {
+              for (int s = 0; s < ns; ++s) {
                 const float ls = stage[s * RT + r2];
                 if (ls != -INFINITY) sum += ex2_approx((ls - mx) * kLog2e);
               }
@@ -531,7 +548,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = 0.f;
 #pragma unroll 4
-            for (int s = 0; s < p.n_splits; ++s) {
+            for (int s = 0; s < ns; ++s) {
               const float w = stage[s * RT + r2];
               const size_t row = ubase + static_cast<size_t>(s) * RT + r2;
               const float4 a = __ldcg(reinterpret_cast<const float4*>(p.part_o + row * D + col));
@@ -554,10 +571,10 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
           if (threadIdx.x < RT) {
             const int r2 = threadIdx.x;
             float mx = -INFINITY;
-            for (int s = 0; s < p.n_splits; ++s) mx = fmaxf(mx, __ldcg(p.part_lse + ubase + static_cast<size_t>(s) * RT + r2));
+            for (int s = 0; s < ns; ++s) mx = fmaxf(mx, __ldcg(p.part_lse + ubase + static_cast<size_t>(s) * RT + r2));
             float sum = 0.f;
             if (mx != -INFINITY) {
-              for (int s = 0; s < p.n_splits; ++s) {
+              for (int s = 0; s < ns; ++s) {
                 const float ls = __ldcg(p.part_lse + ubase + static_cast<size_t>(s) * RT + r2);
                 if (ls != -INFINITY) sum += ex2_approx((ls - mx) * kLog2e);
               }
@@ -578,7 +595,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = 0.f;
             if (Lr != -INFINITY) {
-              for (int s = 0; s < p.n_splits; ++s) {
+              for (int s = 0; s < ns; ++s) {
                 const size_t row = ubase + static_cast<size_t>(s) * RT + r2;
                 const float ls = __ldcg(p.part_lse + row);
                 if (ls == -INFINITY) continue;
@@ -605,6 +622,32 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == C::MMA_WARP) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// In-place append of the new keys and values to the caches: row t of
+// sequence b goes to cache row seqlens[b] + t (rows at or past the capacity
+// Nk are dropped).  One thread per 16 bytes of a row of K and of V.
+__global__ void __launch_bounds__(256)
+    fa_kvcache_append_kernel(__nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache,
+                             const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __restrict__ v_new,
+                             const int* __restrict__ seqlens, int B, int n_new, int Nk, int Hkv, int d) {
+  const int upr = d / 8;  // 16-byte units per row
+  const long long total = static_cast<long long>(B) * n_new * Hkv * upr;
+  for (long long x = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; x < total;
+       x += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int u = static_cast<int>(x % upr);
+    const long long row = x / upr;  // (b, t, h)
+    const int h = static_cast<int>(row % Hkv);
+    const long long bt = row / Hkv;
+    const int t = static_cast<int>(bt % n_new);
+    const int b = static_cast<int>(bt / n_new);
+    const int dst = __ldg(seqlens + b) + t;
+    if (dst < 0 || dst >= Nk) continue;
+    const size_t src_off = static_cast<size_t>(row) * d + u * 8;
+    const size_t dst_off = ((static_cast<size_t>(b) * Nk + dst) * Hkv + h) * d + u * 8;
+    *reinterpret_cast<uint4*>(k_cache + dst_off) = __ldg(reinterpret_cast<const uint4*>(k_new + src_off));
+    *reinterpret_cast<uint4*>(v_cache + dst_off) = __ldg(reinterpret_cast<const uint4*>(v_new + src_off));
+  }
 }
 
 }  // namespace fa

@@ -159,6 +159,39 @@ int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* 
                    int n_splits, void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_fwd_splitkv over a key/value cache, with the cache update of
+ * hysenlabs' `flash_attn_with_kvcache` (Python-interface section): the new
+ * keys and values are written into the caches in place, then the query rows
+ * attend to each sequence's cached keys plus the new ones.
+ *   k_cache, v_cache [B, Nk, Hkv, d] : caches (bf16, device); Nk is their
+ *                      capacity in keys.  Updated in place when n_new > 0.
+ *   k_new, v_new [B, n_new, Hkv, d]   : keys/values to append (bf16, device);
+ *                      ignored (may be NULL) when n_new == 0
+ *   cache_seqlens [B] : int32, device, 4-byte aligned: keys already cached
+ *                      per sequence.  Row t of k_new/v_new goes to cache row
+ *                      cache_seqlens[b] + t (rows at or past Nk are dropped),
+ *                      and sequence b attends to its first
+ *                      min(Nk, cache_seqlens[b] + n_new) keys.  NULL: every
+ *                      sequence holds all Nk keys (then n_new must be 0).
+ *                      The array is not modified.
+ *   q, o, lse, masks, n_splits, workspace: as fa_fwd_splitkv, with the
+ *                      workspace size from fa_fwd_kvcache_workspace_size.
+ *                      The causal diagonal and the window of sequence b are
+ *                      aligned to its own key count (bottom-right).
+ * The keys are split in chunks of equal length planned for the full capacity
+ * Nk, so a shorter sequence takes fewer CTAs.  With cache_seqlens given and
+ * n_splits 0, the library plans about three waves of CTAs at full length
+ * (instead of one), so that ragged batches balance.
+ * Returns FA_OK or an fa_status code.
+ */
+size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Nk, int Hq, int Hkv, int d, int causal,
+                                     int win_l, int win_r, int n_splits, int with_seqlens);
+int fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                   const int* cache_seqlens, void* o, float* lse, int B, int Nq, int Nk, int n_new,
+                   int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r, int n_splits,
+                   void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fp32 variants for small problems (fp32 in, fp32 out, fp32 arithmetic on the
  * CUDA cores).  Same arguments and semantics as fa_fwd / fa_bwd; d <= 256 and
  * d a multiple of 32.
@@ -197,8 +230,9 @@ enum fa_kernel_kind {
   FA_KERNEL_BWD_DQ = 2,   /* backward dQ, bf16 (tcgen05) */
   FA_KERNEL_BWD_DKDV = 3, /* backward dK/dV, bf16 (tcgen05) */
   FA_KERNEL_F32 = 4,      /* any fp32-path kernel */
-  FA_KERNEL_DECODE = 5,   /* fa_fwd_splitkv, bf16 (tcgen05) */
-  FA_KERNEL_KINDS = 6
+  FA_KERNEL_DECODE = 5,   /* fa_fwd_splitkv / fa_fwd_kvcache, bf16 (tcgen05) */
+  FA_KERNEL_KVCACHE_APPEND = 6, /* fa_fwd_kvcache: new keys/values into the cache */
+  FA_KERNEL_KINDS = 7
 };
 int fa_trace_enable(int on);
 int fa_trace_read(double* ms, long long* launches);

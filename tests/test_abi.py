@@ -25,8 +25,8 @@ def declared_functions():
 def test_header_declares_the_expected_entry_points():
     assert declared_functions() == sorted([
         "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
-        "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size",
-        "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
+        "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
+        "fa_fwd_kvcache_workspace_size", "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
 
 
 def test_kernel_kinds_match_the_header():
@@ -171,3 +171,30 @@ def test_splitkv_rejects_unsupported_and_missing_workspace():
     assert _splitkv(ws=0, wsb=need) == WORKSPACE
     assert _splitkv(ws=FAKE, wsb=need - 4) == WORKSPACE
     assert _splitkv(ws=MISALIGNED, wsb=need) == WORKSPACE
+
+
+def _kvcache(**kw):
+    a = dict(q=FAKE, kc=FAKE, vc=FAKE, kn=FAKE, vn=FAKE, sl=FAKE, o=FAKE, lse=FAKE, B=2, Nq=1,
+             Nk=1000, n_new=1, Hq=8, Hkv=2, d=128, scale=0.125, causal=1, win_l=-1, win_r=-1,
+             n_splits=4, ws=FAKE, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return fa.fa_fwd_kvcache(a["q"], a["kc"], a["vc"], a["kn"], a["vn"], a["sl"], a["o"], a["lse"],
+                             a["B"], a["Nq"], a["Nk"], a["n_new"], a["Hq"], a["Hkv"], a["d"],
+                             a["scale"], a["causal"], a["win_l"], a["win_r"], a["n_splits"], a["ws"],
+                             a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=0), dict(kc=0), dict(vc=MISALIGNED), dict(o=0), dict(lse=0), dict(B=0), dict(Nk=0),
+    dict(n_new=-1), dict(kn=0), dict(vn=MISALIGNED), dict(sl=0), dict(sl=FAKE + 2),
+    dict(Hq=6, Hkv=4), dict(scale=float("inf")), dict(n_splits=5000),
+])
+def test_kvcache_rejects_invalid_arguments(kw):
+    assert _kvcache(**kw) == INVALID
+
+
+def test_kvcache_rejects_unsupported_and_missing_workspace():
+    assert _kvcache(d=96) == UNSUPPORTED
+    assert _kvcache(Hq=512, Hkv=2) == UNSUPPORTED
+    assert _kvcache(ws=0) == WORKSPACE
+    assert _kvcache(wsb=16) == WORKSPACE

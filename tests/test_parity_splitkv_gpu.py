@@ -58,7 +58,7 @@ CASES = [
     (2, 1, 1000, 8, 2, 128, False, (-1, -1), 0),    # ragged Nk, library's split count
     (2, 1, 1000, 8, 2, 128, False, (-1, -1), 1),    # no split: output written by the main kernel
     (2, 1, 1000, 8, 2, 128, False, (-1, -1), 3),
-    (1, 1, 700, 4, 4, 64, False, (-1, -1), 16),     # MHA; 6 key tiles, 10 splits get none
+    (1, 1, 700, 4, 4, 64, False, (-1, -1), 16),     # MHA; more splits asked for than its 6 key tiles
     (2, 2, 1500, 16, 1, 64, True, (-1, -1), 5),     # 32 packed rows: 4 copies
     (1, 3, 1200, 16, 1, 256, True, (300, 0), 4),    # 48 rows: 2 copies; window; d 256
     (1, 3, 2000, 32, 1, 128, True, (-1, -1), 0),    # MQA, 96 rows: 1 copy
