@@ -3,13 +3,14 @@
 The C ABI (include/fa.h) is the product boundary; this module only marshals
 arguments to it.  Two layers:
 
-* ``fa_fwd``, ``fa_bwd``, ``fa_fwd_splitkv``, ``fa_fwd_kvcache``, ``fa_fwd_f32``, ``fa_bwd_f32``,
+* ``fa_fwd``, ``fa_bwd``, ``fa_fwd_varlen``, ``fa_fwd_splitkv``, ``fa_fwd_kvcache``,
+  ``fa_fwd_f32``, ``fa_bwd_f32``,
   ``fa_bwd_workspace_size``, ``fa_fwd_splitkv_workspace_size``,
   ``fa_get_device_status``, ``fa_status_string``: the C entry points under the
   same names, taking raw device pointers (ints) and sizes, returning the
   status code.
-* ``attention_forward`` / ``attention_backward`` / ``attention_forward_splitkv`` /
-  ``attention_forward_kvcache``:
+* ``attention_forward`` / ``attention_backward`` / ``attention_forward_varlen`` /
+  ``attention_forward_splitkv`` / ``attention_forward_kvcache``:
   the same calls on torch CUDA tensors (torch only allocates the outputs and
   the workspace and supplies the current stream).
 
@@ -23,11 +24,11 @@ import os
 __all__ = [
     "FAError", "load_library", "library_path",
     "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
-    "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
+    "fa_fwd_varlen", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
     "fa_fwd_kvcache_workspace_size",
     "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
     "KERNEL_KINDS", "attention_forward", "attention_backward", "attention_forward_splitkv",
-    "attention_forward_kvcache",
+    "attention_forward_kvcache", "attention_forward_varlen",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -73,6 +74,7 @@ def load_library():
     lib.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, i, vp, sz, vp]
     lib.fa_fwd_splitkv_workspace_size.argtypes = [i, i, i, i, i, i, i, i, i, i]
     lib.fa_fwd_splitkv_workspace_size.restype = sz
+    lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, i, i, vp]
     lib.fa_fwd_kvcache_workspace_size.argtypes = [i, i, i, i, i, i, i, i, i, i, i]
     lib.fa_fwd_kvcache_workspace_size.restype = sz
     lib.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i,
@@ -82,7 +84,7 @@ def load_library():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_trace_enable.argtypes = [i]
     lib.fa_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
-    for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache",
+    for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache", "fa_fwd_varlen",
                  "fa_get_device_status",
                  "fa_trace_enable", "fa_trace_read"):
         getattr(lib, name).restype = i
@@ -116,6 +118,14 @@ def fa_fwd_splitkv(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l,
     """Forward for few query rows over a long key range, split across CTAs."""
     return load_library().fa_fwd_splitkv(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal,
                                          win_l, win_r, n_splits, workspace, workspace_bytes, stream)
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                  total_q, total_k, Hq, Hkv, d, scale, causal, win_l, win_r, stream):
+    """Forward over packed variable-length sequences."""
+    return load_library().fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q,
+                                        max_seqlen_k, total_q, total_k, Hq, Hkv, d, scale, causal,
+                                        win_l, win_r, stream)
 
 
 def fa_fwd_kvcache(q, k_cache, v_cache, k_new, v_new, cache_seqlens, o, lse, B, Nq, Nk, n_new, Hq,
@@ -254,6 +264,38 @@ def attention_forward_splitkv(q, k, v, scale=None, causal=False, window=(-1, -1)
                           B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, int(n_splits),
                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                           _stream()))
+    return o, lse
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                             scale=None, causal=False, window=(-1, -1), out=None, lse=None):
+    """O, LSE for packed sequences through fa_fwd_varlen (bf16 only).
+
+    q [total_q, Hq, d], k/v [total_k, Hkv, d] contiguous; cu_seqlens_q/k int32
+    CUDA tensors of B + 1 offsets.  Returns (o like q, lse [Hq, total_q])."""
+    import torch
+    if q.dim() != 3 or k.dim() != 3 or v.dim() != 3 or k.shape != v.shape or k.shape[2] != q.shape[2]:
+        raise ValueError("q must be [total_q, Hq, d] and k, v [total_k, Hkv, d]")
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    for t in (cu_seqlens_q, cu_seqlens_k):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.dim() != 1:
+            raise ValueError("cu_seqlens must be contiguous int32 CUDA vectors")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold B + 1 offsets")
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check("fa_fwd_varlen",
+           fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                         cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
+                         int(max_seqlen_k), total_q, total_k, Hq, Hkv, d, scale, c, wl, wr,
+                         _stream()))
     return o, lse
 
 

@@ -145,10 +145,48 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.n_qgroups = (Nq + C::NQT * C::BM - 1) / (C::NQT * C::BM);
   p.head_chunk = head_chunk(B * Hq, 4ll * Nk * C::D);  // K and V of one head, bf16
   p.lse = lse;
+  p.cu_q = nullptr;
+  p.cu_k = nullptr;
+  p.total_q = 0;
+  p.o = static_cast<__nv_bfloat16*>(o);
   p.wait_limit_ns = kWaitLimitNs;
   auto kern = fa_fwd_kernel<C>;
   if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
   const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
+  {
+    TraceScope tr(FA_KERNEL_FWD, stream);
+    kern<<<static_cast<unsigned>(grid), C::NTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+  }
+  return launch_status();
+}
+
+// Packed sequences: the tensors are one batch of total_q / total_k rows;
+// sequence b is rows [cu_q[b], cu_q[b+1]) and [cu_k[b], cu_k[b+1]).
+template <class C>
+int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_q,
+                      const int* cu_k, int B, int max_q, int max_k, int total_q, int total_k, int Hq,
+                      int Hkv, float scale, int causal, int win_l, int win_r, cudaStream_t stream) {
+  static int attr_done[kMaxDevices] = {0};
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_bnhd(&tq, q, 1, total_q, Hq, C::D, C::BM) || !encode_bnhd(&tk, k, 1, total_k, Hkv, C::D, C::BN) ||
+      !encode_bnhd(&tv, v, 1, total_k, Hkv, C::D, C::BN) || !encode_bnhd(&to, o, 1, total_q, Hq, C::D, C::BM))
+    return FA_ERR_CUDA;
+  FwdParams p;
+  p.B = B; p.Nq = max_q; p.Nk = max_k; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
+  p.scale_log2 = scale * kLog2e;
+  p.mask = make_mask(max_q, max_k, causal, win_l, win_r);
+  p.n_qgroups = (max_q + C::NQT * C::BM - 1) / (C::NQT * C::BM);
+  p.head_chunk = head_chunk(B * Hq, 4ll * max_k * C::D);
+  p.lse = lse;
+  p.cu_q = cu_q;
+  p.cu_k = cu_k;
+  p.total_q = total_q;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.wait_limit_ns = kWaitLimitNs;
+  auto kern = fa_fwd_kernel<C>;
+  if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
+  const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
+  if (grid > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
   {
     TraceScope tr(FA_KERNEL_FWD, stream);
     kern<<<static_cast<unsigned>(grid), C::NTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
@@ -555,6 +593,35 @@ int fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_ne
     default:
       return launch_decode<256, Dec256>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
                                         cache_seqlens, n_new, workspace, s);
+  }
+}
+
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                  int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, float scale,
+                  int causal, int win_l, int win_r, fa_stream_t stream) {
+  int st = check_common(q, k, v, 1, total_q, total_k, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || max_seqlen_q < 1 || max_seqlen_k < 1 || max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Hq * ((max_seqlen_q + 127) / 128) > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64:
+      return launch_fwd_varlen<Fwd64>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                                      total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
+    case 128:
+      return launch_fwd_varlen<Fwd128>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                                       total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
+    case 256:
+      return launch_fwd_varlen<Fwd256>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                                       total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
+    default:
+      return FA_ERR_UNSUPPORTED;
   }
 }
 

@@ -42,7 +42,14 @@ struct FwdParams {
   MaskSpec mask;
   int n_qgroups;                  // CTAs along the query axis
   int head_chunk;                 // heads per scheduling chunk (see ChunkedOrder)
-  float* lse;                     // [B, Hq, Nq]
+  float* lse;                     // [B, Hq, Nq]; packed sequences: [Hq, total_q]
+  // packed sequences (null when dense): sequence b holds query rows
+  // [cu_q[b], cu_q[b+1]) and key rows [cu_k[b], cu_k[b+1]) of tensors seen
+  // as one batch; Nq / Nk are then the longest sequence's lengths
+  const int* cu_q;
+  const int* cu_k;
+  int total_q;
+  __nv_bfloat16* o;               // O, for the plain stores of a packed sequence's last tile
   unsigned long long wait_limit_ns;
 };
 
@@ -186,29 +193,42 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const ChunkedOrder order(blockIdx.x, p.B * p.Hq, p.n_qgroups, p.head_chunk);
   const int bh = order.head;
   const int g = p.n_qgroups - 1 - order.rank;
-  const int b = bh / p.Hq, h = bh % p.Hq, hk = h / p.group;
+  const int h = bh % p.Hq, hk = h / p.group;
   const int r0 = g * NQT * BM;
-  const int r_last = min(p.Nq - 1, r0 + NQT * BM - 1);
-  const int key_lo = p.mask.lo(r0), key_hi = p.mask.hi(r_last);
+  // dense: batch b of the tensors; packed: sequence b at row offsets
+  // q_off / k_off of one-batch tensors (tb = 0), its own lengths and masks
+  int b = bh / p.Hq, q_off = 0, k_off = 0;
+  MaskSpec mask = p.mask;
+  if (p.cu_q != nullptr) {
+    q_off = __ldg(p.cu_q + b);
+    k_off = __ldg(p.cu_k + b);
+    mask.Nq = __ldg(p.cu_q + b + 1) - q_off;
+    mask.Nk = __ldg(p.cu_k + b + 1) - k_off;
+    if (r0 >= mask.Nq) return;  // this sequence has no query group g
+  }
+  const int nq = mask.Nq;
+  const int tb = p.cu_q != nullptr ? 0 : b;
+  const int r_last = min(nq - 1, r0 + NQT * BM - 1);
+  const int key_lo = mask.lo(r0), key_hi = mask.hi(r_last);
   const int j_begin = key_lo / BN;
   const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
 
   // Copies of key tile `it` into ring stage it % KST (K and V on one barrier
   // with two Q tiles, on their own barriers with one)
   auto load_k = [&](int it) {
-    const int s = it % KST, krow = (j_begin + it) * BN;
+    const int s = it % KST, krow = k_off + (j_begin + it) * BN;
     uint64_t* bar = &k_full[s];
     mbar_expect_tx(bar, (NQT == 2 ? 2 : 1) * C::KTILE);
     for (int c = 0; c < C::NCHUNK; ++c) {
-      tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, bar, c * 64, hk, krow, b);
-      if (NQT == 2) tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, bar, c * 64, hk, krow, b);
+      tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, bar, c * 64, hk, krow, tb);
+      if (NQT == 2) tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, bar, c * 64, hk, krow, tb);
     }
   };
   auto load_v = [&](int it) {  // NQT == 1 only
-    const int s = it % KST, krow = (j_begin + it) * BN;
+    const int s = it % KST, krow = k_off + (j_begin + it) * BN;
     mbar_expect_tx(&v_full[s], C::KTILE);
     for (int c = 0; c < C::NCHUNK; ++c)
-      tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[s], c * 64, hk, krow, b);
+      tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[s], c * 64, hk, krow, tb);
   };
   // The TMA thread sets up the barriers and issues Q and the first KST key
   // tiles (no stage to wait for yet) before the block-wide sync, so the
@@ -234,7 +254,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       mbar_expect_tx(bar_q, NQT * C::QTILE);
       for (int t = 0; t < NQT; ++t)
         for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sQ + t * C::QTILE + c * C::QCHUNK, &tm_q, bar_q, c * 64, h, r0 + t * BM, b);
+          tma_load_4d(sQ + t * C::QTILE + c * C::QCHUNK, &tm_q, bar_q, c * 64, h, q_off + r0 + t * BM, tb);
       for (int it = 0; it < n_pre; ++it) {
         load_k(it);
         if (NQT == 1) load_v(it);
@@ -400,7 +420,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const int t = warp / 4;          // Q tile of this warpgroup
     const int r = threadIdx.x % BM;  // row within the tile == TMEM lane
     const int row = r0 + t * BM + r;
-    const int lo = p.mask.lo(row), hi = p.mask.hi(row);
+    const int lo = mask.lo(row), hi = mask.hi(row);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     const float sl2 = p.scale_log2;
     float m_ref = -INFINITY;  // reference max, exp2 domain (scale folded in)
@@ -552,16 +572,37 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
     named_bar_sync(1 + t, BM);
     const bool aborted = *abort_flag != 0;
-    if (r == 0 && !aborted && r0 + t * BM < p.Nq) {
-      for (int c = 0; c < C::NCHUNK; ++c)
-        tma_store_4d(&tm_o, sQt + c * C::QCHUNK, c * 64, h, r0 + t * BM, b);
-      tma_store_commit();
-      tma_store_wait_read();
+    const int t_row0 = r0 + t * BM;
+    if (p.cu_q == nullptr || t_row0 + BM <= nq) {
+      // whole tile (or dense, where TMA clips the tensor's last tile itself)
+      if (r == 0 && !aborted && t_row0 < nq) {
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_store_4d(&tm_o, sQt + c * C::QCHUNK, c * 64, h, q_off + t_row0, tb);
+        tma_store_commit();
+        tma_store_wait_read();
+      }
+    } else if (!aborted) {
+      // last tile of a packed sequence: rows past its end belong to the next
+      // sequence, so only the valid rows are stored, 16 bytes at a time
+      constexpr int UPR = D / 8;
+      const int n_rows = nq - t_row0;
+      for (int x = r; x < n_rows * UPR; x += BM) {
+        const int rr = x / UPR, u = x % UPR;
+        const int gq = q_off + t_row0 + rr;
+        if (gq < 0 || gq >= p.total_q) continue;  // offsets outside the tensor: never written
+        uint32_t w0, w1, w2, w3;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                     : "r"(sQt + (u / 8) * C::QCHUNK + sw128_offset(rr, u % 8)));
+        *reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(gq) * p.Hq + h) * D + u * 8) =
+            make_uint4(w0, w1, w2, w3);
+      }
     }
-    if (!aborted && row < p.Nq) {
+    if (!aborted && row < nq && (p.cu_q == nullptr || (q_off + row >= 0 && q_off + row < p.total_q))) {
       const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
-      p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Nq + row] =
-          (l > 0.f) ? (mb + log2f(l)) * kLn2 : -INFINITY;
+      const size_t lse_row = p.cu_q != nullptr ? static_cast<size_t>(h) * p.total_q + q_off + row
+                                                : (static_cast<size_t>(b) * p.Hq + h) * p.Nq + row;
+      p.lse[lse_row] = (l > 0.f) ? (mb + log2f(l)) * kLn2 : -INFINITY;
     }
   } else {
     setmaxnreg_dec<C::REG_PRODUCER>();  // idle members of the producer warpgroup

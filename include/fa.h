@@ -77,6 +77,26 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
            fa_stream_t stream);
 
 /*
+ * Forward pass over packed variable-length sequences (hysenlabs changelog
+ * v2.0: the varlen functions), bf16.  The B sequences are stored back to back:
+ *   q, o [total_q, Hq, d], k, v [total_k, Hkv, d]  (bf16, device)
+ *   lse [Hq, total_q]                                (fp32, device)
+ *   cu_seqlens_q, cu_seqlens_k [B + 1]               (int32, device, 4-byte aligned)
+ * Sequence b is query rows [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key rows
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]); it attends to its own keys only, with
+ * fa_fwd's masks applied to its own lengths (causal bottom-right per
+ * sequence).  The caller guarantees 0 <= cu[b] <= cu[b+1] <= total and every
+ * length <= max_seqlen (a longer sequence is computed only up to
+ * max_seqlen_q rows); the kernel never writes outside [0, total_q) rows of o
+ * and lse whatever the offsets hold.  Rows of o and lse not covered by any
+ * sequence are left untouched.  Other arguments as fa_fwd.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                  int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, float scale,
+                  int causal, int win_l, int win_r, fa_stream_t stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes: two fp32 arrays
  * [B, Hq, Nq rounded up to 256], the row sums D = rowsum(dO * O) and the
  * saved LSE in base 2.  Returns 0 for invalid sizes.

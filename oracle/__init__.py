@@ -129,6 +129,29 @@ def attn_bwd(q, k, v, dout, scale=None, causal=False, window=(-1, -1), nthreads=
     return dq, dk, dv
 
 
+def attn_fwd_varlen(q, k, v, cu_q, cu_k, scale=None, causal=False, window=(-1, -1), nthreads=None):
+    """Packed variable-length sequences: q [total_q, Hq, d], k/v [total_k, Hkv,
+    d], offsets cu_q / cu_k of B + 1 entries.  Each sequence is the plain
+    attention of its own rows (attn_fwd with one batch), masks aligned to its
+    own lengths.  Returns O [total_q, Hq, d] (zero on rows no sequence covers)
+    and LSE [Hq, total_q] (-inf there)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    total_q, Hq, d = q.shape
+    o = np.zeros_like(q)
+    lse = np.full((Hq, total_q), -np.inf)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 <= q0:
+            continue
+        if k1 <= k0:  # no keys at all: every row is empty
+            continue
+        ob, lb = attn_fwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], scale=scale,
+                          causal=causal, window=window, nthreads=nthreads)
+        o[q0:q1] = ob[0]
+        lse[:, q0:q1] = lb[0]
+    return o, lse
+
+
 def merge_partials(o_parts, lse_parts):
     """Merge attention results computed over disjoint key subsets.
 

@@ -12,6 +12,14 @@ P = 1 and dS = P (dP - D) = 0 exactly), a relative error is undefined; the
 GPU value must then be below ZERO_ABS in absolute terms (dS is left with
 rounding noise from the bf16 O used in D).
 
+O is returned in bf16, rounded to nearest-even, so even an exactly rounded
+copy of the oracle's value differs from it by up to half a unit in the last
+place, at most |O| * 2^-8 (8 significant bits).  Where |O| is large -- rows
+that see only a few keys, whose output is close to single V rows -- that
+alone exceeds 1e-2 (|O| = 4 allows 1.6e-2).  The O bound is therefore
+1e-2 on top of that rounding allowance (o_error below); for the |O| << 1 of
+long rows it is the plain 1e-2.
+
 Stress inputs outside the N(0,1) regime (a peaked softmax) use the criterion
 of the FlashAttention test suite (hysenlabs page, section on tests): the
 error against the reference must be at most twice the error of a plain
@@ -30,6 +38,18 @@ from seeded_inputs import make_inputs
 TOL_BF16 = dict(o=1e-2, lse=1e-3, grad=2e-2)
 TOL_F32 = dict(o=1e-4, lse=1e-4, grad=1e-4)
 ZERO_ABS = 1e-3
+
+
+BF16_HALF_ULP_REL = 2.0 ** -8  # bound on bf16 rounding error relative to |x|
+
+
+def o_error(o_gpu, o_ref, dtype="bf16"):
+    """Max |o_gpu - o_ref| beyond the rounding of the output format itself
+    (|o_ref| * 2^-8 for bf16 outputs; none for fp32)."""
+    diff = np.abs(np.asarray(o_gpu, dtype=np.float64) - o_ref)
+    if dtype == "bf16":
+        diff = diff - BF16_HALF_ULP_REL * np.abs(o_ref)
+    return float(diff.max()) if diff.size else 0.0
 
 
 def rel_fro(a, b):
@@ -73,8 +93,8 @@ def run_case(B, Nq, Nk, Hq, Hkv, d, causal=False, window=(-1, -1), seed=0, dtype
                                      window=window)
     what = "B%d Nq%d Nk%d Hq%d Hkv%d d%d causal%d win%s %s" % (B, Nq, Nk, Hq, Hkv, d, causal,
                                                               window, dtype)
-    err_o = float(np.abs(g["o"] - o_ref).max())
-    assert err_o <= tol["o"], "%s: O max err %.3e" % (what, err_o)
+    err_o = o_error(g["o"], o_ref, dtype)
+    assert err_o <= tol["o"], "%s: O max err %.3e (beyond output rounding)" % (what, err_o)
     compare_lse(g["lse"], lse_ref, tol["lse"], what)
     res = {"o": err_o}
     if backward:

@@ -26,7 +26,7 @@ def test_header_declares_the_expected_entry_points():
     assert declared_functions() == sorted([
         "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
         "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
-        "fa_fwd_kvcache_workspace_size", "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
+        "fa_fwd_kvcache_workspace_size", "fa_fwd_varlen", "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
 
 
 def test_kernel_kinds_match_the_header():
@@ -198,3 +198,25 @@ def test_kvcache_rejects_unsupported_and_missing_workspace():
     assert _kvcache(Hq=512, Hkv=2) == UNSUPPORTED
     assert _kvcache(ws=0) == WORKSPACE
     assert _kvcache(wsb=16) == WORKSPACE
+
+
+def _varlen(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, cq=FAKE, ck=FAKE, B=3, mq=100, mk=120, tq=200,
+             tk=250, Hq=4, Hkv=2, d=128, scale=0.125, causal=1, win_l=-1, win_r=-1, stream=None)
+    a.update(kw)
+    return fa.fa_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cq"], a["ck"], a["B"],
+                            a["mq"], a["mk"], a["tq"], a["tk"], a["Hq"], a["Hkv"], a["d"], a["scale"],
+                            a["causal"], a["win_l"], a["win_r"], a["stream"])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(q=0), dict(k=MISALIGNED), dict(o=0), dict(lse=MISALIGNED), dict(cq=0), dict(ck=0),
+    dict(cq=FAKE + 2), dict(B=0), dict(mq=0), dict(mk=0), dict(mq=201), dict(mk=251), dict(tq=0),
+    dict(Hq=3), dict(scale=float("nan")),
+])
+def test_varlen_rejects_invalid_arguments(kw):
+    assert _varlen(**kw) == INVALID
+
+
+def test_varlen_rejects_unsupported_head_dim():
+    assert _varlen(d=96) == UNSUPPORTED

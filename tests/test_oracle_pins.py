@@ -368,3 +368,38 @@ def test_merge_rows_without_keys():
     o, lse = oracle.merge_partials([o_a, o_b], [lse_a, lse_b])
     assert np.isneginf(lse[0, 0, 0]) and np.all(o[0, 0] == 0.0)
     assert lse[0, 0, 1] == 0.25 and np.all(o[0, 1] == 1.0)
+
+
+# ------------------------------------------------------- packed sequences
+
+def test_varlen_of_equal_lengths_is_the_batched_attention():
+    rng = np.random.default_rng(23)
+    B, N, Hq, Hkv, d = 3, 9, 4, 2, 8
+    q = rng.standard_normal((B, N, Hq, d))
+    k = rng.standard_normal((B, N, Hkv, d))
+    v = rng.standard_normal((B, N, Hkv, d))
+    cu = np.arange(B + 1) * N
+    o, lse = oracle.attn_fwd_varlen(q.reshape(B * N, Hq, d), k.reshape(B * N, Hkv, d),
+                                    v.reshape(B * N, Hkv, d), cu, cu, causal=True)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, causal=True)
+    assert np.abs(o - o_ref.reshape(B * N, Hq, d)).max() < 1e-14
+    assert np.abs(lse - np.transpose(lse_ref, (1, 0, 2)).reshape(Hq, B * N)).max() < 1e-14
+
+
+def test_varlen_sequences_do_not_see_each_other():
+    """Changing the keys of one sequence changes no other sequence's output;
+    rows outside every sequence stay empty."""
+    rng = np.random.default_rng(24)
+    cu_q = np.array([0, 3, 3, 10])
+    cu_k = np.array([0, 5, 9, 12])
+    q = rng.standard_normal((12, 2, 4))
+    k = rng.standard_normal((12, 1, 4))
+    v = rng.standard_normal((12, 1, 4))
+    o1, l1 = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k)
+    k2, v2 = k.copy(), v.copy()
+    k2[0:5] += 1.0
+    v2[0:5] -= 2.0
+    o2, l2 = oracle.attn_fwd_varlen(q, k2, v2, cu_q, cu_k)
+    assert np.array_equal(o1[3:10], o2[3:10]) and np.array_equal(l1[:, 3:10], l2[:, 3:10])
+    assert not np.allclose(o1[0:3], o2[0:3])
+    assert np.all(o1[10:] == 0.0) and np.all(np.isneginf(l1[:, 10:]))

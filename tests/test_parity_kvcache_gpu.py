@@ -17,7 +17,7 @@ import torch
 
 import exact_io_aware_89_b200 as fa
 import oracle
-from parity_utils import TOL_BF16, compare_lse
+from parity_utils import TOL_BF16, compare_lse, o_error
 from seeded_inputs import make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -69,7 +69,7 @@ def check_kvcache(B, Nq, Nk, n_new, Hq, Hkv, d, seqlens, causal=True, window=(-1
         f64 = lambda t: t[b:b + 1].double().numpy()
         o_ref, lse_ref = oracle.attn_fwd(f64(q), f64(kc_exp)[:, :L], f64(vc_exp)[:, :L],
                                          scale=scale, causal=causal, window=window)
-        err = float(np.abs(o[b:b + 1] - o_ref).max())
+        err = o_error(o[b:b + 1], o_ref)
         assert err <= TOL_BF16["o"], "%s batch %d: O max err %.3e" % (what, b, err)
         compare_lse(lse[b:b + 1], lse_ref, TOL_BF16["lse"], "%s batch %d" % (what, b))
 

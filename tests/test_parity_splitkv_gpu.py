@@ -17,7 +17,7 @@ import torch
 
 import exact_io_aware_89_b200 as fa
 import oracle
-from parity_utils import TOL_BF16, compare_lse
+from parity_utils import TOL_BF16, compare_lse, o_error
 from seeded_inputs import make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -47,7 +47,7 @@ def check_case(B, Nq, Nk, Hq, Hkv, d, causal, window, n_splits, seed):
                                      window=window)
     what = "splitkv B%d Nq%d Nk%d Hq%d Hkv%d d%d causal%d win%s splits%d" % (
         B, Nq, Nk, Hq, Hkv, d, causal, window, n_splits)
-    err = float(np.abs(o - o_ref).max())
+    err = o_error(o, o_ref)
     assert err <= TOL_BF16["o"], "%s: O max err %.3e" % (what, err)
     compare_lse(lse, lse_ref, TOL_BF16["lse"], what)
     return o, lse
@@ -141,4 +141,4 @@ def test_splitkv_workspace_contents_are_ignored():
     assert fa.fa_get_device_status(None) == 0
     f64 = {n: t.double().numpy() for n, t in inp.items()}
     o_ref, _ = oracle.attn_fwd(f64["q"], f64["k"], f64["v"], scale=1.0 / math.sqrt(d), causal=True)
-    assert float(np.abs(ref_o.float().cpu().numpy() - o_ref).max()) <= TOL_BF16["o"]
+    assert o_error(ref_o.float().cpu().numpy(), o_ref) <= TOL_BF16["o"]
