@@ -719,6 +719,112 @@ def run_decode(args, local):
     del flush
 
 
+# ------------------------------------------------------------ packed sequences
+
+def varlen_workloads():
+    """Packed variable-length training batches: sequence lengths drawn
+    (seeded) uniformly from a range until the token budget is filled."""
+    return [
+        dict(name="packed causal H=16 d=128, 32768 tokens, lengths uniform in [256, 4096]",
+             tokens=32768, lo=256, hi=4096, H=16, Hkv=16, d=128, causal=True, seed=6001),
+        dict(name="packed causal GQA Hq=32 Hkv=8 d=128, 65536 tokens, lengths uniform in [1024, 8192]",
+             tokens=65536, lo=1024, hi=8192, H=32, Hkv=8, d=128, causal=True, seed=6002),
+    ]
+
+
+def varlen_lengths(w):
+    import numpy as np
+    rng = np.random.default_rng(w["seed"])
+    lens, total = [], 0
+    while total < w["tokens"]:
+        n = int(rng.integers(w["lo"], w["hi"] + 1))
+        n = min(n, w["tokens"] - total)
+        lens.append(n)
+        total += n
+    return lens
+
+
+def varlen_fwd_flops(w, lens):
+    """4 d flop per visible (query, key) pair and head: the metric's count
+    applied per sequence (causal: L (L + 1) / 2 pairs)."""
+    pairs = sum(n * (n + 1) // 2 if w["causal"] else n * n for n in lens)
+    return 4.0 * w["H"] * pairs * w["d"]
+
+
+def run_varlen(args, local):
+    """One JSON line per packed workload: fa_fwd_varlen, fa_bwd_varlen and both
+    timed separately (L2 flushed before each call, median of the steps)."""
+    import numpy as np
+    import torch
+    import exact_io_aware_89_b200 as fa
+    from seeded_inputs import make_inputs
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    flush = L2Flush(dev)
+    for w in varlen_workloads():
+        lens = varlen_lengths(w)
+        T, H, Hkv, d = sum(lens), w["H"], w["Hkv"], w["d"]
+        inp = make_inputs(1, T, T, H, Hkv, d, w["seed"])
+        q, k, v, do = (inp[n][0].to(dev) for n in ("q", "k", "v", "do"))
+        del inp
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+        mx = max(lens)
+        scale = 1.0 / math.sqrt(d)
+        o = torch.empty_like(q)
+        lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(max(16, fa.fa_bwd_workspace_size(len(lens), mx, H, d)), dtype=torch.uint8,
+                         device=dev)
+        sp = torch.cuda.current_stream().cuda_stream
+        c = int(w["causal"])
+
+        def fwd():
+            st = fa.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  cu.data_ptr(), cu.data_ptr(), len(lens), mx, mx, T, T, H, Hkv, d, scale,
+                                  c, -1, -1, sp)
+            if st:
+                raise fa.FAError("fa_fwd_varlen", st)
+
+        def bwd():
+            st = fa.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu.data_ptr(),
+                                  cu.data_ptr(), len(lens), mx, mx, T, T, H, Hkv, d, scale, c, -1, -1,
+                                  ws.data_ptr(), ws.numel(), sp)
+            if st:
+                raise fa.FAError("fa_bwd_varlen", st)
+
+        def both():
+            fwd()
+            bwd()
+
+        ms = {}
+        for mode, fn in (("fwd", fwd), ("bwd", bwd), ("fwd_bwd", both)):
+            for _ in range(args.warmup):
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush()
+                ev[i][0].record()
+                fn()
+                ev[i][1].record()
+            torch.cuda.synchronize()
+            ms[mode] = statistics.median(a.elapsed_time(b) for a, b in ev)
+        if fa.fa_get_device_status(None) != 0:
+            raise RuntimeError("device status reports a timed-out wait")
+        F = varlen_fwd_flops(w, lens)
+        tf = {"fwd": F / ms["fwd"] / 1e9, "bwd": 2.5 * F / ms["bwd"] / 1e9,
+              "fwd_bwd": 3.5 * F / ms["fwd_bwd"] / 1e9}
+        line = {"varlen": w["name"], "sequences": len(lens), "tokens": T, "max_seqlen": mx,
+                "H": H, "Hkv": Hkv, "d": d, "causal": w["causal"],
+                "ms": {m: round(x, 4) for m, x in ms.items()},
+                "tflops": {m: round(x, 1) for m, x in tf.items()},
+                "pct_dense_peak": {m: round(100 * x / DENSE_PEAK_TFLOPS, 2) for m, x in tf.items()}}
+        print(json.dumps(line), flush=True)
+        del q, k, v, do, o, lse, dq, dk, dv, ws
+        torch.cuda.empty_cache()
+
+
 def run_ours(args, world, rank, local):
     import torch
     dev = torch.device("cuda", local)
@@ -802,6 +908,9 @@ def main(argv=None):
     ap.add_argument("--decode", action="store_true",
                     help="instead of the benchmark line: the KV-cache decoding workloads through "
                          "fa_fwd_splitkv, one JSON line each")
+    ap.add_argument("--varlen", action="store_true",
+                    help="instead of the benchmark line: packed variable-length workloads through "
+                         "fa_fwd_varlen / fa_bwd_varlen, one JSON line each")
     ap.add_argument("--decode-case", type=int, default=None,
                     help="with --decode: only this workload (index into the list)")
     ap.add_argument("--sweep", action="store_true",
@@ -811,10 +920,10 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     world, rank, local = dist_setup(args)
-    if args.sweep or args.decode:
+    if args.sweep or args.decode or args.varlen:
         if world > 1:
-            raise SystemExit("--sweep and --decode run on one GPU")
-        (run_sweep if args.sweep else run_decode)(args, local)
+            raise SystemExit("--sweep, --decode and --varlen run on one GPU")
+        (run_sweep if args.sweep else run_decode if args.decode else run_varlen)(args, local)
         return
     if args.impl == "reference":
         run_reference(args, world, rank)  # rank 0 alone; no process group

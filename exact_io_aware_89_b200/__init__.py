@@ -3,13 +3,14 @@
 The C ABI (include/fa.h) is the product boundary; this module only marshals
 arguments to it.  Two layers:
 
-* ``fa_fwd``, ``fa_bwd``, ``fa_fwd_varlen``, ``fa_fwd_splitkv``, ``fa_fwd_kvcache``,
+* ``fa_fwd``, ``fa_bwd``, ``fa_fwd_varlen``, ``fa_bwd_varlen``, ``fa_fwd_splitkv``, ``fa_fwd_kvcache``,
   ``fa_fwd_f32``, ``fa_bwd_f32``,
   ``fa_bwd_workspace_size``, ``fa_fwd_splitkv_workspace_size``,
   ``fa_get_device_status``, ``fa_status_string``: the C entry points under the
   same names, taking raw device pointers (ints) and sizes, returning the
   status code.
 * ``attention_forward`` / ``attention_backward`` / ``attention_forward_varlen`` /
+  ``attention_backward_varlen`` /
   ``attention_forward_splitkv`` / ``attention_forward_kvcache``:
   the same calls on torch CUDA tensors (torch only allocates the outputs and
   the workspace and supplies the current stream).
@@ -24,11 +25,11 @@ import os
 __all__ = [
     "FAError", "load_library", "library_path",
     "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
-    "fa_fwd_varlen", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
+    "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
     "fa_fwd_kvcache_workspace_size",
     "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
     "KERNEL_KINDS", "attention_forward", "attention_backward", "attention_forward_splitkv",
-    "attention_forward_kvcache", "attention_forward_varlen",
+    "attention_forward_kvcache", "attention_forward_varlen", "attention_backward_varlen",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -75,6 +76,8 @@ def load_library():
     lib.fa_fwd_splitkv_workspace_size.argtypes = [i, i, i, i, i, i, i, i, i, i]
     lib.fa_fwd_splitkv_workspace_size.restype = sz
     lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, i, i, i, vp]
+    lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i,
+                                  f, i, i, i, vp, sz, vp]
     lib.fa_fwd_kvcache_workspace_size.argtypes = [i, i, i, i, i, i, i, i, i, i, i]
     lib.fa_fwd_kvcache_workspace_size.restype = sz
     lib.fa_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, i,
@@ -84,7 +87,7 @@ def load_library():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_trace_enable.argtypes = [i]
     lib.fa_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
-    for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache", "fa_fwd_varlen",
+    for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache", "fa_fwd_varlen", "fa_bwd_varlen",
                  "fa_get_device_status",
                  "fa_trace_enable", "fa_trace_read"):
         getattr(lib, name).restype = i
@@ -126,6 +129,16 @@ def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, 
     return load_library().fa_fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q,
                                         max_seqlen_k, total_q, total_k, Hq, Hkv, d, scale, causal,
                                         win_l, win_r, stream)
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dO, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q,
+                  max_seqlen_k, total_q, total_k, Hq, Hkv, d, scale, causal, win_l, win_r,
+                  workspace, workspace_bytes, stream):
+    """Backward over packed variable-length sequences (deterministic)."""
+    return load_library().fa_bwd_varlen(q, k, v, o, lse, dO, dq, dk, dv, cu_seqlens_q, cu_seqlens_k,
+                                        B, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d,
+                                        scale, causal, win_l, win_r, workspace, workspace_bytes,
+                                        stream)
 
 
 def fa_fwd_kvcache(q, k_cache, v_cache, k_new, v_new, cache_seqlens, o, lse, B, Nq, Nk, n_new, Hq,
@@ -297,6 +310,33 @@ def attention_forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, 
                          int(max_seqlen_k), total_q, total_k, Hq, Hkv, d, scale, c, wl, wr,
                          _stream()))
     return o, lse
+
+
+def attention_backward_varlen(q, k, v, o, lse, do, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                              max_seqlen_k, scale=None, causal=False, window=(-1, -1), dq=None,
+                              dk=None, dv=None, workspace=None):
+    """dQ, dK, dV for packed sequences through fa_bwd_varlen (bf16 only), in
+    the layouts of attention_forward_varlen."""
+    import torch
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    wsb = fa_bwd_workspace_size(B, int(max_seqlen_q), Hq, d)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
+    _check("fa_bwd_varlen",
+           fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                         do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                         cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
+                         int(max_seqlen_k), total_q, total_k, Hq, Hkv, d, scale, c, wl, wr,
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         _stream()))
+    return dq, dk, dv
 
 
 def attention_forward_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache_seqlens=None,

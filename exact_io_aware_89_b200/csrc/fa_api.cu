@@ -183,7 +183,7 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
   p.total_q = total_q;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.wait_limit_ns = kWaitLimitNs;
-  auto kern = fa_fwd_kernel<C>;
+  auto kern = fa_fwd_kernel<C, true>;
   if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
   const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
   if (grid > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
@@ -195,10 +195,20 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
 }
 
 // ------------------------------------------------------------------ backward
-template <class CQ, class CKV>
+// Packed sequences of a backward call (all null / 0 when dense).
+struct Varlen {
+  const int* cu_q = nullptr;
+  const int* cu_k = nullptr;
+  int total_q = 0, total_k = 0;
+};
+
+// Dense (VL false): B batches of Nq / Nk rows.  Packed (VL true, vl set): B
+// sequences of at most Nq / Nk rows in one-batch tensors of vl.total_q /
+// vl.total_k rows.
+template <class CQ, class CKV, bool VL = false>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
-               float scale, const MaskSpec& mask, float* ws, cudaStream_t stream) {
+               float scale, const MaskSpec& mask, float* ws, cudaStream_t stream, const Varlen& vl = Varlen()) {
   static int attr_dq[kMaxDevices] = {0};
   static int attr_kv[kMaxDevices] = {0};
   constexpr int D = CQ::D;
@@ -209,9 +219,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     constexpr int RPG = 4;    // rows per lane group
     const long long blocks = (rows_pad * G / RPG + 255) / 256;
     TraceScope tr(FA_KERNEL_BWD_PREP, stream);
-    fa_bwd_prep_bf16_kernel<G, RPG><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+    fa_bwd_prep_bf16_kernel<G, RPG, VL><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, ws, B, Nq,
-        Hq, Nq_pad);
+        Hq, Nq_pad, vl.cu_q, vl.total_q);
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
   BwdParams p;
@@ -226,21 +236,31 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.n_kvtiles = (Nk + CKV::BN - 1) / CKV::BN;
   p.head_chunk = head_chunk(B * Hq, 4ll * Nk * D);                  // K and V per query head
   p.head_chunk_kv = head_chunk(B * Hkv, 4ll * Nq * D * (Hq / Hkv));  // Q and dO per key/value head
+  p.cu_q = vl.cu_q;
+  p.cu_k = vl.cu_k;
+  p.total_q = vl.total_q;
+  p.total_k = vl.total_k;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
   p.wait_limit_ns = kWaitLimitNs;
+  // tensor-map shapes: dense [B, N, H, d]; packed [1, total, H, d]
+  const bool packed = VL;
+  const int mB = packed ? 1 : B, mNq = packed ? vl.total_q : Nq, mNk = packed ? vl.total_k : Nk;
   {
     CUtensorMap tq, tk, tv, tdo, tdq;
-    if (!encode_bnhd(&tq, q, B, Nq, Hq, D, CQ::BM) || !encode_bnhd(&tk, k, B, Nk, Hkv, D, CQ::BN) ||
-        !encode_bnhd(&tv, v, B, Nk, Hkv, D, CQ::BN) || !encode_bnhd(&tdo, dO, B, Nq, Hq, D, CQ::BM) ||
-        !encode_bnhd(&tdq, dq, B, Nq, Hq, D, CQ::BM))
+    if (!encode_bnhd(&tq, q, mB, mNq, Hq, D, CQ::BM) || !encode_bnhd(&tk, k, mB, mNk, Hkv, D, CQ::BN) ||
+        !encode_bnhd(&tv, v, mB, mNk, Hkv, D, CQ::BN) || !encode_bnhd(&tdo, dO, mB, mNq, Hq, D, CQ::BM) ||
+        !encode_bnhd(&tdq, dq, mB, mNq, Hq, D, CQ::BM))
       return FA_ERR_CUDA;
     const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
     if constexpr (CQ::ONE_TILE) {
-      auto kern = fa_bwd_dq2_kernel<CQ>;
+      auto kern = fa_bwd_dq2_kernel<CQ, VL>;
       if (smem_attr_once(kern, CQ::SMEM_BYTES, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
       TraceScope tr(FA_KERNEL_BWD_DQ, stream);
       kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
     } else {
-      auto kern = fa_bwd_dq_kernel<CQ>;
+      auto kern = fa_bwd_dq_kernel<CQ, VL>;
       if (smem_attr_once(kern, CQ::SMEM_BYTES, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
       TraceScope tr(FA_KERNEL_BWD_DQ, stream);
       kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
@@ -249,11 +269,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   }
   {
     CUtensorMap tq, tk, tv, tdo, tdk, tdv;
-    if (!encode_bnhd(&tq, q, B, Nq, Hq, D, CKV::BM) || !encode_bnhd(&tk, k, B, Nk, Hkv, D, CKV::BN) ||
-        !encode_bnhd(&tv, v, B, Nk, Hkv, D, CKV::BN) || !encode_bnhd(&tdo, dO, B, Nq, Hq, D, CKV::BM) ||
-        !encode_bnhd(&tdk, dk, B, Nk, Hkv, D, CKV::BN) || !encode_bnhd(&tdv, dv, B, Nk, Hkv, D, CKV::BN))
+    if (!encode_bnhd(&tq, q, mB, mNq, Hq, D, CKV::BM) || !encode_bnhd(&tk, k, mB, mNk, Hkv, D, CKV::BN) ||
+        !encode_bnhd(&tv, v, mB, mNk, Hkv, D, CKV::BN) || !encode_bnhd(&tdo, dO, mB, mNq, Hq, D, CKV::BM) ||
+        !encode_bnhd(&tdk, dk, mB, mNk, Hkv, D, CKV::BN) || !encode_bnhd(&tdv, dv, mB, mNk, Hkv, D, CKV::BN))
       return FA_ERR_CUDA;
-    auto kern = fa_bwd_dkdv_kernel<CKV>;
+    auto kern = fa_bwd_dkdv_kernel<CKV, VL>;
     if (smem_attr_once(kern, CKV::SMEM_BYTES, attr_kv) != cudaSuccess) return FA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(static_cast<long long>(p.n_kvtiles) * B * Hkv), D / CKV::DV);
     TraceScope tr(FA_KERNEL_BWD_DKDV, stream);
@@ -622,6 +642,45 @@ int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* l
                                        total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
     default:
       return FA_ERR_UNSUPPORTED;
+  }
+}
+
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dO, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q,
+                  int total_k, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                  void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_common(q, k, v, 1, total_q, total_k, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || max_seqlen_q < 1 || max_seqlen_k < 1 || max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Hq * ((max_seqlen_q + 127) / 128) > (1ll << 31) - 1 ||
+      static_cast<long long>(B) * Hkv * ((max_seqlen_k + 63) / 64) > (1ll << 31) - 1)
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(workspace) || workspace_bytes_ < workspace_bytes(B, max_seqlen_q, Hq)) return FA_ERR_WORKSPACE;
+  const MaskSpec mask = make_mask(max_seqlen_q, max_seqlen_k, causal, win_l, win_r);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  Varlen vl;
+  vl.cu_q = cu_seqlens_q;
+  vl.cu_k = cu_seqlens_k;
+  vl.total_q = total_q;
+  vl.total_k = total_k;
+  const int Nq = max_seqlen_q, Nk = max_seqlen_k;
+  switch (d) {
+    case 64:
+      return launch_bwd<Dq64, Dkv64, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s, vl);
+    case 128:
+      return launch_bwd<Dq128, Dkv128, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s, vl);
+    default:
+      return launch_bwd<Dq256, Dkv256, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s, vl);
   }
 }
 

@@ -78,12 +78,14 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const T* __restrict__ 
 // that enough bytes are in flight to approach HBM bandwidth.  Same outputs
 // and layout as fa_bwd_prep_kernel; rows_pad must be a multiple of
 // RPG * 256 / G (it is a multiple of 256).
-template <int G, int RPG>
+template <int G, int RPG, bool VL = false>
 __global__ void __launch_bounds__(256) fa_bwd_prep_bf16_kernel(const __nv_bfloat16* __restrict__ o,
                                                                const __nv_bfloat16* __restrict__ dout,
                                                                const float* __restrict__ lse,
                                                                float* __restrict__ ws, int B, int Nq,
-                                                               int Hq, int Nq_pad) {
+                                                               int Hq, int Nq_pad,
+                                                               const int* __restrict__ cu_q = nullptr,
+                                                               int total_q = 0) {
   static_assert(G == 8 || G == 16 || G == 32, "d = 64, 128 or 256");
   constexpr int D = G * 8;
   constexpr int GROUPS = 256 / G;  // lane groups per block
@@ -93,14 +95,22 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_bf16_kernel(const __nv_bfloat
   uint4 ov[RPG], gv[RPG];
   long long row[RPG];
   bool live[RPG];
+  long long grow_[RPG];  // row of O / dO / LSE: (b, i) dense, cu_q[b] + i packed
 #pragma unroll
   for (int k = 0; k < RPG; ++k) {
     row[k] = (static_cast<long long>(blockIdx.x) * RPG + k) * GROUPS + grp;
     const int i = static_cast<int>(row[k] % Nq_pad);
     const long long bh = row[k] / Nq_pad;
     live[k] = row[k] < rows_pad && i < Nq;
+    grow_[k] = (bh / Hq) * Nq + i;
+    if (VL && live[k]) {
+      const int b = static_cast<int>(bh / Hq);
+      const int q0 = __ldg(cu_q + b);
+      grow_[k] = static_cast<long long>(q0) + i;
+      live[k] = i < __ldg(cu_q + b + 1) - q0 && grow_[k] >= 0 && grow_[k] < total_q;
+    }
     if (live[k]) {
-      const size_t base = ((static_cast<size_t>(bh / Hq) * Nq + i) * Hq + bh % Hq) * D + sub * 8;
+      const size_t base = (static_cast<size_t>(grow_[k]) * Hq + bh % Hq) * D + sub * 8;
       ov[k] = __ldg(reinterpret_cast<const uint4*>(o + base));
       gv[k] = __ldg(reinterpret_cast<const uint4*>(dout + base));
     }
@@ -121,13 +131,15 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_bf16_kernel(const __nv_bfloat
 #pragma unroll
     for (int off = G / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (sub == 0 && row[k] < rows_pad) {
-      const int i = static_cast<int>(row[k] % Nq_pad);
-      if (i >= Nq) {  // padding row: D = 0 and lse2 = +inf, so every P there is 0
+      if (!live[k]) {  // padding row: D = 0 and lse2 = +inf, so every P there is 0
         ws[row[k]] = 0.f;
         ws[rows_pad + row[k]] = INFINITY;
       } else {
         ws[row[k]] = acc;
-        const float L = lse[(row[k] / Nq_pad) * Nq + i];
+        // LSE is [B, Hq, Nq] dense, [Hq, total_q] packed
+        const long long bh = row[k] / Nq_pad;
+        const float L = VL ? lse[(bh % Hq) * static_cast<long long>(total_q) + grow_[k]]
+                                        : lse[bh * Nq + row[k] % Nq_pad];
         // a row with no visible key (LSE = -inf) has P = 0 everywhere
         ws[rows_pad + row[k]] = (L == -INFINITY) ? INFINITY : L * kLog2e;
       }
@@ -147,6 +159,16 @@ struct BwdParams {
   int n_kvtiles;      // dkdv kernel: CTAs along the key axis
   int head_chunk;     // dq kernel: heads per scheduling chunk
   int head_chunk_kv;  // dkdv kernel: key/value heads per scheduling chunk
+  // packed sequences (null when dense): sequence b is query rows [cu_q[b],
+  // cu_q[b+1]) and key rows [cu_k[b], cu_k[b+1]) of one-batch tensors; Nq / Nk
+  // are then the longest lengths, and D / lse2 stay [B, Hq, Nq_pad] (rows past
+  // a sequence's end are padding: D = 0, lse2 = +inf)
+  const int* cu_q;
+  const int* cu_k;
+  int total_q, total_k;
+  __nv_bfloat16* dq;  // outputs, for the plain stores of a packed sequence's last tile
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
   unsigned long long wait_limit_ns;
 };
 
@@ -183,7 +205,7 @@ struct DqCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <class C>
+template <class C, bool VL = false>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -213,8 +235,11 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int g = p.n_qgroups - 1 - order.rank;
   const int b = bh / p.Hq, h = bh % p.Hq, hk = h / p.group;
   const int r0 = g * NQT * BM;
-  const int r_last = min(p.Nq - 1, r0 + NQT * BM - 1);
-  const int key_lo = p.mask.lo(r0), key_hi = p.mask.hi(r_last);
+  const SeqView sq(p.mask, VL ? p.cu_q : nullptr, p.cu_k, b);
+  const int nq = sq.mask.Nq;
+  if (VL && r0 >= nq) return;  // this packed sequence has no query group g
+  const int r_last = min(nq - 1, r0 + NQT * BM - 1);
+  const int key_lo = sq.mask.lo(r0), key_hi = sq.mask.hi(r_last);
   const int j_begin = key_lo / BN;
   const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
 
@@ -247,8 +272,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       mbar_expect_tx(q_full, 2 * NQT * C::QTILE);
       for (int t = 0; t < NQT; ++t)
         for (int c = 0; c < C::NCHUNK; ++c) {
-          tma_load_4d(sQ + t * C::QTILE + c * C::QCHUNK, &tm_q, q_full, c * 64, h, r0 + t * BM, b);
-          tma_load_4d(sdO + t * C::QTILE + c * C::QCHUNK, &tm_do, q_full, c * 64, h, r0 + t * BM, b);
+          tma_load_4d(sQ + t * C::QTILE + c * C::QCHUNK, &tm_q, q_full, c * 64, h, sq.q_off + r0 + t * BM, sq.tb);
+          tma_load_4d(sdO + t * C::QTILE + c * C::QCHUNK, &tm_do, q_full, c * 64, h, sq.q_off + r0 + t * BM, sq.tb);
         }
       int n_issued = 0;
       for (int it = 0; it < n_kv; ++it) {
@@ -258,8 +283,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
           break;
         mbar_expect_tx(&kv_full[s], 2 * C::KTILE);
         for (int c = 0; c < C::NCHUNK; ++c) {
-          tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, &kv_full[s], c * 64, hk, krow, b);
-          tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &kv_full[s], c * 64, hk, krow, b);
+          tma_load_4d(sK + s * C::KTILE + c * C::KCHUNK, &tm_k, &kv_full[s], c * 64, hk, sq.k_off + krow, sq.tb);
+          tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &kv_full[s], c * 64, hk, sq.k_off + krow, sq.tb);
         }
         ++n_issued;
       }
@@ -343,7 +368,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const int t = warp / 4;
     const int r = threadIdx.x % BM;
     const int row = r0 + t * BM + r;
-    const int lo = p.mask.lo(row), hi = p.mask.hi(row);
+    const int lo = sq.mask.lo(row), hi = sq.mask.hi(row);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     const size_t srow = (static_cast<size_t>(b) * p.Hq + h) * p.Nq_pad + row;  // row < Nq_pad
     const float lse2 = p.lse2[srow];
@@ -422,11 +447,17 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       fence_proxy_async_smem();
     }
     named_bar_sync(1 + t, BM);
-    if (r == 0 && *abort_flag == 0 && r0 + t * BM < p.Nq) {
-      for (int c = 0; c < C::NCHUNK; ++c)
-        tma_store_4d(&tm_dq, stage + c * C::QCHUNK, c * 64, h, r0 + t * BM, b);
-      tma_store_commit();
-      tma_store_wait_read();
+    const int t_row0 = r0 + t * BM;
+    if (!VL || t_row0 + BM <= nq) {
+      if (r == 0 && *abort_flag == 0 && t_row0 < nq) {
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_store_4d(&tm_dq, stage + c * C::QCHUNK, c * 64, h, sq.q_off + t_row0, sq.tb);
+        tma_store_commit();
+        tma_store_wait_read();
+      }
+    } else if (*abort_flag == 0) {  // last tile of a packed sequence
+      store_rows_sw128(stage, C::QCHUNK, nq - t_row0, D, p.dq, sq.q_off + t_row0, p.total_q, p.Hq, h, D, 0, r,
+                       BM);
     }
   }
 
@@ -479,7 +510,7 @@ struct Dq2Cfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <class C>
+template <class C, bool VL = false>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
     fa_bwd_dq2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -512,8 +543,11 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int g = p.n_qgroups - 1 - order.rank;  // query tile, latest first
   const int b = bh / p.Hq, h = bh % p.Hq, hk = h / p.group;
   const int r0 = g * BM;
-  const int r_last = min(p.Nq - 1, r0 + BM - 1);
-  const int key_lo = p.mask.lo(r0), key_hi = p.mask.hi(r_last);
+  const SeqView sq(p.mask, VL ? p.cu_q : nullptr, p.cu_k, b);
+  const int nq = sq.mask.Nq;
+  if (VL && r0 >= nq) return;  // this packed sequence has no query tile g
+  const int r_last = min(nq - 1, r0 + BM - 1);
+  const int key_lo = sq.mask.lo(r0), key_hi = sq.mask.hi(r_last);
   const int j_begin = key_lo / BN;
   const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
 
@@ -522,13 +556,13 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const int sk = it % KS, krow = (j_begin + it) * BN;
     mbar_expect_tx(&k_full[sk], C::KTILE);
     for (int c = 0; c < C::NCHUNK; ++c)
-      tma_load_4d(sK + sk * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[sk], c * 64, hk, krow, b);
+      tma_load_4d(sK + sk * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[sk], c * 64, hk, sq.k_off + krow, sq.tb);
   };
   auto load_v = [&](int it) {
     const int sv = it % VS, krow = (j_begin + it) * BN;
     mbar_expect_tx(&v_full[sv], C::KTILE);
     for (int c = 0; c < C::NCHUNK; ++c)
-      tma_load_4d(sV + sv * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[sv], c * 64, hk, krow, b);
+      tma_load_4d(sV + sv * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[sv], c * 64, hk, sq.k_off + krow, sq.tb);
   };
   // The TMA thread sets up the barriers and issues Q, dO and the first ring
   // stages (nothing to wait for yet) before the block-wide sync.
@@ -554,8 +588,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     if (n_kv > 0) {
       mbar_expect_tx(q_full, 2 * C::QTILE);
       for (int c = 0; c < C::NCHUNK; ++c) {
-        tma_load_4d(sQ + c * C::QCHUNK, &tm_q, q_full, c * 64, h, r0, b);
-        tma_load_4d(sdO + c * C::QCHUNK, &tm_do, q_full, c * 64, h, r0, b);
+        tma_load_4d(sQ + c * C::QCHUNK, &tm_q, q_full, c * 64, h, sq.q_off + r0, sq.tb);
+        tma_load_4d(sdO + c * C::QCHUNK, &tm_do, q_full, c * 64, h, sq.q_off + r0, sq.tb);
       }
       for (int it = 0; it < n_pre_k; ++it) load_k(it);
       for (int it = 0; it < n_pre_v; ++it) load_v(it);
@@ -659,7 +693,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const int wg = warp / 4;          // key columns [64 wg, 64 wg + 64) of every tile
     const int r = threadIdx.x % BM;   // row == TMEM lane
     const int row = r0 + r;
-    const int lo = p.mask.lo(row), hi = p.mask.hi(row);
+    const int lo = sq.mask.lo(row), hi = sq.mask.hi(row);
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     const size_t srow = (static_cast<size_t>(b) * p.Hq + h) * p.Nq_pad + row;  // row < Nq_pad
     const float lse2 = p.lse2[srow];
@@ -741,10 +775,15 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       fence_proxy_async_smem();
     }
     named_bar_sync(1, 256);
-    if (threadIdx.x == 0 && *abort_flag == 0 && r0 < p.Nq) {
-      for (int c = 0; c < C::NCHUNK; ++c) tma_store_4d(&tm_dq, sQ + c * C::QCHUNK, c * 64, h, r0, b);
-      tma_store_commit();
-      tma_store_wait_read();
+    if (!VL || r0 + BM <= nq) {
+      if (threadIdx.x == 0 && *abort_flag == 0 && r0 < nq) {
+        for (int c = 0; c < C::NCHUNK; ++c)
+          tma_store_4d(&tm_dq, sQ + c * C::QCHUNK, c * 64, h, sq.q_off + r0, sq.tb);
+        tma_store_commit();
+        tma_store_wait_read();
+      }
+    } else if (*abort_flag == 0) {  // last tile of a packed sequence
+      store_rows_sw128(sQ, C::QCHUNK, nq - r0, D, p.dq, sq.q_off + r0, p.total_q, p.Hq, h, D, 0, threadIdx.x, 256);
     }
   }
 
@@ -793,7 +832,7 @@ struct DkvCfg {
   static_assert(STAGE % 1024 == 0, "stages stay 1 KiB aligned");
 };
 
-template <class C>
+template <class C, bool VL = false>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -825,13 +864,16 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
   const int dslice = blockIdx.y;  // which DV-wide slice of d
   const int k0 = j * BN;
-  const int k1 = min(p.Nk - 1, k0 + BN - 1);
+  const SeqView sq(p.mask, VL ? p.cu_q : nullptr, p.cu_k, b);
+  const int nq = sq.mask.Nq, nk = sq.mask.Nk;
+  if (VL && k0 >= nk) return;  // this packed sequence has no key tile j
+  const int k1 = min(nk - 1, k0 + BN - 1);
   // queries that see some key of this tile: i in [q_lo(k0), q_hi(k1)]
-  const int delta = p.mask.delta();
-  int q_lo = (p.mask.wr < 0) ? 0 : k0 - delta - p.mask.wr;
-  int q_hi = (p.mask.wl < 0) ? p.Nq - 1 : k1 - delta + p.mask.wl;
+  const int delta = sq.mask.delta();
+  int q_lo = (sq.mask.wr < 0) ? 0 : k0 - delta - sq.mask.wr;
+  int q_hi = (sq.mask.wl < 0) ? nq - 1 : k1 - delta + sq.mask.wl;
   q_lo = max(q_lo, 0);
-  q_hi = min(q_hi, p.Nq - 1);
+  q_hi = min(q_hi, nq - 1);
   const int i_begin = q_lo / BM;
   const int n_qt = (q_hi >= q_lo) ? (q_hi / BM - i_begin + 1) : 0;
   const int n_steps = n_qt * p.group;  // (query head in group) x (query tile)
@@ -845,8 +887,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const uint32_t st = sSt + s * C::STAGE;
     mbar_expect_tx(&q_full[s], C::STAGE + C::SSTAGE);
     for (int c = 0; c < C::NCHUNK; ++c) {
-      tma_load_4d(st + c * C::QCHUNK, &tm_q, &q_full[s], c * 64, hq, q0, b);
-      tma_load_4d(st + C::QTILE + c * C::QCHUNK, &tm_do, &q_full[s], c * 64, hq, q0, b);
+      tma_load_4d(st + c * C::QCHUNK, &tm_q, &q_full[s], c * 64, hq, sq.q_off + q0, sq.tb);
+      tma_load_4d(st + C::QTILE + c * C::QCHUNK, &tm_do, &q_full[s], c * 64, hq, sq.q_off + q0, sq.tb);
     }
     const size_t srow = (static_cast<size_t>(b) * p.Hq + hq) * p.Nq_pad + q0;
     const uint32_t stat = sbase + C::OFF_STAT + s * C::SSTAGE;
@@ -874,8 +916,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     if (n_steps > 0) {
       mbar_expect_tx(kv_full, 2 * C::KTILE);
       for (int c = 0; c < C::NCHUNK; ++c) {
-        tma_load_4d(sK + c * C::KCHUNK, &tm_k, kv_full, c * 64, hk, k0, b);
-        tma_load_4d(sV + c * C::KCHUNK, &tm_v, kv_full, c * 64, hk, k0, b);
+        tma_load_4d(sK + c * C::KCHUNK, &tm_k, kv_full, c * 64, hk, sq.k_off + k0, sq.tb);
+        tma_load_4d(sV + c * C::KCHUNK, &tm_v, kv_full, c * 64, hk, sq.k_off + k0, sq.tb);
       }
       for (int it = 0; it < n_pre; ++it) load_step(it);
     }
@@ -973,8 +1015,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const int r = threadIdx.x % 128;   // TMEM lane == key within the tile
     const int key = k0 + r;
     // queries that see this key: [kq_lo, kq_hi]
-    const int kq_lo = (p.mask.wr < 0) ? -0x3fffffff : key - delta - p.mask.wr;
-    const int kq_hi = (p.mask.wl < 0) ? 0x3fffffff : key - delta + p.mask.wl;
+    const int kq_lo = (sq.mask.wr < 0) ? -0x3fffffff : key - delta - sq.mask.wr;
+    const int kq_hi = (sq.mask.wl < 0) ? 0x3fffffff : key - delta + sq.mask.wl;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     const float sl2 = p.scale_log2;
     bool ok = true;
@@ -1073,14 +1115,21 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       fence_proxy_async_smem();
     }
     named_bar_sync(1, 256);
-    if (threadIdx.x == 0 && *abort_flag == 0) {
-      for (int c = 0; c < DV / 64; ++c) {
-        const int x = (dslice * (DV / 64) + c) * 64;
-        tma_store_4d(&tm_dk, sK + c * C::KCHUNK, x, hk, k0, b);
-        tma_store_4d(&tm_dv, sV + c * C::KCHUNK, x, hk, k0, b);
+    if (!VL || k0 + BN <= nk) {
+      if (threadIdx.x == 0 && *abort_flag == 0) {
+        for (int c = 0; c < DV / 64; ++c) {
+          const int x = (dslice * (DV / 64) + c) * 64;
+          tma_store_4d(&tm_dk, sK + c * C::KCHUNK, x, hk, sq.k_off + k0, sq.tb);
+          tma_store_4d(&tm_dv, sV + c * C::KCHUNK, x, hk, sq.k_off + k0, sq.tb);
+        }
+        tma_store_commit();
+        tma_store_wait_read();
       }
-      tma_store_commit();
-      tma_store_wait_read();
+    } else if (*abort_flag == 0) {  // last key tile of a packed sequence
+      store_rows_sw128(sK, C::KCHUNK, nk - k0, DV, p.dk, sq.k_off + k0, p.total_k, p.Hkv, hk, D, dslice * DV,
+                       threadIdx.x, 256);
+      store_rows_sw128(sV, C::KCHUNK, nk - k0, DV, p.dv, sq.k_off + k0, p.total_k, p.Hkv, hk, D, dslice * DV,
+                       threadIdx.x, 256);
     }
   }
 

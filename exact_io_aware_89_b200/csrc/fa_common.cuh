@@ -106,4 +106,50 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// One sequence of a call: dense (cu_q null) -- batch b of the tensors, the
+// call's mask -- or packed -- rows [cu_q[b], cu_q[b+1]) and [cu_k[b],
+// cu_k[b+1]) of one-batch tensors (TMA batch coordinate 0), the mask taken
+// with this sequence's own lengths (causal bottom-right per sequence).
+struct SeqView {
+  int q_off = 0, k_off = 0, tb;
+  MaskSpec mask;
+  __device__ __forceinline__ SeqView(const MaskSpec& m, const int* cu_q, const int* cu_k, int b)
+      : tb(b), mask(m) {
+    if (cu_q != nullptr) {
+      q_off = __ldg(cu_q + b);
+      k_off = __ldg(cu_k + b);
+      mask.Nq = __ldg(cu_q + b + 1) - q_off;
+      mask.Nk = __ldg(cu_k + b + 1) - k_off;
+      tb = 0;
+    }
+  }
+};
+
+// Plain 16-byte stores of rows [0, n_rows) of a tile staged in shared memory
+// with the 128-byte swizzle (64-column chunks `chunk_bytes` apart, ncols a
+// multiple of 64) to rows row0 + r of a [rows, H, d] bf16 tensor, head h,
+// columns [col0, col0 + ncols).  Rows outside [0, total) are skipped.  Used
+// for the last tile of a packed sequence, whose following rows belong to the
+// next sequence (a TMA store would write them).
+__device__ __forceinline__ void store_rows_sw128(uint32_t stage, int chunk_bytes, int n_rows, int ncols,
+                                                 __nv_bfloat16* dst, int row0, int total, int H, int h,
+                                                 int d, int col0, int tid, int nthreads) {
+  const int upr = ncols / 8;
+  for (int x = tid; x < n_rows * upr; x += nthreads) {
+    const int rr = x / upr, u = x % upr;
+    const int g = row0 + rr;
+    if (g < 0 || g >= total) continue;
+    const uint4 v = ld_shared_v4(stage + (u / 8) * chunk_bytes + sw128_offset(rr, u % 8));
+    *reinterpret_cast<uint4*>(dst + (static_cast<size_t>(g) * H + h) * d + col0 + u * 8) = v;
+  }
+}
+
 }  // namespace fa

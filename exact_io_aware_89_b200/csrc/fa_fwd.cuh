@@ -161,7 +161,9 @@ __device__ __forceinline__ void fwd_exp_cols(const float* sc, uint64_t scale2, u
   }
 }
 
-template <class C>
+// VL: packed variable-length sequences (FwdParams::cu_q / cu_k); the dense
+// instantiation compiles without any of that code.
+template <class C, bool VL = false>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   // q_off / k_off of one-batch tensors (tb = 0), its own lengths and masks
   int b = bh / p.Hq, q_off = 0, k_off = 0;
   MaskSpec mask = p.mask;
-  if (p.cu_q != nullptr) {
+  if constexpr (VL) {
     q_off = __ldg(p.cu_q + b);
     k_off = __ldg(p.cu_k + b);
     mask.Nq = __ldg(p.cu_q + b + 1) - q_off;
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     if (r0 >= mask.Nq) return;  // this sequence has no query group g
   }
   const int nq = mask.Nq;
-  const int tb = p.cu_q != nullptr ? 0 : b;
+  const int tb = VL ? 0 : b;
   const int r_last = min(nq - 1, r0 + NQT * BM - 1);
   const int key_lo = mask.lo(r0), key_hi = mask.hi(r_last);
   const int j_begin = key_lo / BN;
@@ -573,7 +575,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     named_bar_sync(1 + t, BM);
     const bool aborted = *abort_flag != 0;
     const int t_row0 = r0 + t * BM;
-    if (p.cu_q == nullptr || t_row0 + BM <= nq) {
+    if (!VL || t_row0 + BM <= nq) {
       // whole tile (or dense, where TMA clips the tensor's last tile itself)
       if (r == 0 && !aborted && t_row0 < nq) {
         for (int c = 0; c < C::NCHUNK; ++c)
@@ -584,24 +586,12 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     } else if (!aborted) {
       // last tile of a packed sequence: rows past its end belong to the next
       // sequence, so only the valid rows are stored, 16 bytes at a time
-      constexpr int UPR = D / 8;
-      const int n_rows = nq - t_row0;
-      for (int x = r; x < n_rows * UPR; x += BM) {
-        const int rr = x / UPR, u = x % UPR;
-        const int gq = q_off + t_row0 + rr;
-        if (gq < 0 || gq >= p.total_q) continue;  // offsets outside the tensor: never written
-        uint32_t w0, w1, w2, w3;
-        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
-                     : "r"(sQt + (u / 8) * C::QCHUNK + sw128_offset(rr, u % 8)));
-        *reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(gq) * p.Hq + h) * D + u * 8) =
-            make_uint4(w0, w1, w2, w3);
-      }
+      store_rows_sw128(sQt, C::QCHUNK, nq - t_row0, D, p.o, q_off + t_row0, p.total_q, p.Hq, h, D, 0, r, BM);
     }
-    if (!aborted && row < nq && (p.cu_q == nullptr || (q_off + row >= 0 && q_off + row < p.total_q))) {
+    if (!aborted && row < nq && (!VL || (q_off + row >= 0 && q_off + row < p.total_q))) {
       const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
-      const size_t lse_row = p.cu_q != nullptr ? static_cast<size_t>(h) * p.total_q + q_off + row
-                                                : (static_cast<size_t>(b) * p.Hq + h) * p.Nq + row;
+      const size_t lse_row = VL ? static_cast<size_t>(h) * p.total_q + q_off + row
+                                : (static_cast<size_t>(b) * p.Hq + h) * p.Nq + row;
       p.lse[lse_row] = (l > 0.f) ? (mb + log2f(l)) * kLn2 : -INFINITY;
     }
   } else {

@@ -212,6 +212,23 @@ int fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_ne
                    void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Backward pass over packed variable-length sequences: the gradients of
+ * fa_fwd_varlen, in its layouts (dq like q [total_q, Hq, d], dk / dv like k
+ * [total_k, Hkv, d]; o, lse and dO as fa_fwd_varlen wrote / received them),
+ * deterministic, with fa_bwd's arguments otherwise.  The workspace holds the
+ * row statistics per sequence padded to max_seqlen_q: at least
+ * fa_bwd_workspace_size(B, max_seqlen_q, Hq, d) bytes.  Rows of dq, dk and dv
+ * not covered by any sequence are left untouched.  The caller guarantees the
+ * offsets as for fa_fwd_varlen; the kernels never write outside
+ * [0, total) rows whatever they hold.
+ */
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dO, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q,
+                  int total_k, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                  void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fp32 variants for small problems (fp32 in, fp32 out, fp32 arithmetic on the
  * CUDA cores).  Same arguments and semantics as fa_fwd / fa_bwd; d <= 256 and
  * d a multiple of 32.

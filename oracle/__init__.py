@@ -152,6 +152,22 @@ def attn_fwd_varlen(q, k, v, cu_q, cu_k, scale=None, causal=False, window=(-1, -
     return o, lse
 
 
+def attn_bwd_varlen(q, k, v, dout, cu_q, cu_k, scale=None, causal=False, window=(-1, -1),
+                    nthreads=None):
+    """Gradients for packed sequences (layouts of attn_fwd_varlen): each
+    sequence's own attn_bwd; rows no sequence covers get zero."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_k[b]), int(cu_k[b + 1])
+        if q1 <= q0 or k1 <= k0:
+            continue
+        g = attn_bwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], dout[None, q0:q1],
+                     scale=scale, causal=causal, window=window, nthreads=nthreads)
+        dq[q0:q1], dk[k0:k1], dv[k0:k1] = g[0][0], g[1][0], g[2][0]
+    return dq, dk, dv
+
+
 def merge_partials(o_parts, lse_parts):
     """Merge attention results computed over disjoint key subsets.
 

@@ -26,7 +26,8 @@ def test_header_declares_the_expected_entry_points():
     assert declared_functions() == sorted([
         "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
         "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
-        "fa_fwd_kvcache_workspace_size", "fa_fwd_varlen", "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
+        "fa_fwd_kvcache_workspace_size", "fa_fwd_varlen", "fa_bwd_varlen",
+        "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
 
 
 def test_kernel_kinds_match_the_header():
@@ -220,3 +221,29 @@ def test_varlen_rejects_invalid_arguments(kw):
 
 def test_varlen_rejects_unsupported_head_dim():
     assert _varlen(d=96) == UNSUPPORTED
+
+
+def _bwd_varlen(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dO=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, cq=FAKE,
+             ck=FAKE, B=3, mq=100, mk=120, tq=200, tk=250, Hq=4, Hkv=2, d=128, scale=0.125, causal=1,
+             win_l=-1, win_r=-1, ws=FAKE, wsb=1 << 20, stream=None)
+    a.update(kw)
+    return fa.fa_bwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dO"], a["dq"], a["dk"],
+                            a["dv"], a["cq"], a["ck"], a["B"], a["mq"], a["mk"], a["tq"], a["tk"],
+                            a["Hq"], a["Hkv"], a["d"], a["scale"], a["causal"], a["win_l"],
+                            a["win_r"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw", [
+    dict(dO=0), dict(dq=MISALIGNED), dict(dk=0), dict(dv=0), dict(cq=0), dict(ck=FAKE + 1),
+    dict(B=0), dict(mq=0), dict(mk=251), dict(Hq=3), dict(scale=0.0),
+])
+def test_bwd_varlen_rejects_invalid_arguments(kw):
+    assert _bwd_varlen(**kw) == INVALID
+
+
+def test_bwd_varlen_workspace_and_head_dim():
+    need = fa.fa_bwd_workspace_size(3, 100, 4, 128)   # per sequence, padded to the longest
+    assert _bwd_varlen(wsb=need - 4) == WORKSPACE
+    assert _bwd_varlen(ws=0) == WORKSPACE
+    assert _bwd_varlen(d=96) == UNSUPPORTED

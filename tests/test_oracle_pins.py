@@ -403,3 +403,19 @@ def test_varlen_sequences_do_not_see_each_other():
     assert np.array_equal(o1[3:10], o2[3:10]) and np.array_equal(l1[:, 3:10], l2[:, 3:10])
     assert not np.allclose(o1[0:3], o2[0:3])
     assert np.all(o1[10:] == 0.0) and np.all(np.isneginf(l1[:, 10:]))
+
+
+def test_varlen_gradients_of_equal_lengths_are_the_batched_gradients():
+    rng = np.random.default_rng(25)
+    B, N, Hq, Hkv, d = 2, 7, 2, 1, 4
+    q = rng.standard_normal((B, N, Hq, d))
+    k = rng.standard_normal((B, N, Hkv, d))
+    v = rng.standard_normal((B, N, Hkv, d))
+    do = rng.standard_normal((B, N, Hq, d))
+    cu = np.arange(B + 1) * N
+    g = oracle.attn_bwd_varlen(q.reshape(B * N, Hq, d), k.reshape(B * N, Hkv, d),
+                               v.reshape(B * N, Hkv, d), do.reshape(B * N, Hq, d), cu, cu,
+                               causal=True, window=(3, -1))
+    ref = oracle.attn_bwd(q, k, v, do, causal=True, window=(3, -1))
+    for a, r in zip(g, ref):
+        assert np.abs(a - r.reshape(a.shape)).max() < 1e-14
