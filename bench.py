@@ -52,13 +52,13 @@ WORKLOADS = {
 # only while the kernel sources hash to the ones that were profiled (a changed
 # kernel reports null until it is captured again).
 NCU_TRAFFIC = {
-    ("train", "bwd_dkdv"): dict(bytes=72.78e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
-    ("mid", "bwd_dkdv"): dict(bytes=377.91e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
-    ("mid", "bwd_dq"): dict(bytes=325.89e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
-    ("mid", "fwd"): dict(bytes=250.95e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
-    ("decode0", "decode"): dict(bytes=1078.09e6, profile="profiles/decode_B8Hq32Hkv8Nq1Nk32768d128.md"),
+    ("train", "bwd_dkdv"): dict(bytes=75.92e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
+    ("mid", "bwd_dkdv"): dict(bytes=377.51e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
+    ("mid", "bwd_dq"): dict(bytes=324.89e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
+    ("mid", "fwd"): dict(bytes=250.18e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
+    ("decode0", "decode"): dict(bytes=1078.37e6, profile="profiles/decode_B8Hq32Hkv8Nq1Nk32768d128.md"),
 }
-NCU_SOURCES_SHA256 = "ae64b5eee6d39decc6046491fcc8746f3eb2753cb7e38359a75c5e36e87b7c11"
+NCU_SOURCES_SHA256 = "4864a9c974e614ab6418e92101430d8e43e5a0312cf6f65cf98cc6af68b8c8b4"
 
 
 def sources_sha256():
