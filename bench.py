@@ -223,10 +223,11 @@ def barrier(world):
 
 # ------------------------------------------------------------ GPU arm
 
-def make_device_inputs(w, rank, dev):
+def make_device_inputs(w, rank, dev, dtype="bf16"):
     import torch
     from seeded_inputs import make_inputs
-    inp = make_inputs(w["B"], w["N"], w["N"], w["H"], w["Hkv"], w["d"], w["seed"] + 7919 * rank)
+    inp = make_inputs(w["B"], w["N"], w["N"], w["H"], w["Hkv"], w["d"], w["seed"] + 7919 * rank,
+                      dtype=dtype)
     return {n: t.to(dev) for n, t in inp.items()}, inp
 
 
@@ -484,14 +485,15 @@ def visible_pairs(w):
     return sum(max(0, h - l + 1) for h, l in zip(hi, lo))
 
 
-def time_modes(w, steps, warmup, dev):
+def time_modes(w, steps, warmup, dev, dtype="bf16"):
     """Median ms of fa_fwd alone, fa_bwd alone and fa_fwd + fa_bwd (L2 flushed
     before every timed call, CUDA events on the launching stream)."""
     import torch
     import exact_io_aware_89_b200 as fa
-    x, _ = make_device_inputs(w, 0, dev)
+    x, _ = make_device_inputs(w, 0, dev, dtype)
     q, k, v, do = x["q"], x["k"], x["v"], x["do"]
     B, N, H, Hkv, d = w["B"], w["N"], w["H"], w["Hkv"], w["d"]
+    fa_fwd, fa_bwd = (fa.fa_fwd_f16, fa.fa_bwd_f16) if dtype == "fp16" else (fa.fa_fwd, fa.fa_bwd)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -502,13 +504,13 @@ def time_modes(w, steps, warmup, dev):
     c, (wl, wr) = int(w["causal"]), w["window"]
 
     def fwd():
-        st = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+        st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                        B, N, N, H, Hkv, d, scale, c, wl, wr, sp)
         if st:
             raise fa.FAError("fa_fwd", st)
 
     def bwd():
-        st = fa.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+        st = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                        do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, N, N, H, Hkv,
                        d, scale, c, wl, wr, ws.data_ptr(), ws.numel(), sp)
         if st:
@@ -547,9 +549,11 @@ def run_sweep(args, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     for w in sweep_workloads():
-        t = time_modes(w, args.steps, args.warmup, dev)
+        if args.sweep_filter and args.sweep_filter not in w["name"]:
+            continue
+        t = time_modes(w, args.steps, args.warmup, dev, args.dtype)
         F = fwd_flops(w)
-        line = {"sweep": w["name"], "B": w["B"], "H": w["H"], "Hkv": w["Hkv"], "N": w["N"], "d": w["d"],
+        line = {"sweep": w["name"], "dtype": args.dtype, "B": w["B"], "H": w["H"], "Hkv": w["Hkv"], "N": w["N"], "d": w["d"],
                 "causal": w["causal"], "window": list(w["window"]),
                 "ms": {m: round(v, 4) for m, v in t.items()},
                 "tflops": {"fwd": round(F / t["fwd"] / 1e9, 1), "bwd": round(2.5 * F / t["bwd"] / 1e9, 1),
@@ -913,6 +917,10 @@ def main(argv=None):
                          "fa_fwd_varlen / fa_bwd_varlen, one JSON line each")
     ap.add_argument("--decode-case", type=int, default=None,
                     help="with --decode: only this workload (index into the list)")
+    ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16",
+                    help="with --sweep: the element type of the inputs (bf16 or fp16 entry points)")
+    ap.add_argument("--sweep-filter", default=None,
+                    help="with --sweep: only workloads whose name contains this text")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the benchmark line: the sequence-length sweep and the GQA/window "
                          "and d=256 workloads, fwd / bwd / fwd+bwd timed separately, one JSON line each")

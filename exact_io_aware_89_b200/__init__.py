@@ -4,7 +4,7 @@ The C ABI (include/fa.h) is the product boundary; this module only marshals
 arguments to it.  Two layers:
 
 * ``fa_fwd``, ``fa_bwd``, ``fa_fwd_varlen``, ``fa_bwd_varlen``, ``fa_fwd_splitkv``, ``fa_fwd_kvcache``,
-  ``fa_fwd_f32``, ``fa_bwd_f32``,
+  their fp16 twins ``fa_*_f16``, ``fa_fwd_f32``, ``fa_bwd_f32``,
   ``fa_bwd_workspace_size``, ``fa_fwd_splitkv_workspace_size``,
   ``fa_get_device_status``, ``fa_status_string``: the C entry points under the
   same names, taking raw device pointers (ints) and sizes, returning the
@@ -13,7 +13,8 @@ arguments to it.  Two layers:
   ``attention_backward_varlen`` /
   ``attention_forward_splitkv`` / ``attention_forward_kvcache``:
   the same calls on torch CUDA tensors (torch only allocates the outputs and
-  the workspace and supplies the current stream).
+  the workspace and supplies the current stream); bf16 or fp16 tensors pick
+  the bf16 or fp16 entry point.
 
 There is no fallback: if libfa.so cannot be loaded or built, importing the
 tensor API raises, and every computation runs in the library's CUDA kernels.
@@ -26,7 +27,8 @@ __all__ = [
     "FAError", "load_library", "library_path",
     "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
     "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
-    "fa_fwd_kvcache_workspace_size",
+    "fa_fwd_kvcache_workspace_size", "fa_fwd_f16", "fa_bwd_f16", "fa_fwd_varlen_f16",
+    "fa_bwd_varlen_f16", "fa_fwd_splitkv_f16", "fa_fwd_kvcache_f16",
     "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
     "KERNEL_KINDS", "attention_forward", "attention_backward", "attention_forward_splitkv",
     "attention_forward_kvcache", "attention_forward_varlen", "attention_backward_varlen",
@@ -87,6 +89,10 @@ def load_library():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_trace_enable.argtypes = [i]
     lib.fa_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+    for base in ("fa_fwd", "fa_bwd", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_splitkv",
+                 "fa_fwd_kvcache"):
+        getattr(lib, base + "_f16").argtypes = getattr(lib, base).argtypes
+        getattr(lib, base + "_f16").restype = i
     for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache", "fa_fwd_varlen", "fa_bwd_varlen",
                  "fa_get_device_status",
                  "fa_trace_enable", "fa_trace_read"):
@@ -172,6 +178,22 @@ def fa_bwd_f32(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale, ca
                                      stream)
 
 
+def _f16_twin(name):
+    def call(*args):
+        return getattr(load_library(), name)(*args)
+    call.__name__ = name
+    call.__doc__ = "fp16 twin of %s (same arguments, fp16 tensors)." % name[:-4]
+    return call
+
+
+fa_fwd_f16 = _f16_twin("fa_fwd_f16")
+fa_bwd_f16 = _f16_twin("fa_bwd_f16")
+fa_fwd_varlen_f16 = _f16_twin("fa_fwd_varlen_f16")
+fa_bwd_varlen_f16 = _f16_twin("fa_bwd_varlen_f16")
+fa_fwd_splitkv_f16 = _f16_twin("fa_fwd_splitkv_f16")
+fa_fwd_kvcache_f16 = _f16_twin("fa_fwd_kvcache_f16")
+
+
 def fa_bwd_workspace_size(B, Nq, Hq, d):
     return load_library().fa_bwd_workspace_size(B, Nq, Hq, d)
 
@@ -217,8 +239,8 @@ def _dims(q, k, v):
     for t in (q, k, v):
         if not t.is_cuda or not t.is_contiguous():
             raise ValueError("tensors must be contiguous CUDA tensors")
-        if t.dtype not in (torch.bfloat16, torch.float32) or t.dtype != q.dtype:
-            raise ValueError("tensors must all be bf16 (or all fp32)")
+        if t.dtype not in (torch.bfloat16, torch.float16, torch.float32) or t.dtype != q.dtype:
+            raise ValueError("tensors must all be bf16, all fp16 or all fp32")
     return B, Nq, k.shape[1], Hq, k.shape[2], d
 
 
@@ -245,7 +267,7 @@ def attention_forward(q, k, v, scale=None, causal=False, window=(-1, -1), out=No
     c, wl, wr = _window(causal, window)
     o = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
-    fn = fa_fwd if q.dtype == torch.bfloat16 else fa_fwd_f32
+    fn = {torch.bfloat16: fa_fwd, torch.float16: fa_fwd_f16}.get(q.dtype, fa_fwd_f32)
     _check(fn.__name__, fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                            B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, _stream()))
     return o, lse
@@ -263,8 +285,9 @@ def attention_forward_splitkv(q, k, v, scale=None, causal=False, window=(-1, -1)
     """
     import torch
     B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
-    if q.dtype != torch.bfloat16:
-        raise ValueError("fa_fwd_splitkv takes bf16 tensors")
+    if q.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("fa_fwd_splitkv takes bf16 or fp16 tensors")
+    fn = fa_fwd_splitkv if q.dtype == torch.bfloat16 else fa_fwd_splitkv_f16
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     c, wl, wr = _window(causal, window)
     o = torch.empty_like(q) if out is None else out
@@ -272,8 +295,8 @@ def attention_forward_splitkv(q, k, v, scale=None, causal=False, window=(-1, -1)
     wsb = fa_fwd_splitkv_workspace_size(B, Nq, Nk, Hq, Hkv, d, c, wl, wr, int(n_splits))
     if workspace is None:
         workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
-    _check("fa_fwd_splitkv",
-           fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+    _check(fn.__name__,
+           fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                           B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, int(n_splits),
                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                           _stream()))
@@ -290,8 +313,9 @@ def attention_forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, 
     if q.dim() != 3 or k.dim() != 3 or v.dim() != 3 or k.shape != v.shape or k.shape[2] != q.shape[2]:
         raise ValueError("q must be [total_q, Hq, d] and k, v [total_k, Hkv, d]")
     for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous() or t.dtype != torch.bfloat16:
-            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+        if not t.is_cuda or not t.is_contiguous() or t.dtype not in (torch.bfloat16, torch.float16) \
+                or t.dtype != q.dtype:
+            raise ValueError("q, k, v must be contiguous CUDA tensors, all bf16 or all fp16")
     for t in (cu_seqlens_q, cu_seqlens_k):
         if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.dim() != 1:
             raise ValueError("cu_seqlens must be contiguous int32 CUDA vectors")
@@ -304,8 +328,9 @@ def attention_forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, 
     c, wl, wr = _window(causal, window)
     o = torch.empty_like(q) if out is None else out
     lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device) if lse is None else lse
-    _check("fa_fwd_varlen",
-           fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+    fn = fa_fwd_varlen if q.dtype == torch.bfloat16 else fa_fwd_varlen_f16
+    _check(fn.__name__,
+           fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                          cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
                          int(max_seqlen_k), total_q, total_k, Hq, Hkv, d, scale, c, wl, wr,
                          _stream()))
@@ -329,8 +354,9 @@ def attention_backward_varlen(q, k, v, o, lse, do, cu_seqlens_q, cu_seqlens_k, m
     wsb = fa_bwd_workspace_size(B, int(max_seqlen_q), Hq, d)
     if workspace is None:
         workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
-    _check("fa_bwd_varlen",
-           fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+    fn = fa_bwd_varlen if q.dtype == torch.bfloat16 else fa_bwd_varlen_f16
+    _check(fn.__name__,
+           fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                          do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                          cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, int(max_seqlen_q),
                          int(max_seqlen_k), total_q, total_k, Hq, Hkv, d, scale, c, wl, wr,
@@ -350,8 +376,9 @@ def attention_forward_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache
     k_new / v_new)."""
     import torch
     B, Nq, Nk, Hq, Hkv, d = _dims(q, k_cache, v_cache)
-    if q.dtype != torch.bfloat16:
-        raise ValueError("fa_fwd_kvcache takes bf16 tensors")
+    if q.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("fa_fwd_kvcache takes bf16 or fp16 tensors")
+    fn = fa_fwd_kvcache if q.dtype == torch.bfloat16 else fa_fwd_kvcache_f16
     n_new = 0
     if k_new is not None or v_new is not None:
         if k_new is None or v_new is None or k_new.shape != v_new.shape:
@@ -359,7 +386,7 @@ def attention_forward_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache
         if k_new.dim() != 4 or k_new.shape[0] != B or k_new.shape[2:] != k_cache.shape[2:]:
             raise ValueError("k_new must be [B, n_new, Hkv, d]")
         if not (k_new.is_contiguous() and v_new.is_contiguous()) or k_new.dtype != q.dtype:
-            raise ValueError("k_new / v_new must be contiguous bf16")
+            raise ValueError("k_new / v_new must be contiguous, of q's dtype")
         n_new = int(k_new.shape[1])
     if cache_seqlens is not None:
         if cache_seqlens.dtype != torch.int32 or not cache_seqlens.is_cuda or \
@@ -374,8 +401,8 @@ def attention_forward_kvcache(q, k_cache, v_cache, k_new=None, v_new=None, cache
     if workspace is None:
         workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
     ptr = lambda t: None if t is None else t.data_ptr()
-    _check("fa_fwd_kvcache",
-           fa_fwd_kvcache(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), ptr(k_new),
+    _check(fn.__name__,
+           fn(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), ptr(k_new),
                           ptr(v_new), ptr(cache_seqlens), o.data_ptr(), lse.data_ptr(), B, Nq, Nk,
                           n_new, Hq, Hkv, d, scale, c, wl, wr, int(n_splits), workspace.data_ptr(),
                           workspace.numel() * workspace.element_size(), _stream()))
@@ -399,7 +426,7 @@ def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1
     wsb = fa_bwd_workspace_size(B, Nq, Hq, d)
     if workspace is None:
         workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
-    fn = fa_bwd if q.dtype == torch.bfloat16 else fa_bwd_f32
+    fn = {torch.bfloat16: fa_bwd, torch.float16: fa_bwd_f16}.get(q.dtype, fa_bwd_f32)
     _check(fn.__name__, fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                            do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Nq, Nk,
                            Hq, Hkv, d, scale, c, wl, wr, workspace.data_ptr(),

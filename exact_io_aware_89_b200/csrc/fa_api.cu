@@ -3,6 +3,7 @@
 // stream.  No device memory is allocated here and nothing runs on the CPU
 // besides the checks.
 #include <atomic>
+#include <type_traits>
 #include <cstdio>
 #include <mutex>
 #include <vector>
@@ -84,6 +85,14 @@ constexpr int kMaxDecodeSplits = 4096;
 
 constexpr int kMaxDevices = 64;
 
+// a configuration with bf16 elements (F16 false) or fp16 elements
+template <bool F16, class C>
+using Ty = std::conditional_t<F16, AsF16<C>, C>;
+
+constexpr CUtensorMapDataType tma_type(bool f16) {
+  return f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+}
+
 template <typename Kernel>
 cudaError_t smem_attr_once(Kernel kernel, int bytes, int* done) {
   int dev = 0;
@@ -135,8 +144,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                int Nk, int Hq, int Hkv, float scale, const MaskSpec& mask, cudaStream_t stream) {
   static int attr_done[kMaxDevices] = {0};
   CUtensorMap tq, tk, tv, to;
-  if (!encode_bnhd(&tq, q, B, Nq, Hq, C::D, C::BM) || !encode_bnhd(&tk, k, B, Nk, Hkv, C::D, C::BN) ||
-      !encode_bnhd(&tv, v, B, Nk, Hkv, C::D, C::BN) || !encode_bnhd(&to, o, B, Nq, Hq, C::D, C::BM))
+  if (!encode_bnhd(&tq, q, B, Nq, Hq, C::D, C::BM, tma_type(C::F16)) || !encode_bnhd(&tk, k, B, Nk, Hkv, C::D, C::BN, tma_type(C::F16)) ||
+      !encode_bnhd(&tv, v, B, Nk, Hkv, C::D, C::BN, tma_type(C::F16)) || !encode_bnhd(&to, o, B, Nq, Hq, C::D, C::BM, tma_type(C::F16)))
     return FA_ERR_CUDA;
   FwdParams p;
   p.B = B; p.Nq = Nq; p.Nk = Nk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
@@ -148,7 +157,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.cu_q = nullptr;
   p.cu_k = nullptr;
   p.total_q = 0;
-  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o = static_cast<uint16_t*>(o);
   p.wait_limit_ns = kWaitLimitNs;
   auto kern = fa_fwd_kernel<C>;
   if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
@@ -168,8 +177,8 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
                       int Hkv, float scale, int causal, int win_l, int win_r, cudaStream_t stream) {
   static int attr_done[kMaxDevices] = {0};
   CUtensorMap tq, tk, tv, to;
-  if (!encode_bnhd(&tq, q, 1, total_q, Hq, C::D, C::BM) || !encode_bnhd(&tk, k, 1, total_k, Hkv, C::D, C::BN) ||
-      !encode_bnhd(&tv, v, 1, total_k, Hkv, C::D, C::BN) || !encode_bnhd(&to, o, 1, total_q, Hq, C::D, C::BM))
+  if (!encode_bnhd(&tq, q, 1, total_q, Hq, C::D, C::BM, tma_type(C::F16)) || !encode_bnhd(&tk, k, 1, total_k, Hkv, C::D, C::BN, tma_type(C::F16)) ||
+      !encode_bnhd(&tv, v, 1, total_k, Hkv, C::D, C::BN, tma_type(C::F16)) || !encode_bnhd(&to, o, 1, total_q, Hq, C::D, C::BM, tma_type(C::F16)))
     return FA_ERR_CUDA;
   FwdParams p;
   p.B = B; p.Nq = max_q; p.Nk = max_k; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
@@ -181,7 +190,7 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
   p.cu_q = cu_q;
   p.cu_k = cu_k;
   p.total_q = total_q;
-  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o = static_cast<uint16_t*>(o);
   p.wait_limit_ns = kWaitLimitNs;
   auto kern = fa_fwd_kernel<C, true>;
   if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
@@ -219,8 +228,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     constexpr int RPG = 4;    // rows per lane group
     const long long blocks = (rows_pad * G / RPG + 255) / 256;
     TraceScope tr(FA_KERNEL_BWD_PREP, stream);
-    fa_bwd_prep_bf16_kernel<G, RPG, VL><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, ws, B, Nq,
+    fa_bwd_prep_h16_kernel<G, RPG, VL, CQ::F16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dO), lse, ws, B, Nq,
         Hq, Nq_pad, vl.cu_q, vl.total_q);
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
@@ -240,18 +249,18 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.cu_k = vl.cu_k;
   p.total_q = vl.total_q;
   p.total_k = vl.total_k;
-  p.dq = static_cast<__nv_bfloat16*>(dq);
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dq = static_cast<uint16_t*>(dq);
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
   p.wait_limit_ns = kWaitLimitNs;
   // tensor-map shapes: dense [B, N, H, d]; packed [1, total, H, d]
   const bool packed = VL;
   const int mB = packed ? 1 : B, mNq = packed ? vl.total_q : Nq, mNk = packed ? vl.total_k : Nk;
   {
     CUtensorMap tq, tk, tv, tdo, tdq;
-    if (!encode_bnhd(&tq, q, mB, mNq, Hq, D, CQ::BM) || !encode_bnhd(&tk, k, mB, mNk, Hkv, D, CQ::BN) ||
-        !encode_bnhd(&tv, v, mB, mNk, Hkv, D, CQ::BN) || !encode_bnhd(&tdo, dO, mB, mNq, Hq, D, CQ::BM) ||
-        !encode_bnhd(&tdq, dq, mB, mNq, Hq, D, CQ::BM))
+    if (!encode_bnhd(&tq, q, mB, mNq, Hq, D, CQ::BM, tma_type(CQ::F16)) || !encode_bnhd(&tk, k, mB, mNk, Hkv, D, CQ::BN, tma_type(CQ::F16)) ||
+        !encode_bnhd(&tv, v, mB, mNk, Hkv, D, CQ::BN, tma_type(CQ::F16)) || !encode_bnhd(&tdo, dO, mB, mNq, Hq, D, CQ::BM, tma_type(CQ::F16)) ||
+        !encode_bnhd(&tdq, dq, mB, mNq, Hq, D, CQ::BM, tma_type(CQ::F16)))
       return FA_ERR_CUDA;
     const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
     if constexpr (CQ::ONE_TILE) {
@@ -269,9 +278,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   }
   {
     CUtensorMap tq, tk, tv, tdo, tdk, tdv;
-    if (!encode_bnhd(&tq, q, mB, mNq, Hq, D, CKV::BM) || !encode_bnhd(&tk, k, mB, mNk, Hkv, D, CKV::BN) ||
-        !encode_bnhd(&tv, v, mB, mNk, Hkv, D, CKV::BN) || !encode_bnhd(&tdo, dO, mB, mNq, Hq, D, CKV::BM) ||
-        !encode_bnhd(&tdk, dk, mB, mNk, Hkv, D, CKV::BN) || !encode_bnhd(&tdv, dv, mB, mNk, Hkv, D, CKV::BN))
+    if (!encode_bnhd(&tq, q, mB, mNq, Hq, D, CKV::BM, tma_type(CKV::F16)) || !encode_bnhd(&tk, k, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)) ||
+        !encode_bnhd(&tv, v, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)) || !encode_bnhd(&tdo, dO, mB, mNq, Hq, D, CKV::BM, tma_type(CKV::F16)) ||
+        !encode_bnhd(&tdk, dk, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)) || !encode_bnhd(&tdv, dv, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)))
       return FA_ERR_CUDA;
     auto kern = fa_bwd_dkdv_kernel<CKV, VL>;
     if (smem_attr_once(kern, CKV::SMEM_BYTES, attr_kv) != cudaSuccess) return FA_ERR_CUDA;
@@ -382,17 +391,18 @@ int launch_decode_cfg(const void* q, const CUtensorMap& tk, const CUtensorMap& t
   if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
   TraceScope tr(FA_KERNEL_DECODE, stream);
   kern<<<static_cast<unsigned>(grid), C::NTHREADS, C::SMEM_BYTES, stream>>>(
-      static_cast<const __nv_bfloat16*>(q), tk, tv, p);
+      static_cast<const uint16_t*>(q), tk, tv, p);
   return launch_status();
 }
 
-template <int D, template <int> class Cfg>
+template <int D, template <int> class Cfg, bool F16>
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
                   int Nk, int Hq, int Hkv, float scale, const MaskSpec& mask, const DecodePlan& pl,
                   const int* seqlens, int n_new, void* workspace, cudaStream_t stream) {
   CUtensorMap tk, tv;
   const int bn = Cfg<32>::BN;
-  if (!encode_bnhd(&tk, k, B, Nk, Hkv, D, bn) || !encode_bnhd(&tv, v, B, Nk, Hkv, D, bn)) return FA_ERR_CUDA;
+  if (!encode_bnhd(&tk, k, B, Nk, Hkv, D, bn, tma_type(F16)) || !encode_bnhd(&tv, v, B, Nk, Hkv, D, bn, tma_type(F16)))
+    return FA_ERR_CUDA;
   DecodeParams p;
   p.B = B; p.Nq = Nq; p.Nk = Nk; p.Hq = Hq; p.Hkv = Hkv; p.group = pl.group;
   p.qpt = pl.qpt;
@@ -403,7 +413,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.mask = mask;
   p.seqlens = seqlens;
   p.n_new = n_new;
-  p.o = static_cast<__nv_bfloat16*>(o);
+  p.o = static_cast<uint16_t*>(o);
   p.lse = lse;
   const size_t rows = static_cast<size_t>(pl.units) * pl.n_splits * pl.rt;
   const bool split = pl.n_splits > 1;
@@ -416,9 +426,9 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.wait_limit_ns = kWaitLimitNs;
   const long long grid = pl.units * pl.n_splits;
   switch (pl.rcp) {
-    case 32: return launch_decode_cfg<Cfg<32>>(q, tk, tv, p, grid, stream);
-    case 64: return launch_decode_cfg<Cfg<64>>(q, tk, tv, p, grid, stream);
-    default: return launch_decode_cfg<Cfg<128>>(q, tk, tv, p, grid, stream);
+    case 32: return launch_decode_cfg<Ty<F16, Cfg<32>>>(q, tk, tv, p, grid, stream);
+    case 64: return launch_decode_cfg<Ty<F16, Cfg<64>>>(q, tk, tv, p, grid, stream);
+    default: return launch_decode_cfg<Ty<F16, Cfg<128>>>(q, tk, tv, p, grid, stream);
   }
 }
 
@@ -452,9 +462,10 @@ int scratch_for_current_device(float** out) {
 }
 }  // namespace
 
-extern "C" {
+namespace {
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq, int Nk,
+template <bool F16>
+int fa_fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq, int Nk,
            int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
            fa_stream_t stream) {
   int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
@@ -463,19 +474,15 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (d) {
-    case 64: return launch_fwd<Fwd64>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, s);
-    case 128: return launch_fwd<Fwd128>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, s);
-    case 256: return launch_fwd<Fwd256>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, s);
+    case 64: return launch_fwd<Ty<F16, Fwd64>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, s);
+    case 128: return launch_fwd<Ty<F16, Fwd128>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, s);
+    case 256: return launch_fwd<Ty<F16, Fwd256>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, s);
     default: return FA_ERR_UNSUPPORTED;
   }
 }
 
-size_t fa_bwd_workspace_size(int B, int Nq, int Hq, int d) {
-  if (d < 1) return 0;
-  return workspace_bytes(B, Nq, Hq);
-}
-
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+template <bool F16>
+int fa_bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
            const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
            int d, float scale, int causal, int win_l, int win_r, void* workspace,
            size_t workspace_bytes_, fa_stream_t stream) {
@@ -491,12 +498,186 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
   float* ws = static_cast<float*>(workspace);
   switch (d) {
     case 64:
-      return launch_bwd<Dq64, Dkv64>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+      return launch_bwd<Ty<F16, Dq64>, Ty<F16, Dkv64>>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
     case 128:
-      return launch_bwd<Dq128, Dkv128>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+      return launch_bwd<Ty<F16, Dq128>, Ty<F16, Dkv128>>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
     default:
-      return launch_bwd<Dq256, Dkv256>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
+      return launch_bwd<Ty<F16, Dq256>, Ty<F16, Dkv256>>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s);
   }
+}
+
+template <bool F16>
+int fa_fwd_splitkv_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+                   int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                   int n_splits, void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  DecodePlan pl;
+  st = plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(), false, &pl);
+  if (st != FA_OK) return st;
+  const size_t need = decode_workspace_bytes(pl, d);
+  if (need > 0 && (!aligned16(workspace) || workspace_bytes_ < need)) return FA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64:
+      return launch_decode<64, Dec64, F16>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, nullptr, 0, workspace, s);
+    case 128:
+      return launch_decode<128, Dec128, F16>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, nullptr, 0, workspace, s);
+    default:
+      return launch_decode<256, Dec256, F16>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, nullptr, 0, workspace, s);
+  }
+}
+
+template <bool F16>
+int fa_fwd_kvcache_impl(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                   const int* cache_seqlens, void* o, float* lse, int B, int Nq, int Nk, int n_new,
+                   int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r, int n_splits,
+                   void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_common(q, k_cache, v_cache, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if (n_new < 0) return FA_ERR_INVALID_ARG;
+  if (n_new > 0 && (!aligned16(k_new) || !aligned16(v_new) || cache_seqlens == nullptr))
+    return FA_ERR_INVALID_ARG;
+  if (cache_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  DecodePlan pl;
+  st = plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(),
+                   cache_seqlens != nullptr, &pl);
+  if (st != FA_OK) return st;
+  const size_t need = decode_workspace_bytes(pl, d);
+  if (need > 0 && (!aligned16(workspace) || workspace_bytes_ < need)) return FA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (n_new > 0) {
+    const long long units = static_cast<long long>(B) * n_new * Hkv * (d / 8);
+    const long long blocks = (units + 255) / 256 < 4096 ? (units + 255) / 256 : 4096;
+    TraceScope tr(FA_KERNEL_KVCACHE_APPEND, s);
+    fa_kvcache_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+        static_cast<uint16_t*>(k_cache), static_cast<uint16_t*>(v_cache),
+        static_cast<const uint16_t*>(k_new), static_cast<const uint16_t*>(v_new), cache_seqlens, B,
+        n_new, Nk, Hkv, d);
+    if (launch_status() != FA_OK) return FA_ERR_CUDA;
+  }
+  switch (d) {
+    case 64:
+      return launch_decode<64, Dec64, F16>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
+                                      cache_seqlens, n_new, workspace, s);
+    case 128:
+      return launch_decode<128, Dec128, F16>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
+                                        cache_seqlens, n_new, workspace, s);
+    default:
+      return launch_decode<256, Dec256, F16>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
+                                        cache_seqlens, n_new, workspace, s);
+  }
+}
+
+template <bool F16>
+int fa_fwd_varlen_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                  int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, float scale,
+                  int causal, int win_l, int win_r, fa_stream_t stream) {
+  int st = check_common(q, k, v, 1, total_q, total_k, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || max_seqlen_q < 1 || max_seqlen_k < 1 || max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Hq * ((max_seqlen_q + 127) / 128) > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64:
+      return launch_fwd_varlen<Ty<F16, Fwd64>>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                                      total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
+    case 128:
+      return launch_fwd_varlen<Ty<F16, Fwd128>>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                                       total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
+    case 256:
+      return launch_fwd_varlen<Ty<F16, Fwd256>>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
+                                       total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
+    default:
+      return FA_ERR_UNSUPPORTED;
+  }
+}
+
+template <bool F16>
+int fa_bwd_varlen_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dO, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q,
+                  int total_k, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                  void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_common(q, k, v, 1, total_q, total_k, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv))
+    return FA_ERR_INVALID_ARG;
+  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || max_seqlen_q < 1 || max_seqlen_k < 1 || max_seqlen_q > total_q || max_seqlen_k > total_k)
+    return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Hq * ((max_seqlen_q + 127) / 128) > (1ll << 31) - 1 ||
+      static_cast<long long>(B) * Hkv * ((max_seqlen_k + 63) / 64) > (1ll << 31) - 1)
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(workspace) || workspace_bytes_ < workspace_bytes(B, max_seqlen_q, Hq)) return FA_ERR_WORKSPACE;
+  const MaskSpec mask = make_mask(max_seqlen_q, max_seqlen_k, causal, win_l, win_r);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  Varlen vl;
+  vl.cu_q = cu_seqlens_q;
+  vl.cu_k = cu_seqlens_k;
+  vl.total_q = total_q;
+  vl.total_k = total_k;
+  const int Nq = max_seqlen_q, Nk = max_seqlen_k;
+  switch (d) {
+    case 64:
+      return launch_bwd<Ty<F16, Dq64>, Ty<F16, Dkv64>, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s, vl);
+    case 128:
+      return launch_bwd<Ty<F16, Dq128>, Ty<F16, Dkv128>, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s, vl);
+    default:
+      return launch_bwd<Ty<F16, Dq256>, Ty<F16, Dkv256>, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s, vl);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq, int Nk,
+           int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+           fa_stream_t stream) {
+  return fa_fwd_impl<false>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, stream);
+}
+
+int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq, int Nk,
+           int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+           fa_stream_t stream) {
+  return fa_fwd_impl<true>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, stream);
+}
+
+size_t fa_bwd_workspace_size(int B, int Nq, int Hq, int d) {
+  if (d < 1) return 0;
+  return workspace_bytes(B, Nq, Hq);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
+           int d, float scale, int causal, int win_l, int win_r, void* workspace,
+           size_t workspace_bytes_, fa_stream_t stream) {
+  return fa_bwd_impl<false>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, workspace, workspace_bytes_, stream);
+}
+
+int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const float* lse,
+           const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
+           int d, float scale, int causal, int win_l, int win_r, void* workspace,
+           size_t workspace_bytes_, fa_stream_t stream) {
+  return fa_bwd_impl<true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, workspace, workspace_bytes_, stream);
 }
 
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -552,97 +733,41 @@ size_t fa_fwd_kvcache_workspace_size(int B, int Nq, int Nk, int Hq, int Hkv, int
 int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
                    int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
                    int n_splits, void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
-  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
-  if (st != FA_OK) return st;
-  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
-  DecodePlan pl;
-  st = plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(), false, &pl);
-  if (st != FA_OK) return st;
-  const size_t need = decode_workspace_bytes(pl, d);
-  if (need > 0 && (!aligned16(workspace) || workspace_bytes_ < need)) return FA_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  switch (d) {
-    case 64:
-      return launch_decode<64, Dec64>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, nullptr, 0, workspace, s);
-    case 128:
-      return launch_decode<128, Dec128>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, nullptr, 0, workspace, s);
-    default:
-      return launch_decode<256, Dec256>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl, nullptr, 0, workspace, s);
-  }
+  return fa_fwd_splitkv_impl<false>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, n_splits, workspace, workspace_bytes_, stream);
+}
+
+int fa_fwd_splitkv_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+                   int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                   int n_splits, void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  return fa_fwd_splitkv_impl<true>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, n_splits, workspace, workspace_bytes_, stream);
 }
 
 int fa_fwd_kvcache(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
                    const int* cache_seqlens, void* o, float* lse, int B, int Nq, int Nk, int n_new,
                    int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r, int n_splits,
                    void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
-  int st = check_common(q, k_cache, v_cache, B, Nq, Nk, Hq, Hkv, scale);
-  if (st != FA_OK) return st;
-  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
-  if (n_new < 0) return FA_ERR_INVALID_ARG;
-  if (n_new > 0 && (!aligned16(k_new) || !aligned16(v_new) || cache_seqlens == nullptr))
-    return FA_ERR_INVALID_ARG;
-  if (cache_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
-  DecodePlan pl;
-  st = plan_decode(B, Nq, Hq, Hkv, d, mask, n_splits, n_splits > 0 ? 0 : current_sm_count(),
-                   cache_seqlens != nullptr, &pl);
-  if (st != FA_OK) return st;
-  const size_t need = decode_workspace_bytes(pl, d);
-  if (need > 0 && (!aligned16(workspace) || workspace_bytes_ < need)) return FA_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (n_new > 0) {
-    const long long units = static_cast<long long>(B) * n_new * Hkv * (d / 8);
-    const long long blocks = (units + 255) / 256 < 4096 ? (units + 255) / 256 : 4096;
-    TraceScope tr(FA_KERNEL_KVCACHE_APPEND, s);
-    fa_kvcache_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-        static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache),
-        static_cast<const __nv_bfloat16*>(k_new), static_cast<const __nv_bfloat16*>(v_new), cache_seqlens, B,
-        n_new, Nk, Hkv, d);
-    if (launch_status() != FA_OK) return FA_ERR_CUDA;
-  }
-  switch (d) {
-    case 64:
-      return launch_decode<64, Dec64>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
-                                      cache_seqlens, n_new, workspace, s);
-    case 128:
-      return launch_decode<128, Dec128>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
-                                        cache_seqlens, n_new, workspace, s);
-    default:
-      return launch_decode<256, Dec256>(q, k_cache, v_cache, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, pl,
-                                        cache_seqlens, n_new, workspace, s);
-  }
+  return fa_fwd_kvcache_impl<false>(q, k_cache, v_cache, k_new, v_new, cache_seqlens, o, lse, B, Nq, Nk, n_new, Hq, Hkv, d, scale, causal, win_l, win_r, n_splits, workspace, workspace_bytes_, stream);
+}
+
+int fa_fwd_kvcache_f16(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                   const int* cache_seqlens, void* o, float* lse, int B, int Nq, int Nk, int n_new,
+                   int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r, int n_splits,
+                   void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  return fa_fwd_kvcache_impl<true>(q, k_cache, v_cache, k_new, v_new, cache_seqlens, o, lse, B, Nq, Nk, n_new, Hq, Hkv, d, scale, causal, win_l, win_r, n_splits, workspace, workspace_bytes_, stream);
 }
 
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
                   const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
                   int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, float scale,
                   int causal, int win_l, int win_r, fa_stream_t stream) {
-  int st = check_common(q, k, v, 1, total_q, total_k, Hq, Hkv, scale);
-  if (st != FA_OK) return st;
-  if (!aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
-  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr ||
-      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
-    return FA_ERR_INVALID_ARG;
-  if (B < 1 || max_seqlen_q < 1 || max_seqlen_k < 1 || max_seqlen_q > total_q || max_seqlen_k > total_k)
-    return FA_ERR_INVALID_ARG;
-  if (static_cast<long long>(B) * Hq * ((max_seqlen_q + 127) / 128) > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  switch (d) {
-    case 64:
-      return launch_fwd_varlen<Fwd64>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
-                                      total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
-    case 128:
-      return launch_fwd_varlen<Fwd128>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
-                                       total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
-    case 256:
-      return launch_fwd_varlen<Fwd256>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k,
-                                       total_q, total_k, Hq, Hkv, scale, causal, win_l, win_r, s);
-    default:
-      return FA_ERR_UNSUPPORTED;
-  }
+  return fa_fwd_varlen_impl<false>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d, scale, causal, win_l, win_r, stream);
+}
+
+int fa_fwd_varlen_f16(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                  int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, float scale,
+                  int causal, int win_l, int win_r, fa_stream_t stream) {
+  return fa_fwd_varlen_impl<true>(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d, scale, causal, win_l, win_r, stream);
 }
 
 int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -650,38 +775,15 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
                   const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q,
                   int total_k, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
                   void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
-  int st = check_common(q, k, v, 1, total_q, total_k, Hq, Hkv, scale);
-  if (st != FA_OK) return st;
-  if (!aligned16(o) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
-      !aligned16(dv))
-    return FA_ERR_INVALID_ARG;
-  if (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr ||
-      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) != 0 || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
-    return FA_ERR_INVALID_ARG;
-  if (B < 1 || max_seqlen_q < 1 || max_seqlen_k < 1 || max_seqlen_q > total_q || max_seqlen_k > total_k)
-    return FA_ERR_INVALID_ARG;
-  if (static_cast<long long>(B) * Hq * ((max_seqlen_q + 127) / 128) > (1ll << 31) - 1 ||
-      static_cast<long long>(B) * Hkv * ((max_seqlen_k + 63) / 64) > (1ll << 31) - 1)
-    return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
-  if (!aligned16(workspace) || workspace_bytes_ < workspace_bytes(B, max_seqlen_q, Hq)) return FA_ERR_WORKSPACE;
-  const MaskSpec mask = make_mask(max_seqlen_q, max_seqlen_k, causal, win_l, win_r);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  float* ws = static_cast<float*>(workspace);
-  Varlen vl;
-  vl.cu_q = cu_seqlens_q;
-  vl.cu_k = cu_seqlens_k;
-  vl.total_q = total_q;
-  vl.total_k = total_k;
-  const int Nq = max_seqlen_q, Nk = max_seqlen_k;
-  switch (d) {
-    case 64:
-      return launch_bwd<Dq64, Dkv64, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s, vl);
-    case 128:
-      return launch_bwd<Dq128, Dkv128, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s, vl);
-    default:
-      return launch_bwd<Dq256, Dkv256, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq, Hkv, scale, mask, ws, s, vl);
-  }
+  return fa_bwd_varlen_impl<false>(q, k, v, o, lse, dO, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d, scale, causal, win_l, win_r, workspace, workspace_bytes_, stream);
+}
+
+int fa_bwd_varlen_f16(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                  const void* dO, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                  const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q,
+                  int total_k, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                  void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
+  return fa_bwd_varlen_impl<true>(q, k, v, o, lse, dO, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d, scale, causal, win_l, win_r, workspace, workspace_bytes_, stream);
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Nq,

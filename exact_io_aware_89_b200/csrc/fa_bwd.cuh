@@ -71,16 +71,16 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const T* __restrict__ 
   }
 }
 
-// bf16: G = d / 8 lanes per row, each loading 8 elements of O and of dO with
+// bf16 or fp16 (F16): G = d / 8 lanes per row, each loading 8 elements of O and of dO with
 // one 16-byte load; the G partial dot products are added with shuffles inside
 // the lane group (groups are aligned within the warp, G divides 32).  Each
 // lane group handles RPG rows, with all their loads issued before any use, so
 // that enough bytes are in flight to approach HBM bandwidth.  Same outputs
 // and layout as fa_bwd_prep_kernel; rows_pad must be a multiple of
 // RPG * 256 / G (it is a multiple of 256).
-template <int G, int RPG, bool VL = false>
-__global__ void __launch_bounds__(256) fa_bwd_prep_bf16_kernel(const __nv_bfloat16* __restrict__ o,
-                                                               const __nv_bfloat16* __restrict__ dout,
+template <int G, int RPG, bool VL = false, bool F16 = false>
+__global__ void __launch_bounds__(256) fa_bwd_prep_h16_kernel(const uint16_t* __restrict__ o,
+                                                               const uint16_t* __restrict__ dout,
                                                                const float* __restrict__ lse,
                                                                float* __restrict__ ws, int B, int Nq,
                                                                int Hq, int Nq_pad,
@@ -123,9 +123,8 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_bf16_kernel(const __nv_bfloat
       const uint32_t* gp = reinterpret_cast<const uint32_t*>(&gv[k]);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        // a bf16 is the top half of an fp32
-        acc = fmaf(__uint_as_float(op[u] << 16), __uint_as_float(gp[u] << 16), acc);
-        acc = fmaf(__uint_as_float(op[u] & 0xFFFF0000u), __uint_as_float(gp[u] & 0xFFFF0000u), acc);
+        acc = fmaf(h16_to_f32<F16>(op[u] & 0xFFFFu), h16_to_f32<F16>(gp[u] & 0xFFFFu), acc);
+        acc = fmaf(h16_to_f32<F16>(op[u] >> 16), h16_to_f32<F16>(gp[u] >> 16), acc);
       }
     }
 #pragma unroll
@@ -166,9 +165,9 @@ struct BwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q, total_k;
-  __nv_bfloat16* dq;  // outputs, for the plain stores of a packed sequence's last tile
-  __nv_bfloat16* dk;
-  __nv_bfloat16* dv;
+  uint16_t* dq;  // outputs, for the plain stores of a packed sequence's last tile
+  uint16_t* dk;
+  uint16_t* dv;
   unsigned long long wait_limit_ns;
 };
 
@@ -177,6 +176,7 @@ struct BwdParams {
 // =====================================================================
 template <int D_, int NQT_, int BN_, int KST_>
 struct DqCfg {
+  static constexpr bool F16 = false;  // elements are bf16 (AsF16<> flips it to fp16)
   static constexpr int D = D_, NQT = NQT_, BN = BN_, KST = KST_;
   static constexpr int BM = 128;
   static constexpr bool ONE_TILE = false;
@@ -294,8 +294,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
   } else if (warp == C::MMA_WARP) {
     if (lane == 0 && n_kv > 0) {
-      constexpr uint32_t ID_S = idesc_bf16_f32(128, BN, false, false);
-      constexpr uint32_t ID_DQ = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t ID_S = idesc_kind_f16<C::F16>(128, BN, false, false);
+      constexpr uint32_t ID_DQ = idesc_kind_f16<C::F16>(128, D, false, true);
       auto wait = [&](uint64_t* bar, uint32_t par) {
         const bool ok = mbar_wait(bar, par, abort_flag, &g_status, p.wait_limit_ns);
         tc_fence_after();
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       for (int c = 0; c < BN; c += 2) {
         const float p0 = ex2_approx(fmaf(sc[c], sl2, -lse2));
         const float p1 = ex2_approx(fmaf(sc[c + 1], sl2, -lse2));
-        pk[c / 2] = pack_bf16x2(p0 * (dp[c] - Drow), p1 * (dp[c + 1] - Drow));
+        pk[c / 2] = pack2<C::F16>(p0 * (dp[c] - Drow), p1 * (dp[c + 1] - Drow));
       }
 #pragma unroll
       for (int cc = 0; cc < BN / 64; ++cc) tmem_st_x32(lane_base + col_dp + cc * 32, &pk[cc * 32]);
@@ -439,9 +439,9 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const float* f = reinterpret_cast<const float*>(ov + 8 * u);
-          st_shared_v4(stage + c * C::QCHUNK + sw128_offset(r, u), pack_bf16x2(f[0] * sc, f[1] * sc),
-                       pack_bf16x2(f[2] * sc, f[3] * sc), pack_bf16x2(f[4] * sc, f[5] * sc),
-                       pack_bf16x2(f[6] * sc, f[7] * sc));
+          st_shared_v4(stage + c * C::QCHUNK + sw128_offset(r, u), pack2<C::F16>(f[0] * sc, f[1] * sc),
+                       pack2<C::F16>(f[2] * sc, f[3] * sc), pack2<C::F16>(f[4] * sc, f[5] * sc),
+                       pack2<C::F16>(f[6] * sc, f[7] * sc));
         }
       }
       fence_proxy_async_smem();
@@ -479,6 +479,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 // ring: each tile's loads are issued two steps ahead of their use.
 template <int D_, int KS_, int VS_>
 struct Dq2Cfg {
+  static constexpr bool F16 = false;  // elements are bf16 (AsF16<> flips it to fp16)
   static constexpr int D = D_, KS = KS_, VS = VS_;
   static constexpr int BM = 128, BN = 128;
   static constexpr int NQT = 1;
@@ -629,8 +630,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
   } else if (warp == C::MMA_WARP) {
     if (lane == 0 && n_kv > 0) {
-      constexpr uint32_t ID_S = idesc_bf16_f32(128, BN, false, false);
-      constexpr uint32_t ID_DQ = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t ID_S = idesc_kind_f16<C::F16>(128, BN, false, false);
+      constexpr uint32_t ID_DQ = idesc_kind_f16<C::F16>(128, D, false, true);
       auto wait = [&](uint64_t* bar, uint32_t par) {
         const bool ok = mbar_wait(bar, par, abort_flag, &g_status, p.wait_limit_ns);
         tc_fence_after();
@@ -729,7 +730,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       for (int c = 0; c < 64; c += 2) {
         const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse2));
         const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse2));
-        pk[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - Drow), p1 * (__uint_as_float(dv[c + 1]) - Drow));
+        pk[c / 2] = pack2<C::F16>(p0 * (__uint_as_float(dv[c]) - Drow), p1 * (__uint_as_float(dv[c + 1]) - Drow));
       }
       // the previous key tile's dQ MMA must be done reading dS
       if (it > 0) {
@@ -767,9 +768,9 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const float* f = reinterpret_cast<const float*>(ov + 8 * u);
-          st_shared_v4(sQ + c * C::QCHUNK + sw128_offset(r, u), pack_bf16x2(f[0] * sc, f[1] * sc),
-                       pack_bf16x2(f[2] * sc, f[3] * sc), pack_bf16x2(f[4] * sc, f[5] * sc),
-                       pack_bf16x2(f[6] * sc, f[7] * sc));
+          st_shared_v4(sQ + c * C::QCHUNK + sw128_offset(r, u), pack2<C::F16>(f[0] * sc, f[1] * sc),
+                       pack2<C::F16>(f[2] * sc, f[3] * sc), pack2<C::F16>(f[4] * sc, f[5] * sc),
+                       pack2<C::F16>(f[6] * sc, f[7] * sc));
         }
       }
       fence_proxy_async_smem();
@@ -801,6 +802,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 // depth of the (Q, dO, lse2, D) stages; LA: steps issued ahead (<= 2, <= ST).
 template <int D_, int DV_, int BM_, int ST_>
 struct DkvCfg {
+  static constexpr bool F16 = false;  // elements are bf16 (AsF16<> flips it to fp16)
   static constexpr int D = D_, DV = DV_, BM = BM_, ST = ST_;
   static constexpr int BN = 128;
   static constexpr int LA = ST >= 2 ? 2 : 1;
@@ -946,8 +948,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
   } else if (warp == C::MMA_WARP) {
     if (lane == 0 && n_steps > 0) {
-      constexpr uint32_t ID_S = idesc_bf16_f32(128, BM, false, false);
-      constexpr uint32_t ID_ACC = idesc_bf16_f32(128, DV, false, true);
+      constexpr uint32_t ID_S = idesc_kind_f16<C::F16>(128, BM, false, false);
+      constexpr uint32_t ID_ACC = idesc_kind_f16<C::F16>(128, DV, false, true);
       auto wait = [&](uint64_t* bar, uint32_t par) {
         const bool ok = mbar_wait(bar, par, abort_flag, &g_status, p.wait_limit_ns);
         tc_fence_after();
@@ -1064,11 +1066,11 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
         const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -l4.y));
         const float p2 = ex2_approx(fmaf(__uint_as_float(sv[c + 2]), sl2, -l4.z));
         const float p3 = ex2_approx(fmaf(__uint_as_float(sv[c + 3]), sl2, -l4.w));
-        pp[c / 2] = pack_bf16x2(p0, p1);
-        pp[c / 2 + 1] = pack_bf16x2(p2, p3);
-        dd[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dv[c]) - D4.x), p1 * (__uint_as_float(dv[c + 1]) - D4.y));
+        pp[c / 2] = pack2<C::F16>(p0, p1);
+        pp[c / 2 + 1] = pack2<C::F16>(p2, p3);
+        dd[c / 2] = pack2<C::F16>(p0 * (__uint_as_float(dv[c]) - D4.x), p1 * (__uint_as_float(dv[c + 1]) - D4.y));
         dd[c / 2 + 1] =
-            pack_bf16x2(p2 * (__uint_as_float(dv[c + 2]) - D4.z), p3 * (__uint_as_float(dv[c + 3]) - D4.w));
+            pack2<C::F16>(p2 * (__uint_as_float(dv[c + 2]) - D4.z), p3 * (__uint_as_float(dv[c + 3]) - D4.w));
       }
 #pragma unroll
       for (int cc = 0; cc < BM / 32; ++cc) {
@@ -1106,9 +1108,9 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const float* f = reinterpret_cast<const float*>(ov + 8 * u);
-            st_shared_v4(stage + c * C::KCHUNK + sw128_offset(r, u), pack_bf16x2(f[0] * sc, f[1] * sc),
-                         pack_bf16x2(f[2] * sc, f[3] * sc), pack_bf16x2(f[4] * sc, f[5] * sc),
-                         pack_bf16x2(f[6] * sc, f[7] * sc));
+            st_shared_v4(stage + c * C::KCHUNK + sw128_offset(r, u), pack2<C::F16>(f[0] * sc, f[1] * sc),
+                         pack2<C::F16>(f[2] * sc, f[3] * sc), pack2<C::F16>(f[4] * sc, f[5] * sc),
+                         pack2<C::F16>(f[6] * sc, f[7] * sc));
           }
         }
       }

@@ -3,6 +3,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "sm100_ptx.cuh"
 
@@ -106,6 +107,24 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+// A kernel configuration with fp16 instead of bf16 elements: the same tiles;
+// the tensor-core operand type, the conversions to 16 bits and the TMA data
+// type follow C::F16.
+template <class C>
+struct AsF16 : C {
+  static constexpr bool F16 = true;
+};
+
+// 16-bit float bits to fp32
+template <bool F16>
+__device__ __forceinline__ float h16_to_f32(uint32_t bits16) {
+  if constexpr (F16) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(bits16)));
+  } else {
+    return __uint_as_float(bits16 << 16);
+  }
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -140,7 +159,7 @@ struct SeqView {
 // for the last tile of a packed sequence, whose following rows belong to the
 // next sequence (a TMA store would write them).
 __device__ __forceinline__ void store_rows_sw128(uint32_t stage, int chunk_bytes, int n_rows, int ncols,
-                                                 __nv_bfloat16* dst, int row0, int total, int H, int h,
+                                                 uint16_t* dst, int row0, int total, int H, int h,
                                                  int d, int col0, int tid, int nthreads) {
   const int upr = ncols / 8;
   for (int x = tid; x < n_rows * upr; x += nthreads) {

@@ -47,7 +47,7 @@ struct DecodeParams {
   MaskSpec mask;                  // with Nk = the key capacity; per batch see below
   const int* seqlens;             // [B] cached keys per sequence, or null (all Nk)
   int n_new;                      // keys appended after seqlens[b] by this call
-  __nv_bfloat16* o;               // [B, Nq, Hq, d]
+  uint16_t* o;               // [B, Nq, Hq, d]
   float* lse;                     // [B, Hq, Nq]
   float* part_o;                  // [units, n_splits, RT, d] normalised partial O (n_splits > 1)
   float* part_lse;                // [units, n_splits, RT]    natural-log partial LSE
@@ -59,6 +59,7 @@ struct DecodeParams {
 // RCP: TMEM lanes (rows) one copy of the packed rows spans: 32, 64 or 128.
 template <int D_, int BN_, int KST_, int RCP_>
 struct DecCfg {
+  static constexpr bool F16 = false;  // elements are bf16 (AsF16<> flips it to fp16)
   static constexpr int D = D_, BN = BN_, KST = KST_, RCP = RCP_;
   static constexpr int BM = 128;
   static constexpr int NC = BM / RCP;        // copies of the packed rows
@@ -147,7 +148,7 @@ __device__ __forceinline__ bool decode_claim_last(unsigned long long* ctr, unsig
 
 template <class C>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
-    fa_decode_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap tm_k,
+    fa_decode_kernel(const uint16_t* __restrict__ q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   constexpr int D = C::D, BN = C::BN, KST = C::KST, BM = C::BM, RCP = C::RCP, NC = C::NC, CW = C::CW;
   extern __shared__ uint8_t smem_raw[];
@@ -285,8 +286,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && n_kv > 0) {
-      constexpr uint32_t ID_QK = idesc_bf16_f32(128, BN, false, false);
-      constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t ID_QK = idesc_kind_f16<C::F16>(128, BN, false, false);
+      constexpr uint32_t ID_PV = idesc_kind_f16<C::F16>(128, D, false, true);
       const uint64_t dq0 = sdesc_sw128(sQ, 16, 1024);
       const uint64_t dk0 = sdesc_sw128(sK, 16, 1024);
       const uint64_t dv0 = sdesc_sw128(sV, C::KCHUNK, 1024);
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       for (int x = 0; x < CW; x += 2) {
         const float p0 = ex2_approx(fmaf(sc[x], sl2, -mb));
         const float p1 = ex2_approx(fmaf(sc[x + 1], sl2, -mb));
-        pk[x / 2] = pack_bf16x2(p0, p1);
+        pk[x / 2] = pack2<C::F16>(p0, p1);
         rs0 += p0;
         rs1 += p1;
       }
@@ -482,8 +483,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
           }
           const int hq = hk * G + r2 % G;
           *reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.Nq + i2) * p.Hq + hq) * D + col) =
-              make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                         pack_bf16x2(f[6], f[7]));
+              make_uint4(pack2<C::F16>(f[0], f[1]), pack2<C::F16>(f[2], f[3]), pack2<C::F16>(f[4], f[5]),
+                         pack2<C::F16>(f[6], f[7]));
         }
         if (c == 0 && row_ok)
           p.lse[(static_cast<size_t>(b) * p.Hq + hk * G + rr % G) * p.Nq + i] =
@@ -560,8 +561,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
             }
             const int hq = hk * G + r2 % G;
             *reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.Nq + i2) * p.Hq + hq) * D + col) =
-                make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                           pack_bf16x2(f[6], f[7]));
+                make_uint4(pack2<C::F16>(f[0], f[1]), pack2<C::F16>(f[2], f[3]), pack2<C::F16>(f[4], f[5]),
+                           pack2<C::F16>(f[6], f[7]));
           }
         } else if (*last_flag) {
           // more partial rows than the staging buffer holds: the same merge,
@@ -610,8 +611,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
             }
             const int hq = hk * G + r2 % G;
             *reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.Nq + i2) * p.Hq + hq) * D + col) =
-                make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                           pack_bf16x2(f[6], f[7]));
+                make_uint4(pack2<C::F16>(f[0], f[1]), pack2<C::F16>(f[2], f[3]), pack2<C::F16>(f[4], f[5]),
+                           pack2<C::F16>(f[6], f[7]));
           }
         }
       }
@@ -628,8 +629,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 // sequence b goes to cache row seqlens[b] + t (rows at or past the capacity
 // Nk are dropped).  One thread per 16 bytes of a row of K and of V.
 __global__ void __launch_bounds__(256)
-    fa_kvcache_append_kernel(__nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache,
-                             const __nv_bfloat16* __restrict__ k_new, const __nv_bfloat16* __restrict__ v_new,
+    fa_kvcache_append_kernel(uint16_t* __restrict__ k_cache, uint16_t* __restrict__ v_cache,
+                             const uint16_t* __restrict__ k_new, const uint16_t* __restrict__ v_new,
                              const int* __restrict__ seqlens, int B, int n_new, int Nk, int Hkv, int d) {
   const int upr = d / 8;  // 16-byte units per row
   const long long total = static_cast<long long>(B) * n_new * Hkv * upr;

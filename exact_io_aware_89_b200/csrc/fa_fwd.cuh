@@ -49,12 +49,13 @@ struct FwdParams {
   const int* cu_q;
   const int* cu_k;
   int total_q;
-  __nv_bfloat16* o;               // O, for the plain stores of a packed sequence's last tile
+  uint16_t* o;               // O, for the plain stores of a packed sequence's last tile
   unsigned long long wait_limit_ns;
 };
 
 template <int D_, int NQT_, int BN_, int KST_, int NPOLY_ = 2, bool SPLITP_ = false>
 struct FwdCfg {
+  static constexpr bool F16 = false;  // elements are bf16 (AsF16<> flips it to fp16)
   static constexpr int D = D_, NQT = NQT_, BN = BN_, KST = KST_;
   // NQT == 2 only: P reaches the tensor core in two key halves, so the first
   // half's PV overlaps the softmax of the second (one more wait point per
@@ -153,7 +154,7 @@ __device__ __forceinline__ void fwd_exp_cols(const float* sc, uint64_t scale2, u
       p0 = ex2_approx(x0);
       p1 = ex2_approx(x1);
     }
-    pk[c / 2] = pack_bf16x2(p0, p1);
+    pk[c / 2] = pack2<C::F16>(p0, p1);
     if ((c / 2) & 1)
       acc1 = f2_add(acc1, f2_pack(p0, p1));
     else
@@ -303,8 +304,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     setmaxnreg_dec<C::REG_PRODUCER>();
     if (lane == 0 && n_kv > 0) {
-      constexpr uint32_t ID_QK = idesc_bf16_f32(128, BN, false, false);
-      constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t ID_QK = idesc_kind_f16<C::F16>(128, BN, false, false);
+      constexpr uint32_t ID_PV = idesc_kind_f16<C::F16>(128, D, false, true);
       // Descriptors are built once; every MMA only adds a compile-time offset
       // (in 16-byte units) to the start-address field.  The issuing thread
       // must stay ahead of the tensor core, so it does as little as possible
@@ -566,8 +567,8 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
         for (int u = 0; u < 8; ++u) {
           const float* f = reinterpret_cast<const float*>(ov + 8 * u);
           st_shared_v4(sQt + c * C::QCHUNK + sw128_offset(r, u),
-                       pack_bf16x2(f[0] * inv_l, f[1] * inv_l), pack_bf16x2(f[2] * inv_l, f[3] * inv_l),
-                       pack_bf16x2(f[4] * inv_l, f[5] * inv_l), pack_bf16x2(f[6] * inv_l, f[7] * inv_l));
+                       pack2<C::F16>(f[0] * inv_l, f[1] * inv_l), pack2<C::F16>(f[2] * inv_l, f[3] * inv_l),
+                       pack2<C::F16>(f[4] * inv_l, f[5] * inv_l), pack2<C::F16>(f[6] * inv_l, f[7] * inv_l));
         }
       }
       fence_proxy_async_smem();

@@ -244,12 +244,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major,
-                                                      bool b_mn_major) {
+// Instruction descriptor for kind::f16 with fp32 accumulation; A and B are
+// both bf16 (F16 false) or both fp16 (F16 true) -- never mixed.
+template <bool F16 = false>
+__host__ __device__ constexpr uint32_t idesc_kind_f16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                     // D format: f32
-         | (1u << 7)                                   // A format: bf16
-         | (1u << 10)                                  // B format: bf16
+         | ((F16 ? 0u : 1u) << 7)                      // A format: fp16 0, bf16 1
+         | ((F16 ? 0u : 1u) << 10)                     // B format: the same as A
          | (static_cast<uint32_t>(a_mn_major) << 15)   // A major
          | (static_cast<uint32_t>(b_mn_major) << 16)   // B major
          | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
@@ -338,6 +339,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// two floats to the kernel's 16-bit element type (round to nearest even)
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (F16)
+    return pack_f16x2(lo, hi);
+  else
+    return pack_bf16x2(lo, hi);
 }
 // three-input maximum (one instruction on sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

@@ -21,7 +21,8 @@
  *     lse          : [B, Hq, Nq]      fp32, natural log, scale included:
  *                    lse[b,h,i] = ln sum_j exp(scale * q_i . k_j) over visible j
  * bf16 entry points take and return __nv_bfloat16 data (passed as void*);
- * the _f32 entry points take float data.  Accumulation is fp32 throughout.
+ * the _f16 entry points the same with IEEE fp16 data; the _f32 entry points
+ * take float data.  Accumulation is fp32 throughout.
  *
  * Masking (hysenlabs page, option list and changelog v2.1 / v2.3): with
  * delta = Nk - Nq, key j is visible to query i iff
@@ -227,6 +228,38 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
                   const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q,
                   int total_k, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
                   void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * fp16 variants (hysenlabs page, requirements: fp16 and bf16 inputs): the
+ * same arguments, semantics, layouts and workspace sizes as the bf16 entry
+ * points of the same name without the suffix, with every 16-bit tensor
+ * (q, k, v, o, dO, dq, dk, dv, k_new, v_new, the caches) holding IEEE fp16
+ * instead of bf16.  Accumulation stays fp32; P and dS enter the tensor cores
+ * as fp16 (P <= 2^8 in the forward, P <= 1 in the backward, within range).
+ */
+int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+               int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+               fa_stream_t stream);
+int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
+               int d, float scale, int causal, int win_l, int win_r, void* workspace,
+               size_t workspace_bytes, fa_stream_t stream);
+int fa_fwd_varlen_f16(const void* q, const void* k, const void* v, void* o, float* lse,
+                      const int* cu_seqlens_q, const int* cu_seqlens_k, int B, int max_seqlen_q,
+                      int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d, float scale,
+                      int causal, int win_l, int win_r, fa_stream_t stream);
+int fa_bwd_varlen_f16(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                      const void* dO, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                      const int* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k, int total_q,
+                      int total_k, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                      void* workspace, size_t workspace_bytes, fa_stream_t stream);
+int fa_fwd_splitkv_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq,
+                       int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
+                       int n_splits, void* workspace, size_t workspace_bytes, fa_stream_t stream);
+int fa_fwd_kvcache_f16(const void* q, void* k_cache, void* v_cache, const void* k_new, const void* v_new,
+                       const int* cache_seqlens, void* o, float* lse, int B, int Nq, int Nk, int n_new,
+                       int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r, int n_splits,
+                       void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fp32 variants for small problems (fp32 in, fp32 out, fp32 arithmetic on the

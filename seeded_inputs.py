@@ -8,7 +8,7 @@ dtype.  Both the CUDA path and the oracle receive the same rounded values
 """
 import torch
 
-DTYPES = {"bf16": torch.bfloat16, "fp32": torch.float32, "f32": torch.float32}
+DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32, "f32": torch.float32}
 
 
 def make_inputs(B, Nq, Nk, Hq, Hkv, d, seed, dtype="bf16", with_dout=True, scale_q=1.0):

@@ -6,6 +6,7 @@ Tolerances (bf16 in, fp32 accumulation, inputs ~ N(0,1)):
   LSE max |gpu - oracle|              <= 1e-3   (-inf entries must match)
   dQ, dK, dV  ||gpu - oracle||_F / ||oracle||_F <= 2e-2
 fp32 path (CUDA-core fp32 arithmetic): 1e-4 on all three.
+fp16 inputs (the _f16 entry points) are held to the bf16 bounds.
 
 When the oracle's gradient is exactly zero (every row sees a single key, so
 P = 1 and dS = P (dP - D) = 0 exactly), a relative error is undefined; the
@@ -40,15 +41,17 @@ TOL_F32 = dict(o=1e-4, lse=1e-4, grad=1e-4)
 ZERO_ABS = 1e-3
 
 
-BF16_HALF_ULP_REL = 2.0 ** -8  # bound on bf16 rounding error relative to |x|
+BF16_HALF_ULP_REL = 2.0 ** -8   # bound on bf16 rounding error relative to |x|
+FP16_HALF_ULP_REL = 2.0 ** -11  # the same for fp16 (11 significant bits)
 
 
 def o_error(o_gpu, o_ref, dtype="bf16"):
     """Max |o_gpu - o_ref| beyond the rounding of the output format itself
-    (|o_ref| * 2^-8 for bf16 outputs; none for fp32)."""
+    (|o_ref| * 2^-8 for bf16 outputs, 2^-11 for fp16; none for fp32)."""
     diff = np.abs(np.asarray(o_gpu, dtype=np.float64) - o_ref)
-    if dtype == "bf16":
-        diff = diff - BF16_HALF_ULP_REL * np.abs(o_ref)
+    if dtype in ("bf16", "fp16"):
+        rel = BF16_HALF_ULP_REL if dtype == "bf16" else FP16_HALF_ULP_REL
+        diff = diff - rel * np.abs(o_ref)
     return float(diff.max()) if diff.size else 0.0
 
 
@@ -86,7 +89,7 @@ def run_case(B, Nq, Nk, Hq, Hkv, d, causal=False, window=(-1, -1), seed=0, dtype
     """Full comparison against the full oracle (sizes the oracle finishes in seconds)."""
     inp = make_inputs(B, Nq, Nk, Hq, Hkv, d, seed, dtype=dtype, scale_q=scale_q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    tol = TOL_BF16 if dtype == "bf16" else TOL_F32
+    tol = TOL_BF16 if dtype in ("bf16", "fp16") else TOL_F32
     g = gpu_run(inp, scale, causal, window, backward)
     f64 = {n: t.double().numpy() for n, t in inp.items()}
     o_ref, lse_ref = oracle.attn_fwd(f64["q"], f64["k"], f64["v"], scale=scale, causal=causal,

@@ -26,7 +26,8 @@ def test_header_declares_the_expected_entry_points():
     assert declared_functions() == sorted([
         "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
         "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
-        "fa_fwd_kvcache_workspace_size", "fa_fwd_varlen", "fa_bwd_varlen",
+        "fa_fwd_kvcache_workspace_size", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_f16",
+        "fa_bwd_f16", "fa_fwd_varlen_f16", "fa_bwd_varlen_f16", "fa_fwd_splitkv_f16", "fa_fwd_kvcache_f16",
         "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
 
 
@@ -247,3 +248,12 @@ def test_bwd_varlen_workspace_and_head_dim():
     assert _bwd_varlen(wsb=need - 4) == WORKSPACE
     assert _bwd_varlen(ws=0) == WORKSPACE
     assert _bwd_varlen(d=96) == UNSUPPORTED
+
+
+def test_fp16_entry_points_check_arguments_like_bf16():
+    assert fa.fa_fwd_f16(0, FAKE, FAKE, FAKE, FAKE, 1, 128, 128, 2, 2, 64, 0.125, 0, -1, -1,
+                         None) == INVALID
+    assert fa.fa_fwd_f16(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 128, 2, 2, 96, 0.125, 0, -1, -1,
+                         None) == UNSUPPORTED
+    assert fa.fa_bwd_f16(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 128, 2, 2,
+                         64, 0.125, 0, -1, -1, 0, 0, None) == WORKSPACE
