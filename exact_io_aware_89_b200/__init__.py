@@ -28,7 +28,8 @@ __all__ = [
     "fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_bwd_workspace_size",
     "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
     "fa_fwd_kvcache_workspace_size", "fa_fwd_f16", "fa_bwd_f16", "fa_fwd_varlen_f16",
-    "fa_bwd_varlen_f16", "fa_fwd_splitkv_f16", "fa_fwd_kvcache_f16",
+    "fa_bwd_varlen_f16", "fa_fwd_splitkv_f16", "fa_fwd_kvcache_f16", "fa_fwd_blocksparse",
+    "fa_fwd_blocksparse_f16", "attention_forward_blocksparse",
     "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
     "KERNEL_KINDS", "attention_forward", "attention_backward", "attention_forward_splitkv",
     "attention_forward_kvcache", "attention_forward_varlen", "attention_backward_varlen",
@@ -89,8 +90,11 @@ def load_library():
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_trace_enable.argtypes = [i]
     lib.fa_trace_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_longlong)]
+    ll = ctypes.c_longlong
+    lib.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, ll, ll, i, i, i, i, i, i, f, i, i, i, vp]
+    lib.fa_fwd_blocksparse.restype = i
     for base in ("fa_fwd", "fa_bwd", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_splitkv",
-                 "fa_fwd_kvcache"):
+                 "fa_fwd_kvcache", "fa_fwd_blocksparse"):
         getattr(lib, base + "_f16").argtypes = getattr(lib, base).argtypes
         getattr(lib, base + "_f16").restype = i
     for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache", "fa_fwd_varlen", "fa_bwd_varlen",
@@ -192,6 +196,15 @@ fa_fwd_varlen_f16 = _f16_twin("fa_fwd_varlen_f16")
 fa_bwd_varlen_f16 = _f16_twin("fa_bwd_varlen_f16")
 fa_fwd_splitkv_f16 = _f16_twin("fa_fwd_splitkv_f16")
 fa_fwd_kvcache_f16 = _f16_twin("fa_fwd_kvcache_f16")
+fa_fwd_blocksparse_f16 = _f16_twin("fa_fwd_blocksparse_f16")
+
+
+def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, mask_stride_b, mask_stride_h, B, Nq, Nk, Hq,
+                       Hkv, d, scale, causal, win_l, win_r, stream):
+    """Block-sparse forward: 128 x 128 tiles that block_mask marks zero are skipped."""
+    return load_library().fa_fwd_blocksparse(q, k, v, o, lse, block_mask, mask_stride_b,
+                                             mask_stride_h, B, Nq, Nk, Hq, Hkv, d, scale, causal,
+                                             win_l, win_r, stream)
 
 
 def fa_bwd_workspace_size(B, Nq, Hq, d):
@@ -300,6 +313,42 @@ def attention_forward_splitkv(q, k, v, scale=None, causal=False, window=(-1, -1)
                           B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, int(n_splits),
                           workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                           _stream()))
+    return o, lse
+
+
+BLOCK_SPARSE_TILE = 128
+
+
+def attention_forward_blocksparse(q, k, v, block_mask, scale=None, causal=False, window=(-1, -1),
+                                  out=None, lse=None):
+    """O, LSE with 128 x 128 (query block, key block) tiles left out where
+    block_mask is zero.  q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] bf16 or fp16;
+    block_mask: uint8 (or bool) CUDA tensor [B, Hq, ceil(Nq/128), ceil(Nk/128)]
+    whose batch / head dims may be broadcast (size 1, or expanded with stride 0)."""
+    import torch
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    if q.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("fa_fwd_blocksparse takes bf16 or fp16 tensors")
+    nqb, nkb = -(-Nq // BLOCK_SPARSE_TILE), -(-Nk // BLOCK_SPARSE_TILE)
+    m = block_mask
+    if m.dtype == torch.bool:
+        m = m.to(torch.uint8)
+    if m.dtype != torch.uint8 or not m.is_cuda or m.dim() != 4:
+        raise ValueError("block_mask must be a 4-D uint8 or bool CUDA tensor")
+    if m.shape[2:] != (nqb, nkb) or m.shape[0] not in (1, B) or m.shape[1] not in (1, Hq):
+        raise ValueError("block_mask must be [B or 1, Hq or 1, %d, %d]" % (nqb, nkb))
+    if m.stride(3) != 1 or m.stride(2) != nkb:
+        m = m.contiguous()
+    sb = 0 if m.shape[0] == 1 else m.stride(0)
+    sh = 0 if m.shape[1] == 1 else m.stride(1)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    fn = fa_fwd_blocksparse if q.dtype == torch.bfloat16 else fa_fwd_blocksparse_f16
+    _check(fn.__name__, fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           m.data_ptr(), sb, sh, B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr,
+                           _stream()))
     return o, lse
 
 

@@ -158,6 +158,9 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.cu_k = nullptr;
   p.total_q = 0;
   p.o = static_cast<uint16_t*>(o);
+  p.bmask = nullptr;
+  p.bm_sb = p.bm_sh = 0;
+  p.bm_cols = 0;
   p.wait_limit_ns = kWaitLimitNs;
   auto kern = fa_fwd_kernel<C>;
   if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
@@ -165,6 +168,50 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   {
     TraceScope tr(FA_KERNEL_FWD, stream);
     kern<<<static_cast<unsigned>(grid), C::NTHREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, to, p);
+  }
+  return launch_status();
+}
+
+// Block-sparse forward: the dense launch plus the block mask; each CTA keeps
+// its list of key tiles (4 bytes each) in shared memory after the fixed part.
+constexpr int kBlockSparseTile = 128;
+
+template <class C>
+int launch_fwd_bs(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq, int Nk,
+                  int Hq, int Hkv, float scale, const MaskSpec& mask, const uint8_t* bmask, long long sb,
+                  long long sh, cudaStream_t stream) {
+  static int attr_done[kMaxDevices] = {0};
+  const long long list_bytes = 4ll * ((Nk + C::BN - 1) / C::BN + 1);
+  const long long smem = C::SMEM_BYTES + list_bytes;
+  if (smem > 232448) return FA_ERR_UNSUPPORTED;  // more key tiles than the list has room for
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_bnhd(&tq, q, B, Nq, Hq, C::D, C::BM, tma_type(C::F16)) ||
+      !encode_bnhd(&tk, k, B, Nk, Hkv, C::D, C::BN, tma_type(C::F16)) ||
+      !encode_bnhd(&tv, v, B, Nk, Hkv, C::D, C::BN, tma_type(C::F16)) ||
+      !encode_bnhd(&to, o, B, Nq, Hq, C::D, C::BM, tma_type(C::F16)))
+    return FA_ERR_CUDA;
+  FwdParams p;
+  p.B = B; p.Nq = Nq; p.Nk = Nk; p.Hq = Hq; p.Hkv = Hkv; p.group = Hq / Hkv;
+  p.scale_log2 = scale * kLog2e;
+  p.mask = mask;
+  p.n_qgroups = (Nq + C::NQT * C::BM - 1) / (C::NQT * C::BM);
+  p.head_chunk = head_chunk(B * Hq, 4ll * Nk * C::D);
+  p.lse = lse;
+  p.cu_q = nullptr;
+  p.cu_k = nullptr;
+  p.total_q = 0;
+  p.o = static_cast<uint16_t*>(o);
+  p.bmask = bmask;
+  p.bm_sb = sb;
+  p.bm_sh = sh;
+  p.bm_cols = (Nk + kBlockSparseTile - 1) / kBlockSparseTile;
+  p.wait_limit_ns = kWaitLimitNs;
+  auto kern = fa_fwd_kernel<C, false, true>;
+  if (smem_attr_once(kern, 232448, attr_done) != cudaSuccess) return FA_ERR_CUDA;
+  const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
+  {
+    TraceScope tr(FA_KERNEL_FWD, stream);
+    kern<<<static_cast<unsigned>(grid), C::NTHREADS, static_cast<size_t>(smem), stream>>>(tq, tk, tv, to, p);
   }
   return launch_status();
 }
@@ -191,6 +238,9 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
   p.cu_k = cu_k;
   p.total_q = total_q;
   p.o = static_cast<uint16_t*>(o);
+  p.bmask = nullptr;
+  p.bm_sb = p.bm_sh = 0;
+  p.bm_cols = 0;
   p.wait_limit_ns = kWaitLimitNs;
   auto kern = fa_fwd_kernel<C, true>;
   if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
@@ -645,6 +695,33 @@ int fa_bwd_varlen_impl(const void* q, const void* k, const void* v, const void* 
   }
 }
 
+template <bool F16>
+int fa_fwd_blocksparse_impl(const void* q, const void* k, const void* v, void* o, float* lse,
+                            const unsigned char* block_mask, long long mask_stride_b,
+                            long long mask_stride_h, int B, int Nq, int Nk, int Hq, int Hkv, int d,
+                            float scale, int causal, int win_l, int win_r, fa_stream_t stream) {
+  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse) || block_mask == nullptr) return FA_ERR_INVALID_ARG;
+  if (mask_stride_b < 0 || mask_stride_h < 0) return FA_ERR_INVALID_ARG;
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint8_t* bm = reinterpret_cast<const uint8_t*>(block_mask);
+  switch (d) {
+    case 64:
+      return launch_fwd_bs<Ty<F16, Fwd64>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, bm, mask_stride_b,
+                                           mask_stride_h, s);
+    case 128:
+      return launch_fwd_bs<Ty<F16, Fwd128>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, bm, mask_stride_b,
+                                            mask_stride_h, s);
+    case 256:
+      return launch_fwd_bs<Ty<F16, Fwd256>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, bm, mask_stride_b,
+                                            mask_stride_h, s);
+    default:
+      return FA_ERR_UNSUPPORTED;
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -784,6 +861,22 @@ int fa_bwd_varlen_f16(const void* q, const void* k, const void* v, const void* o
                   int total_k, int Hq, int Hkv, int d, float scale, int causal, int win_l, int win_r,
                   void* workspace, size_t workspace_bytes_, fa_stream_t stream) {
   return fa_bwd_varlen_impl<true>(q, k, v, o, lse, dO, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, B, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq, Hkv, d, scale, causal, win_l, win_r, workspace, workspace_bytes_, stream);
+}
+
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                       const unsigned char* block_mask, long long mask_stride_b, long long mask_stride_h,
+                       int B, int Nq, int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l,
+                       int win_r, fa_stream_t stream) {
+  return fa_fwd_blocksparse_impl<false>(q, k, v, o, lse, block_mask, mask_stride_b, mask_stride_h, B, Nq, Nk, Hq,
+                                        Hkv, d, scale, causal, win_l, win_r, stream);
+}
+
+int fa_fwd_blocksparse_f16(const void* q, const void* k, const void* v, void* o, float* lse,
+                           const unsigned char* block_mask, long long mask_stride_b, long long mask_stride_h,
+                           int B, int Nq, int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l,
+                           int win_r, fa_stream_t stream) {
+  return fa_fwd_blocksparse_impl<true>(q, k, v, o, lse, block_mask, mask_stride_b, mask_stride_h, B, Nq, Nk, Hq,
+                                       Hkv, d, scale, causal, win_l, win_r, stream);
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Nq,

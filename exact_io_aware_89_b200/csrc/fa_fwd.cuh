@@ -50,6 +50,12 @@ struct FwdParams {
   const int* cu_k;
   int total_q;
   uint16_t* o;               // O, for the plain stores of a packed sequence's last tile
+  // block-sparse attention (BS kernels): a byte per 128 x 128 (query block,
+  // key block) of batch b, query head h at bmask + b * bm_sb + h * bm_sh,
+  // rows of bm_cols key blocks; zero = the block is skipped
+  const uint8_t* bmask;
+  long long bm_sb, bm_sh;
+  int bm_cols;
   unsigned long long wait_limit_ns;
 };
 
@@ -162,9 +168,9 @@ __device__ __forceinline__ void fwd_exp_cols(const float* sc, uint64_t scale2, u
   }
 }
 
-// VL: packed variable-length sequences (FwdParams::cu_q / cu_k); the dense
-// instantiation compiles without any of that code.
-template <class C, bool VL = false>
+// VL: packed variable-length sequences (FwdParams::cu_q / cu_k); BS: a block
+// mask (FwdParams::bmask).  The dense instantiation compiles without either.
+template <class C, bool VL = false, bool BS = false>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -214,12 +220,49 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int r_last = min(nq - 1, r0 + NQT * BM - 1);
   const int key_lo = mask.lo(r0), key_hi = mask.hi(r_last);
   const int j_begin = key_lo / BN;
-  const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
+  int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
+
+  // Block-sparse: the TMA warp lists the key tiles of that range whose mask
+  // block is set for either Q tile (bit 30 + t: set for Q tile t), compacted
+  // with warp ballots, before the block-wide sync; every role then walks the
+  // list instead of the range.
+  uint32_t* tile_list = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 16);
+  volatile int* list_count = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  if constexpr (BS) {
+    if (warp == C::TMA_WARP) {
+      const uint8_t* m0 = p.bmask + b * p.bm_sb + h * p.bm_sh + static_cast<long long>(r0 / 128) * p.bm_cols;
+      const bool two = NQT == 2 && r0 + BM < nq;
+      int cnt = 0;
+      for (int c0 = 0; c0 < n_kv; c0 += 32) {
+        const int it = c0 + lane;
+        uint32_t a0 = 0, a1 = 0;
+        if (it < n_kv) {
+          const int blk = ((j_begin + it) * BN) / 128;
+          a0 = __ldg(m0 + blk) != 0;
+          if (two) a1 = __ldg(m0 + p.bm_cols + blk) != 0;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, (a0 | a1) != 0);
+        if (a0 | a1)
+          tile_list[cnt + __popc(bal & ((1u << lane) - 1u))] =
+              static_cast<uint32_t>(j_begin + it) | (a0 << 30) | (a1 << 31);
+        cnt += __popc(bal);
+      }
+      n_kv = cnt;
+      if (lane == 0) *list_count = cnt;
+      __syncwarp();
+    }
+  }
+  auto tile_of = [&](int it) {
+    if constexpr (BS)
+      return static_cast<int>(tile_list[it] & 0x3fffffffu);
+    else
+      return j_begin + it;
+  };
 
   // Copies of key tile `it` into ring stage it % KST (K and V on one barrier
   // with two Q tiles, on their own barriers with one)
   auto load_k = [&](int it) {
-    const int s = it % KST, krow = k_off + (j_begin + it) * BN;
+    const int s = it % KST, krow = k_off + tile_of(it) * BN;
     uint64_t* bar = &k_full[s];
     mbar_expect_tx(bar, (NQT == 2 ? 2 : 1) * C::KTILE);
     for (int c = 0; c < C::NCHUNK; ++c) {
@@ -228,7 +271,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     }
   };
   auto load_v = [&](int it) {  // NQT == 1 only
-    const int s = it % KST, krow = k_off + (j_begin + it) * BN;
+    const int s = it % KST, krow = k_off + tile_of(it) * BN;
     mbar_expect_tx(&v_full[s], C::KTILE);
     for (int c = 0; c < C::NCHUNK; ++c)
       tma_load_4d(sV + s * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[s], c * 64, hk, krow, tb);
@@ -273,6 +316,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if constexpr (BS) n_kv = *list_count;
 
   if (warp == C::TMA_WARP) {
     // ------------------------------------------------------------ producer
@@ -443,13 +487,20 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 #pragma unroll
       for (int cc = 0; cc < BN / 32; ++cc) tmem_ld_wait_x32(&sv[cc * 32]);
       float* sc = reinterpret_cast<float*>(sv);
-      const int k0 = (j_begin + it) * BN;
-      const bool edge = k0 < lo || k0 + BN - 1 > hi;
+      const int k0 = tile_of(it) * BN;
+      int tlo = lo, thi = hi;
+      if constexpr (BS) {
+        if (!((tile_list[it] >> (30 + t)) & 1u)) {  // block off for this Q tile: no key visible
+          tlo = 1;
+          thi = 0;
+        }
+      }
+      const bool edge = k0 < tlo || k0 + BN - 1 > thi;
       if (edge) {
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
           const int key = k0 + c;
-          if (key < lo || key > hi) sc[c] = -INFINITY;
+          if (key < tlo || key > thi) sc[c] = -INFINITY;
         }
       }
       float mx0 = fmaxf(sc[0], sc[1]), mx1 = fmaxf(sc[2], sc[3]);

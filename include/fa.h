@@ -230,6 +230,30 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, co
                   void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Block-sparse forward (abeam.tech FlashAttention summary, the block-sparse
+ * extension): fa_fwd with the 128 x 128 (query block, key block) tiles that
+ * block_mask marks zero left out -- their keys are invisible to their query
+ * rows, on top of the causal / window masks -- and the kernel skips them.
+ *   block_mask : uint8, device; for batch b and query head h the mask is
+ *                block_mask + b * mask_stride_b + h * mask_stride_h, a
+ *                row-major [ceil(Nq / 128)][ceil(Nk / 128)] array, nonzero =
+ *                computed.  Strides are in bytes (elements); 0 shares one
+ *                mask across batches or heads.
+ * Rows that see no key (every block of their row off) get O = 0 and
+ * LSE = -inf.  FA_ERR_UNSUPPORTED also when Nk needs more than the shared
+ * memory left for the CTA's key-tile list (Nk in the hundreds of
+ * thousands).  fa_fwd_blocksparse_f16 takes fp16 tensors.
+ */
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                       const unsigned char* block_mask, long long mask_stride_b, long long mask_stride_h,
+                       int B, int Nq, int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l,
+                       int win_r, fa_stream_t stream);
+int fa_fwd_blocksparse_f16(const void* q, const void* k, const void* v, void* o, float* lse,
+                           const unsigned char* block_mask, long long mask_stride_b, long long mask_stride_h,
+                           int B, int Nq, int Nk, int Hq, int Hkv, int d, float scale, int causal, int win_l,
+                           int win_r, fa_stream_t stream);
+
+/*
  * fp16 variants (hysenlabs page, requirements: fp16 and bf16 inputs): the
  * same arguments, semantics, layouts and workspace sizes as the bf16 entry
  * points of the same name without the suffix, with every 16-bit tensor

@@ -168,6 +168,49 @@ def attn_bwd_varlen(q, k, v, dout, cu_q, cu_k, scale=None, causal=False, window=
     return dq, dk, dv
 
 
+def attn_fwd_blockmask(q, k, v, block_mask, block=128, scale=None, causal=False,
+                       window=(-1, -1)):
+    """Block-sparse attention (abeam.tech FlashAttention summary, the
+    block-sparse extension): the definition of attn_fwd with key j also
+    hidden from query i when block_mask[b, h, i // block, j // block] is
+    zero.  q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]; block_mask broadcastable to
+    [B, Hq, ceil(Nq/block), ceil(Nk/block)].  Plain numpy in fp64, every
+    (b, h) materialising its Nq x Nk scores -- for small problems only.
+    Rows that see no key: O = 0, LSE = -inf."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    G = Hq // Hkv
+    nqb, nkb = -(-Nq // block), -(-Nk // block)
+    bm = np.broadcast_to(np.asarray(block_mask) != 0, (B, Hq, nqb, nkb))
+    i = np.arange(Nq)[:, None]
+    j = np.arange(Nk)[None, :]
+    delta = Nk - Nq
+    wl, wr = window if window is not None else (-1, -1)
+    wr = 0 if causal else wr
+    vis = np.ones((Nq, Nk), dtype=bool)
+    if wr >= 0:
+        vis &= j <= i + delta + wr
+    if wl >= 0:
+        vis &= j >= i + delta - wl
+    o = np.zeros((B, Nq, Hq, d))
+    lse = np.full((B, Hq, Nq), -np.inf)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            blk = np.repeat(np.repeat(bm[b, h], block, axis=0), block, axis=1)[:Nq, :Nk]
+            m = vis & blk
+            s = scale * (q[b, :, h, :] @ k[b, :, hk, :].T)
+            s = np.where(m, s, -np.inf)
+            mx = s.max(axis=1)
+            live = np.isfinite(mx)
+            p = np.where(m, np.exp(s - np.where(live, mx, 0.0)[:, None]), 0.0)
+            l = p.sum(axis=1)
+            o[b, live, h, :] = (p[live] @ v[b, :, hk, :]) / l[live, None]
+            lse[b, h, live] = mx[live] + np.log(l[live])
+    return o, lse
+
+
 def merge_partials(o_parts, lse_parts):
     """Merge attention results computed over disjoint key subsets.
 

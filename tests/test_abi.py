@@ -28,6 +28,7 @@ def test_header_declares_the_expected_entry_points():
         "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
         "fa_fwd_kvcache_workspace_size", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_f16",
         "fa_bwd_f16", "fa_fwd_varlen_f16", "fa_bwd_varlen_f16", "fa_fwd_splitkv_f16", "fa_fwd_kvcache_f16",
+        "fa_fwd_blocksparse", "fa_fwd_blocksparse_f16",
         "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
 
 
@@ -257,3 +258,18 @@ def test_fp16_entry_points_check_arguments_like_bf16():
                          None) == UNSUPPORTED
     assert fa.fa_bwd_f16(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 128, 128, 2, 2,
                          64, 0.125, 0, -1, -1, 0, 0, None) == WORKSPACE
+
+
+def test_blocksparse_rejects_invalid_arguments():
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, m=FAKE, sb=0, sh=0, B=1, Nq=256, Nk=256,
+                 Hq=2, Hkv=2, d=128, scale=0.1, causal=0, wl=-1, wr=-1)
+        a.update(kw)
+        return fa.fa_fwd_blocksparse(a["q"], a["k"], a["v"], a["o"], a["lse"], a["m"], a["sb"],
+                                     a["sh"], a["B"], a["Nq"], a["Nk"], a["Hq"], a["Hkv"], a["d"],
+                                     a["scale"], a["causal"], a["wl"], a["wr"], None)
+    assert call(m=0) == INVALID
+    assert call(sb=-1) == INVALID
+    assert call(q=MISALIGNED) == INVALID
+    assert call(Hq=3) == INVALID
+    assert call(d=96) == UNSUPPORTED

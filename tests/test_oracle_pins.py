@@ -419,3 +419,49 @@ def test_varlen_gradients_of_equal_lengths_are_the_batched_gradients():
     ref = oracle.attn_bwd(q, k, v, do, causal=True, window=(3, -1))
     for a, r in zip(g, ref):
         assert np.abs(a - r.reshape(a.shape)).max() < 1e-14
+
+
+# ------------------------------------------------------------ block-sparse
+
+@pytest.mark.parametrize("causal,window", [(False, (-1, -1)), (True, (-1, -1)), (False, (5, 3))])
+def test_blockmask_all_ones_is_the_dense_attention(causal, window):
+    rng = np.random.default_rng(60)
+    q = rng.standard_normal((2, 13, 4, 6))
+    k = rng.standard_normal((2, 17, 2, 6))
+    v = rng.standard_normal((2, 17, 2, 6))
+    o, lse = oracle.attn_fwd_blockmask(q, k, v, np.ones((1, 1, 4, 5)), block=4, causal=causal,
+                                       window=window)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, causal=causal, window=window)
+    assert np.abs(o - o_ref).max() < 1e-12
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(fin, np.isfinite(lse)) and np.abs(lse[fin] - lse_ref[fin]).max() < 1e-12
+
+
+def test_blockmask_key_blocks_off_equals_dropping_those_keys():
+    """Non-causal: a key block off for every query block is the attention over
+    the remaining keys (the C oracle on the sliced keys)."""
+    rng = np.random.default_rng(61)
+    q = rng.standard_normal((1, 10, 2, 5))
+    k = rng.standard_normal((1, 22, 1, 5))
+    v = rng.standard_normal((1, 22, 1, 5))
+    bm = np.ones((1, 1, 3, 6))
+    bm[..., 1] = 0
+    bm[..., 4] = 0
+    o, lse = oracle.attn_fwd_blockmask(q, k, v, bm, block=4)
+    keep = np.r_[0:4, 8:16, 20:22]
+    o_ref, lse_ref = oracle.attn_fwd(q, k[:, keep], v[:, keep])
+    assert np.abs(o - o_ref).max() < 1e-12 and np.abs(lse - lse_ref).max() < 1e-12
+
+
+def test_blockmask_query_block_off_gives_empty_rows_and_heads_differ():
+    rng = np.random.default_rng(62)
+    q = rng.standard_normal((1, 8, 2, 3))
+    k = rng.standard_normal((1, 8, 2, 3))
+    v = rng.standard_normal((1, 8, 2, 3))
+    bm = np.ones((1, 2, 2, 2))
+    bm[0, 1, 0, :] = 0          # head 1: rows 0-3 see nothing
+    o, lse = oracle.attn_fwd_blockmask(q, k, v, bm, block=4)
+    assert np.all(o[0, :4, 1] == 0) and np.all(np.isneginf(lse[0, 1, :4]))
+    o_ref, _ = oracle.attn_fwd(q, k, v)
+    assert np.abs(o[0, :, 0] - o_ref[0, :, 0]).max() < 1e-12
+    assert np.abs(o[0, 4:, 1] - o_ref[0, 4:, 1]).max() < 1e-12
