@@ -29,7 +29,8 @@ __all__ = [
     "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
     "fa_fwd_kvcache_workspace_size", "fa_fwd_f16", "fa_bwd_f16", "fa_fwd_varlen_f16",
     "fa_bwd_varlen_f16", "fa_fwd_splitkv_f16", "fa_fwd_kvcache_f16", "fa_fwd_blocksparse",
-    "fa_fwd_blocksparse_f16", "attention_forward_blocksparse",
+    "fa_fwd_blocksparse_f16", "attention_forward_blocksparse", "fa_bwd_blocksparse",
+    "fa_bwd_blocksparse_f16", "attention_backward_blocksparse",
     "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
     "KERNEL_KINDS", "attention_forward", "attention_backward", "attention_forward_splitkv",
     "attention_forward_kvcache", "attention_forward_varlen", "attention_backward_varlen",
@@ -93,8 +94,11 @@ def load_library():
     ll = ctypes.c_longlong
     lib.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, ll, ll, i, i, i, i, i, i, f, i, i, i, vp]
     lib.fa_fwd_blocksparse.restype = i
+    lib.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ll, ll, i, i, i, i, i,
+                                       i, f, i, i, i, vp, sz, vp]
+    lib.fa_bwd_blocksparse.restype = i
     for base in ("fa_fwd", "fa_bwd", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_splitkv",
-                 "fa_fwd_kvcache", "fa_fwd_blocksparse"):
+                 "fa_fwd_kvcache", "fa_fwd_blocksparse", "fa_bwd_blocksparse"):
         getattr(lib, base + "_f16").argtypes = getattr(lib, base).argtypes
         getattr(lib, base + "_f16").restype = i
     for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache", "fa_fwd_varlen", "fa_bwd_varlen",
@@ -197,6 +201,17 @@ fa_bwd_varlen_f16 = _f16_twin("fa_bwd_varlen_f16")
 fa_fwd_splitkv_f16 = _f16_twin("fa_fwd_splitkv_f16")
 fa_fwd_kvcache_f16 = _f16_twin("fa_fwd_kvcache_f16")
 fa_fwd_blocksparse_f16 = _f16_twin("fa_fwd_blocksparse_f16")
+fa_bwd_blocksparse_f16 = _f16_twin("fa_bwd_blocksparse_f16")
+
+
+def fa_bwd_blocksparse(q, k, v, o, lse, dO, dq, dk, dv, block_mask, mask_stride_b, mask_stride_h,
+                       B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, workspace,
+                       workspace_bytes, stream):
+    """Gradients of fa_fwd_blocksparse with the same block mask."""
+    return load_library().fa_bwd_blocksparse(q, k, v, o, lse, dO, dq, dk, dv, block_mask,
+                                             mask_stride_b, mask_stride_h, B, Nq, Nk, Hq, Hkv, d,
+                                             scale, causal, win_l, win_r, workspace,
+                                             workspace_bytes, stream)
 
 
 def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, mask_stride_b, mask_stride_h, B, Nq, Nk, Hq,
@@ -319,18 +334,10 @@ def attention_forward_splitkv(q, k, v, scale=None, causal=False, window=(-1, -1)
 BLOCK_SPARSE_TILE = 128
 
 
-def attention_forward_blocksparse(q, k, v, block_mask, scale=None, causal=False, window=(-1, -1),
-                                  out=None, lse=None):
-    """O, LSE with 128 x 128 (query block, key block) tiles left out where
-    block_mask is zero.  q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] bf16 or fp16;
-    block_mask: uint8 (or bool) CUDA tensor [B, Hq, ceil(Nq/128), ceil(Nk/128)]
-    whose batch / head dims may be broadcast (size 1, or expanded with stride 0)."""
+def _block_mask_arg(m, B, Hq, Nq, Nk):
+    """(tensor, batch stride, head stride) of a block mask for the C ABI."""
     import torch
-    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
-    if q.dtype not in (torch.bfloat16, torch.float16):
-        raise ValueError("fa_fwd_blocksparse takes bf16 or fp16 tensors")
     nqb, nkb = -(-Nq // BLOCK_SPARSE_TILE), -(-Nk // BLOCK_SPARSE_TILE)
-    m = block_mask
     if m.dtype == torch.bool:
         m = m.to(torch.uint8)
     if m.dtype != torch.uint8 or not m.is_cuda or m.dim() != 4:
@@ -341,6 +348,44 @@ def attention_forward_blocksparse(q, k, v, block_mask, scale=None, causal=False,
         m = m.contiguous()
     sb = 0 if m.shape[0] == 1 else m.stride(0)
     sh = 0 if m.shape[1] == 1 else m.stride(1)
+    return m, sb, sh
+
+
+def attention_backward_blocksparse(q, k, v, o, lse, do, block_mask, scale=None, causal=False,
+                                   window=(-1, -1), dq=None, dk=None, dv=None, workspace=None):
+    """dQ, dK, dV of attention_forward_blocksparse (same block mask)."""
+    import torch
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    if q.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("fa_bwd_blocksparse takes bf16 or fp16 tensors")
+    m, sb, sh = _block_mask_arg(block_mask, B, Hq, Nq, Nk)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    c, wl, wr = _window(causal, window)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    wsb = fa_bwd_workspace_size(B, Nq, Hq, d)
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 16), dtype=torch.uint8, device=q.device)
+    fn = fa_bwd_blocksparse if q.dtype == torch.bfloat16 else fa_bwd_blocksparse_f16
+    _check(fn.__name__, fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                           do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), m.data_ptr(),
+                           sb, sh, B, Nq, Nk, Hq, Hkv, d, scale, c, wl, wr, workspace.data_ptr(),
+                           workspace.numel() * workspace.element_size(), _stream()))
+    return dq, dk, dv
+
+
+def attention_forward_blocksparse(q, k, v, block_mask, scale=None, causal=False, window=(-1, -1),
+                                  out=None, lse=None):
+    """O, LSE with 128 x 128 (query block, key block) tiles left out where
+    block_mask is zero.  q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d] bf16 or fp16;
+    block_mask: uint8 (or bool) CUDA tensor [B, Hq, ceil(Nq/128), ceil(Nk/128)]
+    whose batch / head dims may be broadcast (size 1, or expanded with stride 0)."""
+    import torch
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    if q.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("fa_fwd_blocksparse takes bf16 or fp16 tensors")
+    m, sb, sh = _block_mask_arg(block_mask, B, Hq, Nq, Nk)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     c, wl, wr = _window(causal, window)
     o = torch.empty_like(q) if out is None else out

@@ -85,6 +85,9 @@ constexpr int kMaxDecodeSplits = 4096;
 
 constexpr int kMaxDevices = 64;
 
+// block-sparse masks are over tiles of 128 query rows x 128 keys
+constexpr int kBlockSparseTile = 128;
+
 // a configuration with bf16 elements (F16 false) or fp16 elements
 template <bool F16, class C>
 using Ty = std::conditional_t<F16, AsF16<C>, C>;
@@ -174,7 +177,6 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 
 // Block-sparse forward: the dense launch plus the block mask; each CTA keeps
 // its list of key tiles (4 bytes each) in shared memory after the fixed part.
-constexpr int kBlockSparseTile = 128;
 
 template <class C>
 int launch_fwd_bs(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Nq, int Nk,
@@ -264,12 +266,25 @@ struct Varlen {
 // Dense (VL false): B batches of Nq / Nk rows.  Packed (VL true, vl set): B
 // sequences of at most Nq / Nk rows in one-batch tensors of vl.total_q /
 // vl.total_k rows.
-template <class CQ, class CKV, bool VL = false>
+// Block mask of a block-sparse backward call (null when dense).
+struct BlockMask {
+  const uint8_t* mask = nullptr;
+  long long sb = 0, sh = 0;
+};
+
+template <class CQ, class CKV, bool VL = false, bool BS = false>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
-               float scale, const MaskSpec& mask, float* ws, cudaStream_t stream, const Varlen& vl = Varlen()) {
+               float scale, const MaskSpec& mask, float* ws, cudaStream_t stream, const Varlen& vl = Varlen(),
+               const BlockMask& bm = BlockMask()) {
   static int attr_dq[kMaxDevices] = {0};
   static int attr_kv[kMaxDevices] = {0};
+  // block-sparse: each CTA's list of key tiles (dQ) or steps (dK/dV), 4 bytes
+  // an entry, after the fixed shared memory
+  const long long dq_smem = CQ::SMEM_BYTES + (BS ? 4ll * ((Nk + CQ::BN - 1) / CQ::BN + 1) : 0);
+  const long long kv_smem =
+      CKV::SMEM_BYTES + (BS ? 4ll * (Hq / Hkv) * ((Nq + CKV::BM - 1) / CKV::BM + 1) : 0);
+  if (dq_smem > 232448 || kv_smem > 232448) return FA_ERR_UNSUPPORTED;
   constexpr int D = CQ::D;
   const int Nq_pad = pad_rows(Nq);
   const long long rows_pad = static_cast<long long>(B) * Hq * Nq_pad;
@@ -302,6 +317,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.dq = static_cast<uint16_t*>(dq);
   p.dk = static_cast<uint16_t*>(dk);
   p.dv = static_cast<uint16_t*>(dv);
+  p.bmask = bm.mask;
+  p.bm_sb = bm.sb;
+  p.bm_sh = bm.sh;
+  p.bm_cols = (Nk + kBlockSparseTile - 1) / kBlockSparseTile;
   p.wait_limit_ns = kWaitLimitNs;
   // tensor-map shapes: dense [B, N, H, d]; packed [1, total, H, d]
   const bool packed = VL;
@@ -313,16 +332,19 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         !encode_bnhd(&tdq, dq, mB, mNq, Hq, D, CQ::BM, tma_type(CQ::F16)))
       return FA_ERR_CUDA;
     const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
+    const int attr_bytes = BS ? 232448 : CQ::SMEM_BYTES;
     if constexpr (CQ::ONE_TILE) {
-      auto kern = fa_bwd_dq2_kernel<CQ, VL>;
-      if (smem_attr_once(kern, CQ::SMEM_BYTES, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
+      auto kern = fa_bwd_dq2_kernel<CQ, VL, BS>;
+      if (smem_attr_once(kern, attr_bytes, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
       TraceScope tr(FA_KERNEL_BWD_DQ, stream);
-      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
+      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, static_cast<size_t>(dq_smem), stream>>>(tq, tk, tv, tdo,
+                                                                                              tdq, p);
     } else {
-      auto kern = fa_bwd_dq_kernel<CQ, VL>;
-      if (smem_attr_once(kern, CQ::SMEM_BYTES, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
+      auto kern = fa_bwd_dq_kernel<CQ, VL, BS>;
+      if (smem_attr_once(kern, attr_bytes, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
       TraceScope tr(FA_KERNEL_BWD_DQ, stream);
-      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, CQ::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
+      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, static_cast<size_t>(dq_smem), stream>>>(tq, tk, tv, tdo,
+                                                                                              tdq, p);
     }
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
@@ -332,11 +354,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         !encode_bnhd(&tv, v, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)) || !encode_bnhd(&tdo, dO, mB, mNq, Hq, D, CKV::BM, tma_type(CKV::F16)) ||
         !encode_bnhd(&tdk, dk, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)) || !encode_bnhd(&tdv, dv, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)))
       return FA_ERR_CUDA;
-    auto kern = fa_bwd_dkdv_kernel<CKV, VL>;
-    if (smem_attr_once(kern, CKV::SMEM_BYTES, attr_kv) != cudaSuccess) return FA_ERR_CUDA;
+    auto kern = fa_bwd_dkdv_kernel<CKV, VL, BS>;
+    if (smem_attr_once(kern, BS ? 232448 : CKV::SMEM_BYTES, attr_kv) != cudaSuccess) return FA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(static_cast<long long>(p.n_kvtiles) * B * Hkv), D / CKV::DV);
     TraceScope tr(FA_KERNEL_BWD_DKDV, stream);
-    kern<<<grid, CKV::NTHREADS, CKV::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdk, tdv, p);
+    kern<<<grid, CKV::NTHREADS, static_cast<size_t>(kv_smem), stream>>>(tq, tk, tv, tdo, tdk, tdv, p);
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
   return FA_OK;
@@ -722,6 +744,40 @@ int fa_fwd_blocksparse_impl(const void* q, const void* k, const void* v, void* o
   }
 }
 
+template <bool F16>
+int fa_bwd_blocksparse_impl(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                            const void* dO, void* dq, void* dk, void* dv, const unsigned char* block_mask,
+                            long long mask_stride_b, long long mask_stride_h, int B, int Nq, int Nk, int Hq,
+                            int Hkv, int d, float scale, int causal, int win_l, int win_r, void* workspace,
+                            size_t workspace_bytes_, fa_stream_t stream) {
+  int st = check_common(q, k, v, B, Nq, Nk, Hq, Hkv, scale);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || block_mask == nullptr || mask_stride_b < 0 || mask_stride_h < 0)
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(workspace) || workspace_bytes_ < workspace_bytes(B, Nq, Hq)) return FA_ERR_WORKSPACE;
+  const MaskSpec mask = make_mask(Nq, Nk, causal, win_l, win_r);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* ws = static_cast<float*>(workspace);
+  BlockMask bm;
+  bm.mask = reinterpret_cast<const uint8_t*>(block_mask);
+  bm.sb = mask_stride_b;
+  bm.sh = mask_stride_h;
+  const Varlen vl;
+  switch (d) {
+    case 64:
+      return launch_bwd<Ty<F16, Dq64>, Ty<F16, Dkv64>, false, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk, Hq,
+                                                                    Hkv, scale, mask, ws, s, vl, bm);
+    case 128:
+      return launch_bwd<Ty<F16, Dq128>, Ty<F16, Dkv128>, false, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk,
+                                                                      Hq, Hkv, scale, mask, ws, s, vl, bm);
+    default:
+      return launch_bwd<Ty<F16, Dq256>, Ty<F16, Dkv256>, false, true>(q, k, v, o, lse, dO, dq, dk, dv, B, Nq, Nk,
+                                                                      Hq, Hkv, scale, mask, ws, s, vl, bm);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -877,6 +933,26 @@ int fa_fwd_blocksparse_f16(const void* q, const void* k, const void* v, void* o,
                            int win_r, fa_stream_t stream) {
   return fa_fwd_blocksparse_impl<true>(q, k, v, o, lse, block_mask, mask_stride_b, mask_stride_h, B, Nq, Nk, Hq,
                                        Hkv, d, scale, causal, win_l, win_r, stream);
+}
+
+int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dO, void* dq, void* dk, void* dv, const unsigned char* block_mask,
+                       long long mask_stride_b, long long mask_stride_h, int B, int Nq, int Nk, int Hq,
+                       int Hkv, int d, float scale, int causal, int win_l, int win_r, void* workspace,
+                       size_t workspace_bytes_, fa_stream_t stream) {
+  return fa_bwd_blocksparse_impl<false>(q, k, v, o, lse, dO, dq, dk, dv, block_mask, mask_stride_b, mask_stride_h,
+                                        B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, workspace,
+                                        workspace_bytes_, stream);
+}
+
+int fa_bwd_blocksparse_f16(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                           const void* dO, void* dq, void* dk, void* dv, const unsigned char* block_mask,
+                           long long mask_stride_b, long long mask_stride_h, int B, int Nq, int Nk, int Hq,
+                           int Hkv, int d, float scale, int causal, int win_l, int win_r, void* workspace,
+                           size_t workspace_bytes_, fa_stream_t stream) {
+  return fa_bwd_blocksparse_impl<true>(q, k, v, o, lse, dO, dq, dk, dv, block_mask, mask_stride_b, mask_stride_h,
+                                       B, Nq, Nk, Hq, Hkv, d, scale, causal, win_l, win_r, workspace,
+                                       workspace_bytes_, stream);
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int Nq,

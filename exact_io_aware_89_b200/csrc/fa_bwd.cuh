@@ -168,6 +168,12 @@ struct BwdParams {
   uint16_t* dq;  // outputs, for the plain stores of a packed sequence's last tile
   uint16_t* dk;
   uint16_t* dv;
+  // block-sparse (BS kernels): a byte per 128 x 128 (query block, key block)
+  // of batch b, query head h at bmask + b * bm_sb + h * bm_sh, rows of
+  // bm_cols key blocks; zero = the block is skipped
+  const uint8_t* bmask;
+  long long bm_sb, bm_sh;
+  int bm_cols;
   unsigned long long wait_limit_ns;
 };
 
@@ -205,7 +211,7 @@ struct DqCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <class C, bool VL = false>
+template <class C, bool VL = false, bool BS = false>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -241,7 +247,25 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int r_last = min(nq - 1, r0 + NQT * BM - 1);
   const int key_lo = sq.mask.lo(r0), key_hi = sq.mask.hi(r_last);
   const int j_begin = key_lo / BN;
-  const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
+  int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
+  // block-sparse: the key tiles of that range whose mask block is set for
+  // this query block, listed by the TMA warp before the block-wide sync
+  uint32_t* tile_list = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 16);
+  volatile int* list_count = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  if constexpr (BS) {
+    if (warp == C::TMA_WARP) {
+      const uint8_t* mrow = p.bmask + b * p.bm_sb + h * p.bm_sh + static_cast<long long>(r0 / 128) * p.bm_cols;
+      const int cnt = warp_compact(n_kv, tile_list, [&](int it) { return __ldg(mrow + (j_begin + it) * BN / 128) != 0; });
+      if (lane == 0) *list_count = cnt;
+      __syncwarp();
+    }
+  }
+  auto tile_of = [&](int it) {
+    if constexpr (BS)
+      return j_begin + static_cast<int>(tile_list[it]);
+    else
+      return j_begin + it;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -266,6 +290,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if constexpr (BS) n_kv = *list_count;
 
   if (warp == C::TMA_WARP) {
     if (lane == 0 && n_kv > 0) {
@@ -278,7 +303,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       int n_issued = 0;
       for (int it = 0; it < n_kv; ++it) {
         const int s = it % KST, use = it / KST;
-        const int krow = (j_begin + it) * BN;
+        const int krow = tile_of(it) * BN;
         if (use > 0 && !mbar_wait(&kv_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns))
           break;
         mbar_expect_tx(&kv_full[s], 2 * C::KTILE);
@@ -394,7 +419,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       }
       float* sc = reinterpret_cast<float*>(sv);
       const float* dp = reinterpret_cast<const float*>(dv);
-      const int k0 = (j_begin + it) * BN;
+      const int k0 = tile_of(it) * BN;
       if (k0 < lo || k0 + BN - 1 > hi) {
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
@@ -511,7 +536,7 @@ struct Dq2Cfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <class C, bool VL = false>
+template <class C, bool VL = false, bool BS = false>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
     fa_bwd_dq2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -550,17 +575,35 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   const int r_last = min(nq - 1, r0 + BM - 1);
   const int key_lo = sq.mask.lo(r0), key_hi = sq.mask.hi(r_last);
   const int j_begin = key_lo / BN;
-  const int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
+  int n_kv = (key_hi >= key_lo) ? (key_hi / BN - j_begin + 1) : 0;
+  // block-sparse: the key tiles of that range whose mask block is set for
+  // this query tile, listed by the TMA warp before the block-wide sync
+  uint32_t* tile_list = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 16);
+  volatile int* list_count = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  if constexpr (BS) {
+    if (warp == C::TMA_WARP) {
+      const uint8_t* mrow = p.bmask + b * p.bm_sb + h * p.bm_sh + static_cast<long long>(r0 / 128) * p.bm_cols;
+      n_kv = warp_compact(n_kv, tile_list, [&](int it) { return __ldg(mrow + (j_begin + it) * BN / 128) != 0; });
+      if (lane == 0) *list_count = n_kv;
+      __syncwarp();
+    }
+  }
+  auto tile_of = [&](int it) {
+    if constexpr (BS)
+      return j_begin + static_cast<int>(tile_list[it]);
+    else
+      return j_begin + it;
+  };
 
   // copies of K or V of key tile `it` into their rings
   auto load_k = [&](int it) {
-    const int sk = it % KS, krow = (j_begin + it) * BN;
+    const int sk = it % KS, krow = tile_of(it) * BN;
     mbar_expect_tx(&k_full[sk], C::KTILE);
     for (int c = 0; c < C::NCHUNK; ++c)
       tma_load_4d(sK + sk * C::KTILE + c * C::KCHUNK, &tm_k, &k_full[sk], c * 64, hk, sq.k_off + krow, sq.tb);
   };
   auto load_v = [&](int it) {
-    const int sv = it % VS, krow = (j_begin + it) * BN;
+    const int sv = it % VS, krow = tile_of(it) * BN;
     mbar_expect_tx(&v_full[sv], C::KTILE);
     for (int c = 0; c < C::NCHUNK; ++c)
       tma_load_4d(sV + sv * C::KTILE + c * C::KCHUNK, &tm_v, &v_full[sv], c * 64, hk, sq.k_off + krow, sq.tb);
@@ -604,6 +647,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if constexpr (BS) n_kv = *list_count;
 
   if (warp == C::TMA_WARP) {
     if (lane == 0 && n_kv > 0) {
@@ -717,7 +761,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       tmem_ld_wait_x32(dv + 32);
       tc_fence_before();
       mbar_arrive(sp_free);  // S/dP may now be overwritten by the next key tile
-      const int k0 = (j_begin + it) * BN + wg * 64;
+      const int k0 = tile_of(it) * BN + wg * 64;
       if (k0 < lo || k0 + 63 > hi) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -834,7 +878,7 @@ struct DkvCfg {
   static_assert(STAGE % 1024 == 0, "stages stay 1 KiB aligned");
 };
 
-template <class C, bool VL = false>
+template <class C, bool VL = false, bool BS = false>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -878,10 +922,30 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   q_hi = min(q_hi, nq - 1);
   const int i_begin = q_lo / BM;
   const int n_qt = (q_hi >= q_lo) ? (q_hi / BM - i_begin + 1) : 0;
-  const int n_steps = n_qt * p.group;  // (query head in group) x (query tile)
-
-  auto step_head = [&](int step) { return hk * p.group + step / n_qt; };
-  auto step_q0 = [&](int step) { return (i_begin + step % n_qt) * BM; };
+  int n_steps = n_qt * p.group;  // (query head in group) x (query tile)
+  // block-sparse: the steps whose (query head, query block) mask block is set
+  // for this key block, listed by the TMA warp before the block-wide sync
+  uint32_t* step_list = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 16);
+  volatile int* list_count = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  if constexpr (BS) {
+    if (warp == C::TMA_WARP) {
+      const uint8_t* mb = p.bmask + b * p.bm_sb + k0 / 128;
+      n_steps = warp_compact(n_steps, step_list, [&](int st) {
+        const int hq = hk * p.group + st / n_qt, qb = (i_begin + st % n_qt) * BM / 128;
+        return __ldg(mb + hq * p.bm_sh + static_cast<long long>(qb) * p.bm_cols) != 0;
+      });
+      if (lane == 0) *list_count = n_steps;
+      __syncwarp();
+    }
+  }
+  auto step_of = [&](int it) {
+    if constexpr (BS)
+      return static_cast<int>(step_list[it]);
+    else
+      return it;
+  };
+  auto step_head = [&](int it) { return hk * p.group + step_of(it) / n_qt; };
+  auto step_q0 = [&](int it) { return (i_begin + step_of(it) % n_qt) * BM; };
   // copies of step `it` (Q, dO and their lse2 / D rows) into stage it % ST
   auto load_step = [&](int it) {
     const int s = it % ST;
@@ -932,6 +996,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if constexpr (BS) n_steps = *list_count;
 
   if (warp == C::TMA_WARP) {
     if (lane == 0 && n_steps > 0) {

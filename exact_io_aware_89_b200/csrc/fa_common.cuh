@@ -107,6 +107,23 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+// Block-sparse attention: the calling warp (all 32 lanes) appends, in
+// order, the indices i in [0, n) with on(i) true to `list` (ballot
+// compaction, 32 indices per round) and returns how many there are.
+template <class F>
+__device__ __forceinline__ int warp_compact(int n, uint32_t* list, F on) {
+  const int lane = threadIdx.x % 32;
+  int cnt = 0;
+  for (int c0 = 0; c0 < n; c0 += 32) {
+    const int i = c0 + lane;
+    const bool a = i < n && on(i);
+    const unsigned bal = __ballot_sync(0xffffffffu, a);
+    if (a) list[cnt + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint32_t>(i);
+    cnt += __popc(bal);
+  }
+  return cnt;
+}
+
 // A kernel configuration with fp16 instead of bf16 elements: the same tiles;
 // the tensor-core operand type, the conversions to 16 bits and the TMA data
 // type follow C::F16.

@@ -254,6 +254,24 @@ int fa_fwd_blocksparse_f16(const void* q, const void* k, const void* v, void* o,
                            int win_r, fa_stream_t stream);
 
 /*
+ * Block-sparse backward: the gradients of fa_fwd_blocksparse with the same
+ * block mask (the skipped tiles contribute nothing, and are not computed),
+ * deterministic, with fa_bwd's other arguments and workspace.
+ * FA_ERR_UNSUPPORTED also when the per-CTA lists of tiles do not fit in
+ * shared memory (Nk or (Hq / Hkv) * Nq in the hundreds of thousands).
+ */
+int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dO, void* dq, void* dk, void* dv, const unsigned char* block_mask,
+                       long long mask_stride_b, long long mask_stride_h, int B, int Nq, int Nk, int Hq,
+                       int Hkv, int d, float scale, int causal, int win_l, int win_r, void* workspace,
+                       size_t workspace_bytes, fa_stream_t stream);
+int fa_bwd_blocksparse_f16(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                           const void* dO, void* dq, void* dk, void* dv, const unsigned char* block_mask,
+                           long long mask_stride_b, long long mask_stride_h, int B, int Nq, int Nk, int Hq,
+                           int Hkv, int d, float scale, int causal, int win_l, int win_r, void* workspace,
+                           size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fp16 variants (hysenlabs page, requirements: fp16 and bf16 inputs): the
  * same arguments, semantics, layouts and workspace sizes as the bf16 entry
  * points of the same name without the suffix, with every 16-bit tensor

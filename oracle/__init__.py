@@ -211,6 +211,52 @@ def attn_fwd_blockmask(q, k, v, block_mask, block=128, scale=None, causal=False,
     return o, lse
 
 
+def attn_bwd_blockmask(q, k, v, dout, block_mask, block=128, scale=None, causal=False,
+                       window=(-1, -1)):
+    """Gradients of sum(dout * O) for attn_fwd_blockmask's O: the backward
+    formulas of attn_bwd (D = rowsum(dO * O), dS = P (dP - D), dQ = scale dS K,
+    dK = scale dS^T Q, dV = P^T dO, summed over a key/value head's query
+    heads) with P zero wherever the block mask or the causal / window masks
+    hide a key.  Plain numpy in fp64, for small problems."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    G = Hq // Hkv
+    nqb, nkb = -(-Nq // block), -(-Nk // block)
+    bm = np.broadcast_to(np.asarray(block_mask) != 0, (B, Hq, nqb, nkb))
+    i = np.arange(Nq)[:, None]
+    j = np.arange(Nk)[None, :]
+    delta = Nk - Nq
+    wl, wr = window if window is not None else (-1, -1)
+    wr = 0 if causal else wr
+    vis = np.ones((Nq, Nk), dtype=bool)
+    if wr >= 0:
+        vis &= j <= i + delta + wr
+    if wl >= 0:
+        vis &= j >= i + delta - wl
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            blk = np.repeat(np.repeat(bm[b, h], block, axis=0), block, axis=1)[:Nq, :Nk]
+            m = vis & blk
+            s = np.where(m, scale * (q[b, :, h, :] @ k[b, :, hk, :].T), -np.inf)
+            mx = s.max(axis=1)
+            live = np.isfinite(mx)
+            e = np.where(m, np.exp(s - np.where(live, mx, 0.0)[:, None]), 0.0)
+            l = e.sum(axis=1)
+            p = np.where(live[:, None], e / np.where(live, l, 1.0)[:, None], 0.0)
+            o = p @ v[b, :, hk, :]
+            do = dout[b, :, h, :]
+            Drow = (do * o).sum(axis=1)
+            dp = do @ v[b, :, hk, :].T
+            ds = p * (dp - Drow[:, None])
+            dq[b, :, h, :] = scale * (ds @ k[b, :, hk, :])
+            dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])
+            dv[b, :, hk, :] += p.T @ do
+    return dq, dk, dv
+
+
 def merge_partials(o_parts, lse_parts):
     """Merge attention results computed over disjoint key subsets.
 

@@ -28,7 +28,7 @@ def test_header_declares_the_expected_entry_points():
         "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_kvcache",
         "fa_fwd_kvcache_workspace_size", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_f16",
         "fa_bwd_f16", "fa_fwd_varlen_f16", "fa_bwd_varlen_f16", "fa_fwd_splitkv_f16", "fa_fwd_kvcache_f16",
-        "fa_fwd_blocksparse", "fa_fwd_blocksparse_f16",
+        "fa_fwd_blocksparse", "fa_fwd_blocksparse_f16", "fa_bwd_blocksparse", "fa_bwd_blocksparse_f16",
         "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
 
 

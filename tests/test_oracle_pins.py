@@ -465,3 +465,33 @@ def test_blockmask_query_block_off_gives_empty_rows_and_heads_differ():
     o_ref, _ = oracle.attn_fwd(q, k, v)
     assert np.abs(o[0, :, 0] - o_ref[0, :, 0]).max() < 1e-12
     assert np.abs(o[0, 4:, 1] - o_ref[0, 4:, 1]).max() < 1e-12
+
+
+@pytest.mark.parametrize("causal,window", [(False, (-1, -1)), (True, (-1, -1)), (True, (4, -1))])
+def test_blockmask_gradients_all_ones_are_the_dense_gradients(causal, window):
+    rng = np.random.default_rng(63)
+    q = rng.standard_normal((1, 11, 4, 5))
+    k = rng.standard_normal((1, 14, 2, 5))
+    v = rng.standard_normal((1, 14, 2, 5))
+    do = rng.standard_normal((1, 11, 4, 5))
+    g = oracle.attn_bwd_blockmask(q, k, v, do, np.ones((1, 1, 3, 4)), block=4, causal=causal,
+                                  window=window)
+    ref = oracle.attn_bwd(q, k, v, do, causal=causal, window=window)
+    for a, r in zip(g, ref):
+        assert np.abs(a - r).max() < 1e-11
+
+
+def test_blockmask_gradients_with_key_blocks_off_are_those_of_the_remaining_keys():
+    rng = np.random.default_rng(64)
+    q = rng.standard_normal((1, 9, 2, 4))
+    k = rng.standard_normal((1, 16, 1, 4))
+    v = rng.standard_normal((1, 16, 1, 4))
+    do = rng.standard_normal((1, 9, 2, 4))
+    bm = np.ones((1, 1, 3, 4))
+    bm[..., 2] = 0
+    dq, dk, dv = oracle.attn_bwd_blockmask(q, k, v, do, bm, block=4)
+    keep = np.r_[0:8, 12:16]
+    rq, rk, rv = oracle.attn_bwd(q, k[:, keep], v[:, keep], do)
+    assert np.abs(dq - rq).max() < 1e-11
+    assert np.abs(dk[:, keep] - rk).max() < 1e-11 and np.abs(dv[:, keep] - rv).max() < 1e-11
+    assert np.all(dk[:, 8:12] == 0) and np.all(dv[:, 8:12] == 0)

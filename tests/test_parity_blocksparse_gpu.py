@@ -1,5 +1,6 @@
-"""GPU parity of fa_fwd_blocksparse against the fp64 oracle's block-masked
-attention (same seeded inputs, same 128 x 128 block mask).
+"""GPU parity of fa_fwd_blocksparse and fa_bwd_blocksparse against the fp64
+oracle's block-masked attention and gradients (same seeded inputs, same
+128 x 128 block mask).
 
 Random masks per (batch, head) -- so the two 128-row Q tiles of a CTA often
 have different key tiles on -- and masks shared across batch and heads
@@ -14,7 +15,7 @@ import torch
 
 import exact_io_aware_89_b200 as fa
 import oracle
-from parity_utils import TOL_BF16, compare_lse, o_error
+from parity_utils import TOL_BF16, ZERO_ABS, compare_lse, o_error, rel_fro
 from seeded_inputs import make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -95,3 +96,54 @@ def test_local_plus_global_pattern_long():
         mask[0, 0, i, max(0, i - 2):i + 1] = True
         mask[0, 0, i, 0] = True
     check_bs(B, N, N, Hq, Hkv, d, mask, causal=True, seed=76)
+
+
+def check_bs_bwd(B, Nq, Nk, Hq, Hkv, d, mask, causal=False, window=(-1, -1), seed=0):
+    inp = make_inputs(B, Nq, Nk, Hq, Hkv, d, seed)
+    dev = torch.device("cuda")
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    scale = 1.0 / math.sqrt(d)
+    m = torch.from_numpy(np.ascontiguousarray(mask.astype(np.uint8))).to(dev)
+    o, lse = fa.attention_forward_blocksparse(q, k, v, m, scale=scale, causal=causal, window=window)
+    g1 = fa.attention_backward_blocksparse(q, k, v, o, lse, do, m, scale=scale, causal=causal,
+                                           window=window)
+    g2 = fa.attention_backward_blocksparse(q, k, v, o, lse, do, m, scale=scale, causal=causal,
+                                           window=window)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status(None) == 0
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b), "block-sparse backward not deterministic"
+    f64 = {n: t.double().numpy() for n, t in inp.items()}
+    refs = oracle.attn_bwd_blockmask(f64["q"], f64["k"], f64["v"], f64["do"], mask, block=T,
+                                     scale=scale, causal=causal, window=window)
+    what = "blocksparse bwd B%d Nq%d Nk%d Hq%d Hkv%d d%d causal%d win%s" % (
+        B, Nq, Nk, Hq, Hkv, d, causal, window)
+    for name, g, r in zip(("dq", "dk", "dv"), g1, refs):
+        g = g.float().cpu().numpy()
+        if not np.any(r):
+            assert float(np.abs(g).max()) <= ZERO_ABS, "%s: %s should be ~0" % (what, name)
+            continue
+        e = rel_fro(g, r)
+        assert e <= TOL_BF16["grad"], "%s: %s rel err %.3e" % (what, name, e)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal,window", [(False, (-1, -1)), (True, (-1, -1)), (False, (300, 200))])
+def test_backward_random_masks_per_head(d, causal, window):
+    B, Nq, Nk, Hq, Hkv = 2, 700, 900, 4, 2
+    mask = rand_mask((B, Hq, -(-Nq // T), -(-Nk // T)), 0.5, seed=3 * d + causal)
+    check_bs_bwd(B, Nq, Nk, Hq, Hkv, d, mask, causal, window, seed=81)
+
+
+def test_backward_all_ones_mask_is_the_dense_backward_bit_for_bit():
+    B, N, Hq, Hkv, d = 2, 1000, 4, 2, 128
+    inp = make_inputs(B, N, N, Hq, Hkv, d, 82)
+    dev = torch.device("cuda")
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    ones = torch.ones((1, 1, 8, 8), dtype=torch.uint8, device=dev)
+    o, lse = fa.attention_forward(q, k, v, causal=True)
+    g1 = fa.attention_backward_blocksparse(q, k, v, o, lse, do, ones, causal=True)
+    g2 = fa.attention_backward(q, k, v, o, lse, do, causal=True)
+    torch.cuda.synchronize()
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)
