@@ -829,6 +829,92 @@ def run_varlen(args, local):
         torch.cuda.empty_cache()
 
 
+# ------------------------------------------------------------ block-sparse
+
+def blocksparse_workloads():
+    """Block-sparse patterns over 128 x 128 tiles at long sequence lengths:
+    a band of local blocks plus global first blocks (local + global sparse
+    attention), and random blocks at a fixed density (seeded)."""
+    return [
+        dict(name="block-sparse local (4 blocks) + global (first block) B=2 H=16 N=8192 d=128",
+             B=2, N=8192, H=16, d=128, pattern="local_global", band=4, causal=False, seed=7001),
+        dict(name="block-sparse random 25% of blocks B=2 H=16 N=8192 d=128",
+             B=2, N=8192, H=16, d=128, pattern="random", density=0.25, causal=False, seed=7002),
+    ]
+
+
+def blocksparse_mask(w):
+    import numpy as np
+    nb = -(-w["N"] // 128)
+    if w["pattern"] == "local_global":
+        m = np.zeros((nb, nb), dtype=bool)
+        for i in range(nb):
+            m[i, max(0, i - w["band"] + 1):i + 1] = True
+            m[i, 0] = True
+            m[0, i] = True
+        return m[None, None]
+    rng = np.random.default_rng(w["seed"])
+    return rng.random((1, w["H"], nb, nb)) < w["density"]
+
+
+def run_blocksparse(args, local):
+    """One JSON line per block-sparse workload: fa_fwd_blocksparse,
+    fa_bwd_blocksparse and both, L2 flushed before every call; TFLOP/s
+    counted on the computed blocks (4 d flop per (query, key) pair inside
+    them, backward 2.5x), and the dense kernels on the same inputs."""
+    import numpy as np
+    import torch
+    import exact_io_aware_89_b200 as fa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    flush = L2Flush(dev)
+    for w in blocksparse_workloads():
+        B, N, H, d = w["B"], w["N"], w["H"], w["d"]
+        x, _ = make_device_inputs(dict(B=B, N=N, H=H, Hkv=H, d=d, seed=w["seed"]), 0, dev)
+        q, k, v, do = x["q"], x["k"], x["v"], x["do"]
+        mask_np = blocksparse_mask(w)
+        m = torch.from_numpy(mask_np.astype(np.uint8)).to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(max(16, fa.fa_bwd_workspace_size(B, N, H, d)), dtype=torch.uint8, device=dev)
+        c = w["causal"]
+        fns = {
+            "fwd": lambda: fa.attention_forward_blocksparse(q, k, v, m, causal=c, out=o, lse=lse),
+            "bwd": lambda: fa.attention_backward_blocksparse(q, k, v, o, lse, do, m, causal=c, dq=dq,
+                                                             dk=dk, dv=dv, workspace=ws),
+            "dense_fwd": lambda: fa.attention_forward(q, k, v, causal=c, out=o, lse=lse),
+            "dense_bwd": lambda: fa.attention_backward(q, k, v, o, lse, do, causal=c, dq=dq, dk=dk,
+                                                       dv=dv, workspace=ws),
+        }
+        ms = {}
+        for mode, fn in fns.items():
+            for _ in range(args.warmup):
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush()
+                ev[i][0].record()
+                fn()
+                ev[i][1].record()
+            torch.cuda.synchronize()
+            ms[mode] = statistics.median(a.elapsed_time(b) for a, b in ev)
+        if fa.fa_get_device_status(None) != 0:
+            raise RuntimeError("device status reports a timed-out wait")
+        density = float(np.broadcast_to(mask_np, (B, H) + mask_np.shape[2:]).mean())
+        F = 4.0 * B * H * N * N * d * density
+        line = {"blocksparse": w["name"], "block_density": round(density, 4),
+                "ms": {k2: round(x2, 4) for k2, x2 in ms.items()},
+                "tflops_on_computed_blocks": {"fwd": round(F / ms["fwd"] / 1e9, 1),
+                                              "bwd": round(2.5 * F / ms["bwd"] / 1e9, 1)},
+                "speedup_vs_dense": {"fwd": round(ms["dense_fwd"] / ms["fwd"], 2),
+                                     "bwd": round(ms["dense_bwd"] / ms["bwd"], 2)}}
+        print(json.dumps(line), flush=True)
+        del q, k, v, do, o, lse, dq, dk, dv, ws, m
+        torch.cuda.empty_cache()
+
+
 def run_ours(args, world, rank, local):
     import torch
     dev = torch.device("cuda", local)
@@ -912,6 +998,9 @@ def main(argv=None):
     ap.add_argument("--decode", action="store_true",
                     help="instead of the benchmark line: the KV-cache decoding workloads through "
                          "fa_fwd_splitkv, one JSON line each")
+    ap.add_argument("--blocksparse", action="store_true",
+                    help="instead of the benchmark line: block-sparse workloads through "
+                         "fa_fwd_blocksparse / fa_bwd_blocksparse, one JSON line each")
     ap.add_argument("--varlen", action="store_true",
                     help="instead of the benchmark line: packed variable-length workloads through "
                          "fa_fwd_varlen / fa_bwd_varlen, one JSON line each")
@@ -928,10 +1017,12 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     world, rank, local = dist_setup(args)
-    if args.sweep or args.decode or args.varlen:
+    if args.sweep or args.decode or args.varlen or args.blocksparse:
         if world > 1:
-            raise SystemExit("--sweep, --decode and --varlen run on one GPU")
-        (run_sweep if args.sweep else run_decode if args.decode else run_varlen)(args, local)
+            raise SystemExit("--sweep, --decode, --varlen and --blocksparse run on one GPU")
+        fn = (run_sweep if args.sweep else run_decode if args.decode else
+              run_varlen if args.varlen else run_blocksparse)
+        fn(args, local)
         return
     if args.impl == "reference":
         run_reference(args, world, rank)  # rank 0 alone; no process group
