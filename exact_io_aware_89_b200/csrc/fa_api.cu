@@ -67,6 +67,10 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 using Fwd64 = FwdCfg<64, 2, 128, 3, 2, true>;
 using Fwd128 = FwdCfg<128, 2, 128, 2, 2>;
 using Fwd256 = FwdCfg<256, 1, 64, 2>;
+// block-sparse forward: one 128-row Q tile per CTA, so a CTA loads only the
+// key tiles of its own query block (two Q tiles would load the union of both)
+using FwdBs64 = FwdCfg<64, 1, 128, 4>;
+using FwdBs128 = FwdCfg<128, 1, 128, 2>;
 // dQ: one 128-row query tile per CTA with 128-key tiles {d, K ring, V ring};
 // d = 256 keeps 64-key tiles {d, Q tiles per CTA, key tile, K/V ring depth}
 using Dq64 = Dq2Cfg<64, 4, 3>;
@@ -731,10 +735,10 @@ int fa_fwd_blocksparse_impl(const void* q, const void* k, const void* v, void* o
   const uint8_t* bm = reinterpret_cast<const uint8_t*>(block_mask);
   switch (d) {
     case 64:
-      return launch_fwd_bs<Ty<F16, Fwd64>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, bm, mask_stride_b,
+      return launch_fwd_bs<Ty<F16, FwdBs64>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, bm, mask_stride_b,
                                            mask_stride_h, s);
     case 128:
-      return launch_fwd_bs<Ty<F16, Fwd128>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, bm, mask_stride_b,
+      return launch_fwd_bs<Ty<F16, FwdBs128>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, bm, mask_stride_b,
                                             mask_stride_h, s);
     case 256:
       return launch_fwd_bs<Ty<F16, Fwd256>>(q, k, v, o, lse, B, Nq, Nk, Hq, Hkv, scale, mask, bm, mask_stride_b,
