@@ -234,7 +234,8 @@ def fa_status_string(status):
     return load_library().fa_status_string(int(status)).decode()
 
 
-KERNEL_KINDS = ("fwd", "bwd_prep", "bwd_dq", "bwd_dkdv", "f32", "decode", "kvcache_append")
+KERNEL_KINDS = ("fwd", "bwd_prep", "bwd_dq", "bwd_dkdv", "f32", "decode", "kvcache_append",
+                "bwd_call")
 
 
 def fa_trace_enable(on):

@@ -260,6 +260,33 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
 }
 
 // ------------------------------------------------------------------ backward
+// The backward's dQ and dK/dV kernels depend only on the preprocess, not on
+// each other: dQ runs on a side stream of the device (forked from and joined
+// back into the caller's stream with events), so the last partial wave of
+// one kernel overlaps the other's CTAs.  Created once per device; the fork /
+// launch / join sequence holds a lock so concurrent callers cannot swap each
+// other's events.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+SideStream g_side[kMaxDevices];
+
+int side_stream(SideStream** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  SideStream& ss = g_side[dev];
+  if (ss.stream == nullptr) {
+    if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  *out = &ss;
+  return FA_OK;
+}
+
 // Packed sequences of a backward call (all null / 0 when dense).
 struct Varlen {
   const int* cu_q = nullptr;
@@ -289,6 +316,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   const long long kv_smem =
       CKV::SMEM_BYTES + (BS ? 4ll * (Hq / Hkv) * ((Nq + CKV::BM - 1) / CKV::BM + 1) : 0);
   if (dq_smem > 232448 || kv_smem > 232448) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> side_lock(g_side_mu);
+  SideStream* side = nullptr;
+  if (side_stream(&side) != FA_OK) return FA_ERR_CUDA;
+  TraceScope whole(FA_KERNEL_BWD_CALL, stream);  // ends after the join below
   constexpr int D = CQ::D;
   const int Nq_pad = pad_rows(Nq);
   const long long rows_pad = static_cast<long long>(B) * Hq * Nq_pad;
@@ -337,20 +368,26 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
       return FA_ERR_CUDA;
     const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
     const int attr_bytes = BS ? 232448 : CQ::SMEM_BYTES;
+    // fork: the side stream waits for the preprocess
+    if (cudaEventRecord(side->fork, stream) != cudaSuccess ||
+        cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+      return FA_ERR_CUDA;
+    cudaStream_t dq_stream = side->stream;
     if constexpr (CQ::ONE_TILE) {
       auto kern = fa_bwd_dq2_kernel<CQ, VL, BS>;
       if (smem_attr_once(kern, attr_bytes, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
-      TraceScope tr(FA_KERNEL_BWD_DQ, stream);
-      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, static_cast<size_t>(dq_smem), stream>>>(tq, tk, tv, tdo,
-                                                                                              tdq, p);
+      TraceScope tr(FA_KERNEL_BWD_DQ, dq_stream);
+      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, static_cast<size_t>(dq_smem), dq_stream>>>(tq, tk, tv,
+                                                                                                 tdo, tdq, p);
     } else {
       auto kern = fa_bwd_dq_kernel<CQ, VL, BS>;
       if (smem_attr_once(kern, attr_bytes, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
-      TraceScope tr(FA_KERNEL_BWD_DQ, stream);
-      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, static_cast<size_t>(dq_smem), stream>>>(tq, tk, tv, tdo,
-                                                                                              tdq, p);
+      TraceScope tr(FA_KERNEL_BWD_DQ, dq_stream);
+      kern<<<static_cast<unsigned>(grid), CQ::NTHREADS, static_cast<size_t>(dq_smem), dq_stream>>>(tq, tk, tv,
+                                                                                                 tdo, tdq, p);
     }
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
+    if (cudaEventRecord(side->join, dq_stream) != cudaSuccess) return FA_ERR_CUDA;
   }
   {
     CUtensorMap tq, tk, tv, tdo, tdk, tdv;
@@ -361,10 +398,14 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     auto kern = fa_bwd_dkdv_kernel<CKV, VL, BS>;
     if (smem_attr_once(kern, BS ? 232448 : CKV::SMEM_BYTES, attr_kv) != cudaSuccess) return FA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(static_cast<long long>(p.n_kvtiles) * B * Hkv), D / CKV::DV);
-    TraceScope tr(FA_KERNEL_BWD_DKDV, stream);
-    kern<<<grid, CKV::NTHREADS, static_cast<size_t>(kv_smem), stream>>>(tq, tk, tv, tdo, tdk, tdv, p);
+    {
+      TraceScope tr(FA_KERNEL_BWD_DKDV, stream);
+      kern<<<grid, CKV::NTHREADS, static_cast<size_t>(kv_smem), stream>>>(tq, tk, tv, tdo, tdk, tdv, p);
+    }
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
+  // join: the caller's stream continues after dQ too
+  if (cudaStreamWaitEvent(stream, side->join, 0) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
 }
 

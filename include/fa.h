@@ -328,7 +328,9 @@ const char* fa_status_string(int status);
 
 /*
  * Kernel tracing.  While enabled, every kernel the library launches is
- * bracketed by two CUDA events recorded on the caller's stream (events come
+ * bracketed by two CUDA events recorded on the stream it runs on (the
+ * caller's, or for the backward's dQ kernel the library's side stream of the
+ * device, forked from and joined back into the caller's stream) (events come
  * from a pool created when tracing is switched on; no device memory is
  * allocated).  fa_trace_read() waits for the recorded events, adds each
  * launch's device time to ms[kind] and one to launches[kind] for the
@@ -344,7 +346,9 @@ enum fa_kernel_kind {
   FA_KERNEL_F32 = 4,      /* any fp32-path kernel */
   FA_KERNEL_DECODE = 5,   /* fa_fwd_splitkv / fa_fwd_kvcache, bf16 (tcgen05) */
   FA_KERNEL_KVCACHE_APPEND = 6, /* fa_fwd_kvcache: new keys/values into the cache */
-  FA_KERNEL_KINDS = 7
+  FA_KERNEL_BWD_CALL = 7, /* not a kernel: a whole backward call, preprocess to the end of
+                             the dQ and dK/dV kernels (which run concurrently) */
+  FA_KERNEL_KINDS = 8
 };
 int fa_trace_enable(int on);
 int fa_trace_read(double* ms, long long* launches);

@@ -18,24 +18,32 @@ def test_flop_accounting_matches_the_metric():
     F = bench.fwd_flops(w)
     assert F == 4 * 2 * 16 * 2048 * 2048 * 128 / 2
     alg = bench.kernel_algorithmic(w)
-    tensor = sum(work for kind, (bound, work) in alg.items() if bound == "tensor")
+    kernels = {k: v for k, v in alg.items() if k not in bench.SPAN_KINDS}
+    tensor = sum(work for kind, (bound, work) in kernels.items() if bound == "tensor")
     assert tensor == pytest.approx(3.5 * F)  # forward + 2.5x for the backward
     assert alg["bwd_prep"][0] == "hbm"
+    # the whole backward call carries the backward's work once
+    assert alg["bwd_call"] == ("tensor", pytest.approx(2.5 * F))
+    assert sum(alg[k][1] for k in bench.STEP_UNITS) == pytest.approx(3.5 * F)
 
 
-def test_roofline_picks_the_longest_kernel_and_uses_the_measured_peak():
+def test_roofline_picks_the_longer_step_unit_and_uses_the_measured_peak():
     w = bench.WORKLOADS["train"]
     F = bench.fwd_flops(w)
-    res = {"trace_ms": {"fwd": 1.0, "bwd_dkdv": 3.0, "bwd_dq": 2.0, "bwd_prep": 0.5},
-           "trace_n": {"fwd": 10, "bwd_dkdv": 10, "bwd_dq": 10, "bwd_prep": 10}}
+    # dQ and dK/dV overlap: their spans add up to more than the backward call
+    res = {"trace_ms": {"fwd": 1.0, "bwd_dkdv": 3.0, "bwd_dq": 2.8, "bwd_prep": 0.5,
+                        "bwd_call": 3.6},
+           "trace_n": {"fwd": 10, "bwd_dkdv": 10, "bwd_dq": 10, "bwd_prep": 10, "bwd_call": 10}}
     peaks = dict(hbm_gbs=6000.0, bf16=1600.0, bf16_sustained=1400.0, source="test")
     dom, per = bench.roofline(w, res, peaks)
-    assert dom == "bwd_dkdv"
-    assert per["bwd_dkdv"]["achieved"] == pytest.approx(2 * F / 0.3e-3 / 1e12, rel=1e-3)
-    assert per["bwd_dkdv"]["peak"] == 1400.0
-    assert per["bwd_dkdv"]["frac"] == pytest.approx(per["bwd_dkdv"]["achieved"] / 1400.0, abs=1e-4)
-    assert sum(p["share"] for p in per.values()) == pytest.approx(1.0, abs=1e-3)
+    assert dom == "bwd_call"
+    assert per["bwd_call"]["achieved"] == pytest.approx(2.5 * F / 0.36e-3 / 1e12, rel=1e-3)
+    assert per["bwd_call"]["peak"] == 1400.0
+    assert per["bwd_call"]["frac"] == pytest.approx(per["bwd_call"]["achieved"] / 1400.0, abs=1e-4)
+    # shares partition the step over its units, the forward and the backward call
+    assert per["fwd"]["share"] + per["bwd_call"]["share"] == pytest.approx(1.0, abs=1e-3)
     assert per["bwd_prep"]["unit"] == "GB/s"
+    assert "note" in per["bwd_dq"] and "note" in per["bwd_dkdv"]
 
 
 def test_ncu_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
