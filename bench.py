@@ -52,13 +52,16 @@ WORKLOADS = {
 # only while the kernel sources hash to the ones that were profiled (a changed
 # kernel reports null until it is captured again).
 NCU_TRAFFIC = {
-    ("train", "bwd_dkdv"): dict(bytes=75.92e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
-    ("mid", "bwd_dkdv"): dict(bytes=377.51e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
-    ("mid", "bwd_dq"): dict(bytes=324.89e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
-    ("mid", "fwd"): dict(bytes=250.18e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
-    ("decode0", "decode"): dict(bytes=1078.37e6, profile="profiles/decode_B8Hq32Hkv8Nq1Nk32768d128.md"),
+    ("train", "bwd_call"): dict(bytes=178.76e6, profile="profiles/bwd_B2H16N2048d128_causal.md"),
+    ("train", "bwd_dkdv"): dict(bytes=72.97e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
+    ("train", "bwd_dq"): dict(bytes=71.95e6, profile="profiles/bwd_B2H16N2048d128_causal.md"),
+    ("train", "bwd_prep"): dict(bytes=33.84e6, profile="profiles/bwd_B2H16N2048d128_causal.md"),
+    ("mid", "bwd_dkdv"): dict(bytes=377.45e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
+    ("mid", "bwd_dq"): dict(bytes=324.64e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
+    ("mid", "fwd"): dict(bytes=250.54e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
+    ("decode0", "decode"): dict(bytes=1077.98e6, profile="profiles/decode_B8Hq32Hkv8Nq1Nk32768d128.md"),
 }
-NCU_SOURCES_SHA256 = "4864a9c974e614ab6418e92101430d8e43e5a0312cf6f65cf98cc6af68b8c8b4"
+NCU_SOURCES_SHA256 = "d6486c3313d478726c2ad018c2d947d8d5662e289649ce983765e51cc05008ee"
 
 
 def sources_sha256():
