@@ -147,3 +147,22 @@ def test_backward_all_ones_mask_is_the_dense_backward_bit_for_bit():
     torch.cuda.synchronize()
     for a, b in zip(g1, g2):
         assert torch.equal(a, b)
+
+
+def test_backward_fp16_random_mask():
+    B, Nq, Nk, Hq, Hkv, d = 1, 520, 700, 4, 2, 64
+    mask = rand_mask((B, Hq, -(-Nq // T), -(-Nk // T)), 0.5, seed=91)
+    inp = make_inputs(B, Nq, Nk, Hq, Hkv, d, 92, dtype="fp16")
+    dev = torch.device("cuda")
+    q, k, v, do = (inp[n].to(dev) for n in ("q", "k", "v", "do"))
+    m = torch.from_numpy(mask.astype(np.uint8)).to(dev)
+    o, lse = fa.attention_forward_blocksparse(q, k, v, m, causal=True)
+    dq, dk, dv = fa.attention_backward_blocksparse(q, k, v, o, lse, do, m, causal=True)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status(None) == 0 and dq.dtype == torch.float16
+    f64 = {n: t.double().numpy() for n, t in inp.items()}
+    refs = oracle.attn_bwd_blockmask(f64["q"], f64["k"], f64["v"], f64["do"], mask, block=T,
+                                     scale=1 / math.sqrt(d), causal=True)
+    for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
+        e = rel_fro(g.float().cpu().numpy(), r)
+        assert e <= TOL_BF16["grad"], "blocksparse fp16 %s rel err %.3e" % (name, e)
