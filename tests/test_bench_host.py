@@ -145,3 +145,35 @@ def test_sweep_covers_the_sequence_length_grid():
     for w in ws:
         if w["name"].startswith("sweep"):
             assert w["B"] * w["N"] == 16384 and w["H"] * w["d"] == 2048
+
+
+def test_varlen_flops_reduce_to_the_dense_count():
+    w = dict(H=16, d=128, causal=True)
+    lens = [2048, 2048]
+    dense = bench.fwd_flops(dict(B=2, H=16, N=2048, d=128, causal=True))
+    # per sequence L (L + 1) / 2 causal pairs: the diagonal counted, as in the dense kernels' work
+    assert bench.varlen_fwd_flops(w, lens) == pytest.approx(dense * (2049 / 2048))
+    for wl in bench.varlen_workloads():
+        l = bench.varlen_lengths(wl)
+        assert sum(l) == wl["tokens"] and max(l) <= wl["hi"] and min(l[:-1]) >= wl["lo"]
+
+
+def test_blocksparse_masks_have_the_stated_structure():
+    import numpy as np
+    for w in bench.blocksparse_workloads():
+        m = bench.blocksparse_mask(w)
+        nb = -(-w["N"] // 128)
+        assert m.shape[2:] == (nb, nb) and m.dtype == bool
+        if w["pattern"] == "local_global":
+            assert m[0, 0].diagonal().all() and m[0, 0, :, 0].all() and m[0, 0, 0, :].all()
+        else:
+            assert abs(m.mean() - w["density"]) < 0.02
+
+
+def test_decode_bytes_of_ragged_lengths():
+    w = [x for x in bench.decode_workloads() if x.get("ragged")][0]
+    row = w["Hkv"] * w["d"] * 2
+    lens = bench.decode_lengths(w)
+    expect = 2 * row * sum(min(w["Nk"], n + 1) for n in lens) + 4 * w["B"] * row \
+        + 2 * w["B"] * w["Nq"] * w["Hq"] * w["d"] * 2 + 4 * w["B"] * w["Hq"] * w["Nq"]
+    assert bench.decode_bytes(w) == expect
