@@ -3,11 +3,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step = the whole hot path over one batch: fa_fwd (O, LSE) then fa_bwd
-(dQ, dK, dV).  The headline workload is the training shape (B=2, H=16,
-N=2048, d=128, causal); the long wide shape (B=1, H=96, N=8192, d=128,
-causal) that the throughput target names is measured alongside it under
-``extra``.  FLOPs follow the metric: forward 4*B*H*N^2*d, halved when causal;
-forward+backward = 3.5x forward.
+(dQ, dK, dV).  The headline workload is the long wide shape (B=1, H=96,
+N=8192, d=128, causal), the largest causal d=128 configuration that fits one
+GPU; the training shape (B=2, H=16, N=2048, d=128, causal) is measured
+alongside it under ``extra``.  FLOPs follow the metric: forward 4*B*H*N^2*d,
+halved when causal; forward+backward = 3.5x forward.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
 on the launching stream, with L2 flushed between steps outside the events (a
@@ -48,20 +48,23 @@ WORKLOADS = {
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch,
-# from the ncu capture summarised in the named profile file.  It is reported
-# only while the kernel sources hash to the ones that were profiled (a changed
-# kernel reports null until it is captured again).
-NCU_TRAFFIC = {
-    ("train", "bwd_call"): dict(bytes=178.76e6, profile="profiles/bwd_B2H16N2048d128_causal.md"),
-    ("train", "bwd_dkdv"): dict(bytes=72.97e6, profile="profiles/bwd_dkdv_B2H16N2048d128_causal.md"),
-    ("train", "bwd_dq"): dict(bytes=71.95e6, profile="profiles/bwd_B2H16N2048d128_causal.md"),
-    ("train", "bwd_prep"): dict(bytes=33.84e6, profile="profiles/bwd_B2H16N2048d128_causal.md"),
-    ("mid", "bwd_dkdv"): dict(bytes=377.45e6, profile="profiles/bwd_dkdv_B1H32N8192d128_causal.md"),
-    ("mid", "bwd_dq"): dict(bytes=324.64e6, profile="profiles/bwd_dq_B1H32N8192d128_causal.md"),
-    ("mid", "fwd"): dict(bytes=250.54e6, profile="profiles/fwd_B1H32N8192d128_causal.md"),
-    ("decode0", "decode"): dict(bytes=1077.98e6, profile="profiles/decode_B8Hq32Hkv8Nq1Nk32768d128.md"),
-}
-NCU_SOURCES_SHA256 = "d6486c3313d478726c2ad018c2d947d8d5662e289649ce983765e51cc05008ee"
+# from the ncu captures summarised under profiles/; the table itself lives in
+# profiles/traffic.json (workload key, kernel kind, bytes, the capture's
+# summary file, and a sha256 of the kernel sources that were profiled).  A
+# figure is reported only while the current sources hash to that value: a
+# changed kernel reports null until it is captured again.
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def load_traffic():
+    try:
+        with open(TRAFFIC_TABLE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return "", {}
+    rows = {(r["workload"], r["kernel"]): dict(bytes=float(r["bytes"]), profile=r["profile"])
+            for r in t.get("captures", [])}
+    return t.get("sources_sha256", ""), rows
 
 
 def sources_sha256():
@@ -78,9 +81,10 @@ def sources_sha256():
     return h.hexdigest()
 
 
-def ncu_traffic(workload_key, kernel):
-    t = NCU_TRAFFIC.get((workload_key, kernel))
-    if t is None or sources_sha256() != NCU_SOURCES_SHA256:
+def ncu_traffic(workload_key, kernel, table=None):
+    sha, rows = table if table is not None else load_traffic()
+    t = rows.get((workload_key, kernel))
+    if t is None or not sha or sources_sha256() != sha:
         return None, None
     return t["bytes"], t["profile"]
 
@@ -313,7 +317,7 @@ def time_gpu(w, steps, warmup, world, rank, dev, with_e2e=True, with_trace=True)
     if with_e2e:
         hin = {n: t.pin_memory() for n, t in host.items()}
         hout = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                for n, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv))}
+                for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
         dbuf = {n: torch.empty_like(x[n]) for n in ("q", "k", "v", "do")}
         h2d = sum(t.numel() * t.element_size() for t in hin.values())
         d2h = sum(t.numel() * t.element_size() for t in hout.values())
@@ -328,6 +332,7 @@ def time_gpu(w, steps, warmup, world, rank, dev, with_e2e=True, with_trace=True)
                 dbuf[n].copy_(hin[n], non_blocking=True)
             step(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["do"])
             hout["o"].copy_(o, non_blocking=True)
+            hout["lse"].copy_(lse, non_blocking=True)
             hout["dq"].copy_(dq, non_blocking=True)
             hout["dk"].copy_(dk, non_blocking=True)
             hout["dv"].copy_(dv, non_blocking=True)
@@ -368,8 +373,22 @@ STEP_UNITS = ("fwd", "bwd_call")
 SPAN_KINDS = ("bwd_call",)  # traced spans that are not kernels
 
 
+def tensor_peak(peaks, clocks):
+    """The measured bf16 peak that applies to a kernel timed in this run: the
+    burst figure when the SM clock sampled over the timed region stayed at its
+    maximum with no power cap active (the cuBLAS burst ran under the same
+    conditions), else the sustained figure, measured under the power cap.
+    Returns (TFLOP/s, label)."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    capped = "sw_power_cap" in (clocks.get("reasons") or [])
+    if mhz and mx and mhz >= 0.95 * mx and not capped:
+        return peaks["bf16"], "burst"
+    return peaks["bf16_sustained"], "sustained"
+
+
 def roofline(w, res, peaks):
     alg = kernel_algorithmic(w)
+    tpeak, tlabel = tensor_peak(peaks, res.get("clocks") or {})
     per = {}
     for kind, (bound, work) in alg.items():
         n = res["trace_n"].get(kind, 0)
@@ -378,20 +397,20 @@ def roofline(w, res, peaks):
         avg_ms = res["trace_ms"][kind] / n
         if bound == "tensor":
             ach = work / (avg_ms * 1e-3) / 1e12
-            peak = peaks["bf16_sustained"]
+            peak, label = tpeak, tlabel
             unit = "TFLOP/s"
         else:
             ach = work / (avg_ms * 1e-3) / 1e9
-            peak = peaks["hbm_gbs"]
+            peak, label = peaks["hbm_gbs"], "copy"
             unit = "GB/s"
-        per[kind] = dict(bound=bound, achieved=round(ach, 2), peak=peak, unit=unit,
+        per[kind] = dict(bound=bound, achieved=round(ach, 2), peak=peak, peak_kind=label, unit=unit,
                          frac=round(ach / peak, 4), avg_ms=round(avg_ms, 4), launches=n,
                          share=None)
     units = [k for k in STEP_UNITS if k in per]
     total = sum(res["trace_ms"].get(k, 0.0) for k in units)
     for k in per:
         per[k]["share"] = round(res["trace_ms"][k] / total, 4) if total else None
-        if k in ("bwd_dq", "bwd_dkdv"):
+        if k in ("bwd_dq", "bwd_dkdv") and "bwd_dq" in per and "bwd_dkdv" in per:
             per[k]["note"] = "runs concurrently with the other backward kernel; span includes its share"
     dom = max(units, key=lambda k: res["trace_ms"][k]) if units else None
     return dom, per
@@ -946,28 +965,34 @@ def run_ours(args, world, rank, local):
     launches = int(sum(n for k, n in res["trace_n"].items() if k not in SPAN_KINDS))
 
     extra = []
-    if args.extra and args.workload != "wide":
-        we = WORKLOADS["wide"]
-        r2 = time_gpu(we, max(3, args.steps // 2), max(3, args.warmup), world, rank, dev,
-                      with_e2e=False)
-        F2 = fwd_flops(we)
-        tf2 = job_throughput(3.5 * F2, len(r2["step_ms"]), sum(r2["step_ms"]), world)
-        ff2 = job_throughput(F2, len(r2["fwd_ms"]), sum(r2["fwd_ms"]), world)
-        d2, per2 = roofline(we, r2, peaks)
-        extra.append({"workload": we["name"], "fwd_bwd_tflops": round(tf2, 2),
-                      "fwd_tflops": round(ff2, 2),
-                      "fwd_bwd_pct_dense_peak": round(100 * tf2 / (world * DENSE_PEAK_TFLOPS), 2),
-                      "fwd_pct_dense_peak": round(100 * ff2 / (world * DENSE_PEAK_TFLOPS), 2),
-                      "ms_per_step": round(statistics.mean(r2["step_ms"]), 4),
-                      "kernels": per2, "clocks": r2["clocks"]})
+    if args.extra:
+        for key in ("wide", "train"):
+            if key == args.workload:
+                continue
+            we = WORKLOADS[key]
+            r2 = time_gpu(we, max(3, args.steps // 2), max(3, args.warmup), world, rank, dev,
+                          with_e2e=False)
+            F2 = fwd_flops(we)
+            tf2 = job_throughput(3.5 * F2, len(r2["step_ms"]), sum(r2["step_ms"]), world)
+            ff2 = job_throughput(F2, len(r2["fwd_ms"]), sum(r2["fwd_ms"]), world)
+            d2, per2 = roofline(we, r2, peaks)
+            extra.append({"workload": we["name"], "fwd_bwd_tflops": round(tf2, 2),
+                          "fwd_tflops": round(ff2, 2),
+                          "fwd_bwd_pct_dense_peak": round(100 * tf2 / (world * DENSE_PEAK_TFLOPS), 2),
+                          "fwd_pct_dense_peak": round(100 * ff2 / (world * DENSE_PEAK_TFLOPS), 2),
+                          "ms_per_step": round(statistics.mean(r2["step_ms"]), 4),
+                          "dominant": d2, "kernels": per2, "clocks": r2["clocks"]})
 
     if rank != 0:
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         tf_c, heads, secs, threads = oracle_sample(w, budget_s=args.oracle_budget)
+        total = w["B"] * w["H"]
         cpu = {"value": round(tf_c, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": "%d of %d heads, full N, fwd+bwd, %.1f s" % (heads, w["B"] * w["H"], secs)}
+               "sample": "%d of %d heads, full N, fwd+bwd, %.1f s%s" % (
+                   heads, total, secs,
+                   "; batch throughput extrapolated from the sampled heads" if heads < total else "")}
     dk = per.get(dom, {}) if dom else {}
     traffic, traffic_profile = ncu_traffic(args.workload, dom)
     line = {
@@ -987,8 +1012,7 @@ def run_ours(args, world, rank, local):
         "roofline": {"kernel": dom, "bound": dk.get("bound"), "achieved": dk.get("achieved"),
                      "peak": dk.get("peak"), "unit": dk.get("unit"), "frac": dk.get("frac"),
                      "traffic": traffic, "traffic_profile": traffic_profile,
-                     "peak_source": "%s, %s" % (peaks["source"],
-                                                "sustained" if dk.get("bound") == "tensor" else "copy")},
+                     "peak_source": "%s, %s" % (peaks["source"], dk.get("peak_kind"))},
         "kernels": per,
         "gpu_launches": launches,
         "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": res["h2d"],
@@ -1006,7 +1030,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="train")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="wide")
     ap.add_argument("--no-extra", dest="extra", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-budget", type=float, default=15.0,

@@ -260,30 +260,55 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
 }
 
 // ------------------------------------------------------------------ backward
-// The backward's dQ and dK/dV kernels depend only on the preprocess, not on
-// each other: dQ runs on a side stream of the device (forked from and joined
-// back into the caller's stream with events), so the last partial wave of
-// one kernel overlaps the other's CTAs.  Created once per device; the fork /
-// launch / join sequence holds a lock so concurrent callers cannot swap each
-// other's events.
+// The backward's dQ and dK/dV kernels (the split backward) depend only on the
+// preprocess, not on each other: dQ runs on a side stream (forked from and
+// joined back into the caller's stream with events), so the last partial wave
+// of one kernel overlaps the other's CTAs.  Each caller stream of a device
+// gets its own side stream, so callers on independent streams never wait for
+// each other; the fork / launch / join sequence holds that entry's lock so
+// concurrent callers on the same stream cannot swap each other's events.
+// While the caller's stream is being captured into a CUDA graph, or when the
+// table of side streams is full, dQ is launched on the caller's stream itself
+// (in order, after the preprocess and before dK/dV): a capture then pulls in
+// no stream but the caller's.
 struct SideStream {
+  cudaStream_t owner = nullptr;  // the caller stream this entry serves
+  bool used = false;
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex mu;
 };
-std::mutex g_side_mu;
-SideStream g_side[kMaxDevices];
+constexpr int kSideStreamsPerDevice = 32;
+std::mutex g_side_table_mu;
+SideStream g_side[kMaxDevices][kSideStreamsPerDevice];
 
-int side_stream(SideStream** out) {
+// The side stream of `caller` on the current device, or nullptr when dQ should
+// run on the caller's stream (capture in progress, table full).  FA_ERR_CUDA
+// when a CUDA call fails.
+int side_stream(cudaStream_t caller, SideStream** out) {
+  *out = nullptr;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
-  SideStream& ss = g_side[dev];
-  if (ss.stream == nullptr) {
-    if (cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
-      return FA_ERR_CUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(caller, &cap) != cudaSuccess) return FA_ERR_CUDA;
+  if (cap != cudaStreamCaptureStatusNone) return FA_OK;
+  std::lock_guard<std::mutex> lock(g_side_table_mu);
+  SideStream* free_slot = nullptr;
+  for (SideStream& ss : g_side[dev]) {
+    if (ss.used && ss.owner == caller) {
+      *out = &ss;
+      return FA_OK;
+    }
+    if (!ss.used && free_slot == nullptr) free_slot = &ss;
   }
-  *out = &ss;
+  if (free_slot == nullptr) return FA_OK;
+  if (cudaStreamCreateWithFlags(&free_slot->stream, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&free_slot->fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&free_slot->join, cudaEventDisableTiming) != cudaSuccess)
+    return FA_ERR_CUDA;
+  free_slot->owner = caller;
+  free_slot->used = true;
+  *out = free_slot;
   return FA_OK;
 }
 
@@ -316,9 +341,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   const long long kv_smem =
       CKV::SMEM_BYTES + (BS ? 4ll * (Hq / Hkv) * ((Nq + CKV::BM - 1) / CKV::BM + 1) : 0);
   if (dq_smem > 232448 || kv_smem > 232448) return FA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> side_lock(g_side_mu);
   SideStream* side = nullptr;
-  if (side_stream(&side) != FA_OK) return FA_ERR_CUDA;
+  if (side_stream(stream, &side) != FA_OK) return FA_ERR_CUDA;
+  std::unique_lock<std::mutex> side_lock;
+  if (side != nullptr) side_lock = std::unique_lock<std::mutex>(side->mu);
   TraceScope whole(FA_KERNEL_BWD_CALL, stream);  // ends after the join below
   constexpr int D = CQ::D;
   const int Nq_pad = pad_rows(Nq);
@@ -369,10 +395,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
     const int attr_bytes = BS ? 232448 : CQ::SMEM_BYTES;
     // fork: the side stream waits for the preprocess
-    if (cudaEventRecord(side->fork, stream) != cudaSuccess ||
-        cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+    if (side != nullptr && (cudaEventRecord(side->fork, stream) != cudaSuccess ||
+                            cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess))
       return FA_ERR_CUDA;
-    cudaStream_t dq_stream = side->stream;
+    cudaStream_t dq_stream = side != nullptr ? side->stream : stream;
     if constexpr (CQ::ONE_TILE) {
       auto kern = fa_bwd_dq2_kernel<CQ, VL, BS>;
       if (smem_attr_once(kern, attr_bytes, attr_dq) != cudaSuccess) return FA_ERR_CUDA;
@@ -387,7 +413,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
                                                                                                  tdo, tdq, p);
     }
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
-    if (cudaEventRecord(side->join, dq_stream) != cudaSuccess) return FA_ERR_CUDA;
+    if (side != nullptr && cudaEventRecord(side->join, dq_stream) != cudaSuccess) return FA_ERR_CUDA;
   }
   {
     CUtensorMap tq, tk, tv, tdo, tdk, tdv;
@@ -405,7 +431,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     if (launch_status() != FA_OK) return FA_ERR_CUDA;
   }
   // join: the caller's stream continues after dQ too
-  if (cudaStreamWaitEvent(stream, side->join, 0) != cudaSuccess) return FA_ERR_CUDA;
+  if (side != nullptr && cudaStreamWaitEvent(stream, side->join, 0) != cudaSuccess) return FA_ERR_CUDA;
   return FA_OK;
 }
 

@@ -123,24 +123,32 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const flo
 
 /*
  * fa_bwd without a workspace argument, for callers that cannot allocate
- * device memory: code running inside a CUDA graph capture or a driver
- * callback, an allocator-free runtime, or a host program with a fixed
- * memory budget that has no cudaMalloc on its path.  The pages have no
- * counterpart; it is an addition of this library.
+ * device memory: an allocator-free runtime (an inference engine that carves
+ * all of its device memory out of one arena at start-up and forbids
+ * cudaMalloc afterwards), a host program with a fixed memory budget that has
+ * no cudaMalloc on its path, or code that records work into a CUDA graph and
+ * must not allocate while doing so.  The pages have no counterpart; it is an
+ * addition of this library.
  *
- * Same arguments, results and determinism as fa_bwd.  Its scratch (the
- * 8 * B * Hq * ceil(Nq/256)*256 bytes fa_bwd_workspace_size() reports) lives in
- * a fixed 16 MiB array inside the library's device image, so it handles
- * problems with B * Hq * ceil(Nq / 256) * 256 <= 2097152 rows and returns
- * FA_ERR_WORKSPACE, without launching anything, for larger ones.  The library
+ * Same arguments, results and determinism as fa_bwd (the same kernels run, so
+ * the outputs are bit-identical to fa_bwd's).  Its scratch (the bytes
+ * fa_bwd_workspace_size() reports for these sizes) lives in a fixed 16 MiB
+ * array inside the library's device image, which every GPU that loads the
+ * library holds until the process exits; problems whose workspace would not
+ * fit get FA_ERR_WORKSPACE, without anything being launched.  The library
  * calls no cudaMalloc/cudaFree and no allocating routine on this path.
  *
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  Every call on a device shares the one array and
- * overwrites it (nothing in it needs to start at zero): calls that can
- * overlap on the GPU -- on different streams without ordering between them --
- * race on it and must be serialised by the caller.
+ * The first backward call on a device (this one or fa_bwd) sets up
+ * per-device state: it looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and sets the kernels'
+ * shared-memory attributes; the first call from a given caller stream also
+ * creates that stream's side stream and two events.  Make one eager call on
+ * each device before any stream capture.  While the caller's stream is being
+ * captured, the backward keeps all of its launches on that stream.  Every
+ * call on a device shares the one array and overwrites it (the call clears
+ * what must start at zero itself): calls that can overlap on the GPU -- on
+ * different streams without ordering between them, or graph replays that
+ * overlap another call -- race on it and must be serialised by the caller.
  */
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                    const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq,

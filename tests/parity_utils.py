@@ -15,11 +15,13 @@ rounding noise from the bf16 O used in D).
 
 O is returned in bf16, rounded to nearest-even, so even an exactly rounded
 copy of the oracle's value differs from it by up to half a unit in the last
-place, at most |O| * 2^-8 (8 significant bits).  Where |O| is large -- rows
-that see only a few keys, whose output is close to single V rows -- that
-alone exceeds 1e-2 (|O| = 4 allows 1.6e-2).  The O bound is therefore
-1e-2 on top of that rounding allowance (o_error below); for the |O| << 1 of
-long rows it is the plain 1e-2.
+place of its binade: 2^(e - 8) for |O| in [2^e, 2^(e+1)) (8 significant
+bits; 2^(e - 11) for fp16, whose smallest normal binade 2^-14 also bounds the
+half unit below 2^-25).  Where |O| is large -- rows that see only a few keys,
+whose output is close to single V rows -- that alone exceeds 1e-2 (a half
+unit is 2^-6 = 1.6e-2 for |O| in [4, 8)).  The O bound is therefore 1e-2 on
+top of exactly that rounding (o_error below); for the |O| < 2^-0 of long rows
+the allowance is at most 2^-9, and the bound is essentially the plain 1e-2.
 
 Stress inputs outside the N(0,1) regime (a peaked softmax) use the criterion
 of the FlashAttention test suite (hysenlabs page, section on tests): the
@@ -41,17 +43,28 @@ TOL_F32 = dict(o=1e-4, lse=1e-4, grad=1e-4)
 ZERO_ABS = 1e-3
 
 
-BF16_HALF_ULP_REL = 2.0 ** -8   # bound on bf16 rounding error relative to |x|
-FP16_HALF_ULP_REL = 2.0 ** -11  # the same for fp16 (11 significant bits)
+# significant bits of the 16-bit output formats, and the smallest normal
+# binade's exponent (below it the spacing stops shrinking)
+_FORMAT = {"bf16": (8, -126), "fp16": (11, -14)}
+
+
+def half_ulp(x, dtype="bf16"):
+    """Half the spacing of the output format at the binade of each |x|: the
+    largest error of rounding x to nearest in that format (0 where x is 0)."""
+    bits, emin = _FORMAT[dtype]
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, emin)
+    return np.where(a > 0, np.exp2(e - bits), 0.0)
 
 
 def o_error(o_gpu, o_ref, dtype="bf16"):
-    """Max |o_gpu - o_ref| beyond the rounding of the output format itself
-    (|o_ref| * 2^-8 for bf16 outputs, 2^-11 for fp16; none for fp32)."""
+    """Max |o_gpu - o_ref| beyond the rounding of the output format itself:
+    half a unit in the last place of o_ref's binade for bf16 / fp16 outputs,
+    nothing for fp32."""
     diff = np.abs(np.asarray(o_gpu, dtype=np.float64) - o_ref)
     if dtype in ("bf16", "fp16"):
-        rel = BF16_HALF_ULP_REL if dtype == "bf16" else FP16_HALF_ULP_REL
-        diff = diff - rel * np.abs(o_ref)
+        diff = diff - half_ulp(o_ref, dtype)
     return float(diff.max()) if diff.size else 0.0
 
 

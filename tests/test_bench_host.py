@@ -46,23 +46,28 @@ def test_roofline_picks_the_longer_step_unit_and_uses_the_measured_peak():
     assert "note" in per["bwd_dq"] and "note" in per["bwd_dkdv"]
 
 
-def test_ncu_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
-    monkeypatch.setattr(bench, "NCU_SOURCES_SHA256", bench.sources_sha256())
-    b, prof = bench.ncu_traffic("train", "bwd_dkdv")
+def test_ncu_traffic_is_reported_only_for_the_profiled_sources():
+    _, rows = bench.load_traffic()
+    assert rows, "the traffic table lists no capture"
+    key = sorted(rows)[0]
+    current = (bench.sources_sha256(), rows)
+    b, prof = bench.ncu_traffic(*key, table=current)
     assert b > 0 and os.path.exists(os.path.join(ROOT, prof))
-    monkeypatch.setattr(bench, "NCU_SOURCES_SHA256", "0" * 64)
-    assert bench.ncu_traffic("train", "bwd_dkdv") == (None, None)
-    monkeypatch.setattr(bench, "NCU_SOURCES_SHA256", bench.sources_sha256())
-    assert bench.ncu_traffic("train", "no_such_kernel") == (None, None)
+    assert bench.ncu_traffic(*key, table=("0" * 64, rows)) == (None, None)
+    assert bench.ncu_traffic(*key, table=("", rows)) == (None, None)
+    assert bench.ncu_traffic("train", "no_such_kernel", table=current) == (None, None)
 
 
-def test_profiles_named_in_the_traffic_table_exist():
+def test_traffic_table_names_existing_summaries_and_known_workloads():
+    sha, rows = bench.load_traffic()
+    assert len(sha) == 64
     n_decode = len(bench.decode_workloads())
-    for (wl, kern), t in bench.NCU_TRAFFIC.items():
+    for (wl, kern), t in rows.items():
         if wl.startswith("decode"):
             assert kern == "decode" and 0 <= int(wl[len("decode"):]) < n_decode
         else:
             assert wl in bench.WORKLOADS
+        assert t["bytes"] > 0
         assert os.path.exists(os.path.join(ROOT, t["profile"])), t["profile"]
 
 
@@ -177,3 +182,29 @@ def test_decode_bytes_of_ragged_lengths():
     expect = 2 * row * sum(min(w["Nk"], n + 1) for n in lens) + 4 * w["B"] * row \
         + 2 * w["B"] * w["Nq"] * w["Hq"] * w["d"] * 2 + 4 * w["B"] * w["Hq"] * w["Nq"]
     assert bench.decode_bytes(w) == expect
+
+
+def test_tensor_peak_is_burst_at_full_clock_and_sustained_under_the_power_cap():
+    peaks = dict(hbm_gbs=6000.0, bf16=1662.1, bf16_sustained=1414.8, source="test")
+    full = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}
+    assert bench.tensor_peak(peaks, full) == (1662.1, "burst")
+    capped = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]}
+    assert bench.tensor_peak(peaks, capped) == (1414.8, "sustained")
+    slow = {"sm_mhz": 1400, "sm_max_mhz": 1965, "reasons": []}
+    assert bench.tensor_peak(peaks, slow) == (1414.8, "sustained")
+    assert bench.tensor_peak(peaks, {}) == (1414.8, "sustained")
+    w = bench.WORKLOADS["wide"]
+    F = bench.fwd_flops(w)
+    res = {"trace_ms": {"fwd": 16.0, "bwd_call": 50.0}, "trace_n": {"fwd": 10, "bwd_call": 10},
+           "clocks": full}
+    dom, per = bench.roofline(w, res, peaks)
+    assert dom == "bwd_call" and per[dom]["peak"] == 1662.1 and per[dom]["peak_kind"] == "burst"
+    assert per[dom]["frac"] == pytest.approx(2.5 * F / 5e-3 / 1e12 / 1662.1, abs=1e-4)
+
+
+def test_headline_workload_is_the_long_wide_shape():
+    import inspect
+    src = inspect.getsource(bench.main)
+    assert 'default="wide"' in src
+    w = bench.WORKLOADS["wide"]
+    assert (w["B"], w["H"], w["N"], w["d"], w["causal"]) == (1, 96, 8192, 128, True)

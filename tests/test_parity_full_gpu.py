@@ -39,10 +39,6 @@ def sweep(N, d, causal):
 WORKLOADS = {
     "train_B2_H16_N2048_d128_causal":
         dict(B=2, N=2048, Hq=16, Hkv=16, d=128, causal=True, window=(-1, -1), seed=config_seed(2)),
-    "sweep_N512_d64_noncausal": sweep(512, 64, False),
-    "sweep_N4096_d64_causal": sweep(4096, 64, True),
-    "sweep_N16384_d128_causal": sweep(16384, 128, True),
-    "sweep_N16384_d128_noncausal": sweep(16384, 128, False),
     "gqa_Hq32_Hkv8_N8192_d128_window4096":
         dict(B=1, N=8192, Hq=32, Hkv=8, d=128, causal=True, window=(4096, 0), seed=config_seed(4)),
     "wide_B1_H96_N8192_d128_causal":
@@ -50,6 +46,12 @@ WORKLOADS = {
     "d256_B1_H16_N16384_causal":
         dict(B=1, N=16384, Hq=16, Hkv=16, d=256, causal=True, window=(-1, -1), seed=config_seed(5) + 50),
 }
+# every point of the sequence-length sweep: N in 512 .. 16k, d in {64, 128},
+# causal and non-causal (hidden 2048, B = 16384 / N)
+for _N in (512, 1024, 2048, 4096, 8192, 16384):
+    for _d in (64, 128):
+        for _c in (True, False):
+            WORKLOADS["sweep_N%d_d%d_%s" % (_N, _d, "causal" if _c else "noncausal")] = sweep(_N, _d, _c)
 
 
 def sample_rows(N, rng, extra=4):
