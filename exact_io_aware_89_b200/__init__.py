@@ -34,6 +34,8 @@ __all__ = [
     "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
     "KERNEL_KINDS", "attention_forward", "attention_backward", "attention_forward_splitkv",
     "attention_forward_kvcache", "attention_forward_varlen", "attention_backward_varlen",
+    "fa_lse_merge", "fa_lse_merge_f16", "fa_grad_accumulate", "fa_grad_accumulate_f16",
+    "lse_merge", "grad_accumulate",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -101,6 +103,12 @@ def load_library():
                  "fa_fwd_kvcache", "fa_fwd_blocksparse", "fa_bwd_blocksparse"):
         getattr(lib, base + "_f16").argtypes = getattr(lib, base).argtypes
         getattr(lib, base + "_f16").restype = i
+    for name in ("fa_lse_merge", "fa_lse_merge_f16"):
+        getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+        getattr(lib, name).restype = i
+    for name in ("fa_grad_accumulate", "fa_grad_accumulate_f16"):
+        getattr(lib, name).argtypes = [vp, vp, vp, ll, i, vp]
+        getattr(lib, name).restype = i
     for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache", "fa_fwd_varlen", "fa_bwd_varlen",
                  "fa_get_device_status",
                  "fa_trace_enable", "fa_trace_read"):
@@ -234,8 +242,26 @@ def fa_status_string(status):
     return load_library().fa_status_string(int(status)).decode()
 
 
+def fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream):
+    """Fold one partial forward result (bf16 O, fp32 LSE) into a running fp32 one."""
+    return load_library().fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream)
+
+
+def fa_lse_merge_f16(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream):
+    return load_library().fa_lse_merge_f16(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream)
+
+
+def fa_grad_accumulate(acc, part, out, n, first, stream):
+    """acc (fp32) = (first ? 0 : acc) + part (bf16); out (bf16) = rounded acc."""
+    return load_library().fa_grad_accumulate(acc, part, out, n, first, stream)
+
+
+def fa_grad_accumulate_f16(acc, part, out, n, first, stream):
+    return load_library().fa_grad_accumulate_f16(acc, part, out, n, first, stream)
+
+
 KERNEL_KINDS = ("fwd", "bwd_prep", "bwd_dq", "bwd_dkdv", "f32", "decode", "kvcache_append",
-                "bwd_call")
+                "bwd_call", "merge")
 
 
 def fa_trace_enable(on):
@@ -527,3 +553,28 @@ def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1
                            Hq, Hkv, d, scale, c, wl, wr, workspace.data_ptr(),
                            workspace.numel() * workspace.element_size(), _stream()))
     return dq, dk, dv
+
+
+def lse_merge(o_acc, lse_acc, o_part, lse_part, first=False, out=None):
+    """Fold (o_part [B, Nq, H, d] bf16/fp16, lse_part [B, H, Nq] fp32) into the
+    running fp32 result (o_acc, lse_acc), in place; with ``out`` given, also
+    write the merged O rounded to out's type.  Returns ``out``."""
+    import torch
+    B, Nq, H, d = o_part.shape
+    fn = fa_lse_merge_f16 if o_part.dtype == torch.float16 else fa_lse_merge
+    _check(fn.__name__, fn(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
+                           out.data_ptr() if out is not None else None, B, Nq, H, d, int(bool(first)),
+                           _stream()))
+    return out
+
+
+def grad_accumulate(acc, part=None, first=False, out=None):
+    """acc (fp32) = (first ? 0 : acc) + part (bf16/fp16), in place; with ``out``
+    given, also write acc rounded to out's type.  Returns ``out``."""
+    import torch
+    ref = part if part is not None else out
+    fn = fa_grad_accumulate_f16 if ref.dtype == torch.float16 else fa_grad_accumulate
+    _check(fn.__name__, fn(acc.data_ptr(), part.data_ptr() if part is not None else None,
+                           out.data_ptr() if out is not None else None, acc.numel(), int(bool(first)),
+                           _stream()))
+    return out

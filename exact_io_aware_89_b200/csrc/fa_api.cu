@@ -12,6 +12,7 @@
 #include "fa_decode.cuh"
 #include "fa_f32.cuh"
 #include "fa_fwd.cuh"
+#include "fa_merge.cuh"
 #include "fa_host.cuh"
 
 using namespace fa;
@@ -1091,6 +1092,78 @@ int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, c
     fa_bwd_dkdv_f32_kernel<<<static_cast<unsigned>((wk + 3) / 4), 128, 0, s>>>(q, k, v, dO, dk, dv, p);
   }
   return launch_status();
+}
+
+// ------------------------------------------------ ring attention: combining
+}  // extern "C"
+
+namespace {
+
+template <bool F16>
+int lse_merge_impl(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                   int Nq, int H, int d, int first, fa_stream_t stream) {
+  if (!aligned16(o_acc) || !aligned16(lse_acc) || !aligned16(o_part) || !aligned16(lse_part) ||
+      (o_out != nullptr && !aligned16(o_out)))
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || Nq < 1 || H < 1) return FA_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * Nq * H;
+  if (rows > (1ll << 40)) return FA_ERR_INVALID_ARG;
+  const long long blocks = (rows * 32 + 255) / 256;
+  if (blocks > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto* op = static_cast<const uint16_t*>(o_part);
+  auto* oo = static_cast<uint16_t*>(o_out);
+  TraceScope tr(FA_KERNEL_MERGE, s);
+  switch (d) {
+    case 64:
+      fa_lse_merge_kernel<64, F16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo, B,
+                                                                                Nq, H, first);
+      break;
+    case 128:
+      fa_lse_merge_kernel<128, F16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo,
+                                                                                 B, Nq, H, first);
+      break;
+    case 256:
+      fa_lse_merge_kernel<256, F16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo,
+                                                                                 B, Nq, H, first);
+      break;
+    default:
+      return FA_ERR_UNSUPPORTED;
+  }
+  return launch_status();
+}
+
+template <bool F16>
+int grad_accumulate_impl(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream) {
+  if (!aligned16(acc) || (part != nullptr && !aligned16(part)) || (out != nullptr && !aligned16(out)))
+    return FA_ERR_INVALID_ARG;
+  if (n < 8 || n % 8 != 0 || (part == nullptr && out == nullptr)) return FA_ERR_INVALID_ARG;
+  const long long blocks = (n / 8 + 255) / 256;
+  if (blocks > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  TraceScope tr(FA_KERNEL_MERGE, s);
+  fa_grad_accumulate_kernel<F16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      acc, static_cast<const uint16_t*>(part), static_cast<uint16_t*>(out), n, first);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                 int Nq, int H, int d, int first, fa_stream_t stream) {
+  return lse_merge_impl<false>(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream);
+}
+int fa_lse_merge_f16(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                     int Nq, int H, int d, int first, fa_stream_t stream) {
+  return lse_merge_impl<true>(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream);
+}
+int fa_grad_accumulate(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream) {
+  return grad_accumulate_impl<false>(acc, part, out, n, first, stream);
+}
+int fa_grad_accumulate_f16(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream) {
+  return grad_accumulate_impl<true>(acc, part, out, n, first, stream);
 }
 
 int fa_get_device_status(fa_stream_t stream) {

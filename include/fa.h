@@ -325,6 +325,45 @@ int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, c
                size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Ring (context-parallel) attention: combining partial results.  A long
+ * sequence is split across GPUs; each GPU keeps its slice of query rows while
+ * the key/value slices travel around the ring of GPUs (zocula.com fla guide,
+ * the flame bullets and the glossary entry on context parallelism).  Each GPU
+ * runs fa_fwd / fa_bwd on its (query slice, key/value slice) pairs; these two
+ * calls combine the pieces.
+ *
+ * fa_lse_merge folds the forward result over one more key set into a
+ * running result (abeam.tech FlashAttention summary, "computing softmax
+ * blockwise correctly", applied to whole key sets): with lse_s the natural
+ * log-sum-exp and O_s the normalised output of set s,
+ *     lse = ln sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.
+ *   o_acc  [B, Nq, H, d] fp32, lse_acc [B, H, Nq] fp32 : the running result,
+ *            updated in place; with first != 0 they are overwritten by the part
+ *            (their contents are ignored)
+ *   o_part [B, Nq, H, d] bf16 (_f16: fp16), lse_part [B, H, Nq] fp32 : the
+ *            result over the next key set, as fa_fwd wrote it
+ *   o_out  [B, Nq, H, d] bf16 / fp16, or NULL: the merged O, rounded
+ *   d in {64, 128, 256}.  Rows empty in both (lse = -inf) stay O = 0,
+ *   lse = -inf.  Merging parts in a fixed order gives the same bits every time.
+ *
+ * fa_grad_accumulate sums backward shares in fp32: the gradients fa_bwd
+ * computes for one key set, given the full rows' o and lse, are that set's
+ * share of dq and its keys' dk / dv.
+ *   acc  [n] fp32 : running sum, updated in place (first != 0: acc = part)
+ *   part [n] bf16 / fp16, or NULL (only convert)
+ *   out  [n] bf16 / fp16, or NULL: the sum, rounded
+ *   n a multiple of 8; at least one of part, out given.
+ * Both return FA_OK or FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED / FA_ERR_CUDA;
+ * pointers are device pointers aligned to 16 bytes; stream-ordered.
+ */
+int fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                 int Nq, int H, int d, int first, fa_stream_t stream);
+int fa_lse_merge_f16(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
+                     int Nq, int H, int d, int first, fa_stream_t stream);
+int fa_grad_accumulate(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream);
+int fa_grad_accumulate_f16(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
  * the current device: FA_OK, FA_ERR_TIMEOUT if a kernel gave up on a bounded
  * wait since the last call, or FA_ERR_CUDA if the synchronisation failed.
@@ -356,7 +395,8 @@ enum fa_kernel_kind {
   FA_KERNEL_KVCACHE_APPEND = 6, /* fa_fwd_kvcache: new keys/values into the cache */
   FA_KERNEL_BWD_CALL = 7, /* not a kernel: a whole backward call, preprocess to the end of
                              the dQ and dK/dV kernels (which run concurrently) */
-  FA_KERNEL_KINDS = 8
+  FA_KERNEL_MERGE = 8,    /* fa_lse_merge / fa_grad_accumulate */
+  FA_KERNEL_KINDS = 9
 };
 int fa_trace_enable(int on);
 int fa_trace_read(double* ms, long long* launches);

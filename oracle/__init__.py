@@ -289,6 +289,52 @@ def merge_partials(o_parts, lse_parts):
     return o, lse
 
 
+def attn_bwd_given_stats(q, k, v, dout, o, lse, scale=None, causal=False, window=(-1, -1)):
+    """The share of one key set in the gradients of sum(dout * O), where O
+    [B,Nq,Hq,d] and LSE [B,Hq,Nq] are the forward results of the full rows
+    (over a key set that contains k/v): the backward formulas of attn_bwd
+    with P taken from the given LSE and D from the given O (abeam.tech
+    FlashAttention summary, "backward uses recomputation": P is recomputed
+    from the saved statistics),
+        P = exp(scale q.k - LSE), D = rowsum(dout * O), dS = P (dP - D),
+        dQ_share = scale dS K, dK = scale dS^T Q, dV = P^T dout,
+    dK / dV summed over a key/value head's query heads.  The causal / window
+    masks apply within this set as in attn_fwd (bottom-right aligned).  Over
+    a partition of the keys the dQ shares add up to dQ, and each set's dK / dV
+    are the rows of the full dK / dV.  Plain numpy in fp64, small problems."""
+    q, k, v, dout, o = _f64(q), _f64(k), _f64(v), _f64(dout), _f64(o)
+    lse = np.asarray(lse, dtype=np.float64)
+    B, Nq, Nk, Hq, Hkv, d = _dims(q, k, v)
+    scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    G = Hq // Hkv
+    i = np.arange(Nq)[:, None]
+    j = np.arange(Nk)[None, :]
+    delta = Nk - Nq
+    wl, wr = window if window is not None else (-1, -1)
+    wr = 0 if causal else wr
+    vis = np.ones((Nq, Nk), dtype=bool)
+    if wr >= 0:
+        vis &= j <= i + delta + wr
+    if wl >= 0:
+        vis &= j >= i + delta - wl
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            s = scale * (q[b, :, h, :] @ k[b, :, hk, :].T)
+            L = lse[b, h, :]
+            live = np.isfinite(L)[:, None]
+            p = np.where(vis & live, np.exp(np.where(vis & live, s - np.where(live, L[:, None], 0.0), -np.inf)), 0.0)
+            do = dout[b, :, h, :]
+            Drow = (do * o[b, :, h, :]).sum(axis=1)
+            dp = do @ v[b, :, hk, :].T
+            ds = p * (dp - Drow[:, None])
+            dq[b, :, h, :] = scale * (ds @ k[b, :, hk, :])
+            dk[b, :, hk, :] += scale * (ds.T @ q[b, :, h, :])
+            dv[b, :, hk, :] += p.T @ do
+    return dq, dk, dv
+
+
 def _rows(rows):
     r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).ravel())
     return r, r.ctypes.data_as(ctypes.POINTER(ctypes.c_int))

@@ -29,7 +29,8 @@ def test_header_declares_the_expected_entry_points():
         "fa_fwd_kvcache_workspace_size", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_f16",
         "fa_bwd_f16", "fa_fwd_varlen_f16", "fa_bwd_varlen_f16", "fa_fwd_splitkv_f16", "fa_fwd_kvcache_f16",
         "fa_fwd_blocksparse", "fa_fwd_blocksparse_f16", "fa_bwd_blocksparse", "fa_bwd_blocksparse_f16",
-        "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read"])
+        "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
+        "fa_lse_merge", "fa_lse_merge_f16", "fa_grad_accumulate", "fa_grad_accumulate_f16"])
 
 
 def test_kernel_kinds_match_the_header():
@@ -273,3 +274,22 @@ def test_blocksparse_rejects_invalid_arguments():
     assert call(q=MISALIGNED) == INVALID
     assert call(Hq=3) == INVALID
     assert call(d=96) == UNSUPPORTED
+
+
+def test_ring_combining_calls_reject_invalid_arguments_before_launching():
+    ok = dict(o_acc=FAKE, lse_acc=FAKE, o_part=FAKE, lse_part=FAKE, o_out=None, B=1, Nq=8, H=2, d=64, first=1)
+
+    def merge(**kw):
+        a = dict(ok, **kw)
+        return fa.fa_lse_merge(a["o_acc"], a["lse_acc"], a["o_part"], a["lse_part"], a["o_out"], a["B"],
+                               a["Nq"], a["H"], a["d"], a["first"], None)
+    for kw in (dict(o_acc=0), dict(lse_part=FAKE + 4), dict(o_out=FAKE + 8), dict(B=0), dict(Nq=0), dict(H=-1)):
+        assert merge(**kw) == INVALID, kw
+    assert merge(d=96) == UNSUPPORTED
+    assert fa.fa_lse_merge_f16(FAKE, FAKE, FAKE, FAKE, None, 1, 8, 2, 100, 0, None) == UNSUPPORTED
+    acc = fa.fa_grad_accumulate
+    assert acc(FAKE, FAKE, None, 12, 0, None) == INVALID        # n not a multiple of 8
+    assert acc(FAKE, FAKE, None, 0, 0, None) == INVALID
+    assert acc(FAKE, None, None, 16, 0, None) == INVALID         # nothing to do
+    assert acc(FAKE + 4, FAKE, None, 16, 0, None) == INVALID     # misaligned
+    assert fa.fa_grad_accumulate_f16(0, FAKE, None, 16, 0, None) == INVALID

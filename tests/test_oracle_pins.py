@@ -495,3 +495,74 @@ def test_blockmask_gradients_with_key_blocks_off_are_those_of_the_remaining_keys
     assert np.abs(dq - rq).max() < 1e-11
     assert np.abs(dk[:, keep] - rk).max() < 1e-11 and np.abs(dv[:, keep] - rv).max() < 1e-11
     assert np.all(dk[:, 8:12] == 0) and np.all(dv[:, 8:12] == 0)
+
+
+# ---------------------------------------------------------------- a key set's share of the gradients
+
+@pytest.mark.parametrize("causal,window", [(False, (-1, -1)), (True, (-1, -1)), (False, (3, 2))])
+def test_share_of_the_whole_key_set_is_the_gradient(causal, window):
+    """With every key in the set, the share is attn_bwd's gradient (the
+    given O and LSE are then the set's own)."""
+    rng = np.random.default_rng(11)
+    B, N, Hq, Hkv, d = 1, 10, 4, 2, 6
+    q, k, v, do = (rng.standard_normal(s) for s in ((B, N, Hq, d), (B, N, Hkv, d), (B, N, Hkv, d), (B, N, Hq, d)))
+    o, lse = oracle.attn_fwd(q, k, v, causal=causal, window=window)
+    for got, ref in zip(oracle.attn_bwd_given_stats(q, k, v, do, o, lse, causal=causal, window=window),
+                        oracle.attn_bwd(q, k, v, do, causal=causal, window=window)):
+        np.testing.assert_allclose(got, ref, atol=1e-12)
+
+
+def test_shares_over_scattered_key_sets_add_up_to_the_gradients():
+    """Non-causal attention over keys split into scattered sets (every third
+    key): the dQ shares sum to dQ, and each set's dK / dV are the full
+    gradients' rows of its keys."""
+    rng = np.random.default_rng(12)
+    B, N, Hq, Hkv, d = 2, 12, 2, 1, 5
+    q, k, v, do = (rng.standard_normal(s) for s in ((B, N, Hq, d), (B, N, Hkv, d), (B, N, Hkv, d), (B, N, Hq, d)))
+    o, lse = oracle.attn_fwd(q, k, v)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do)
+    sdq = np.zeros_like(dq)
+    for m in range(3):
+        idx = np.arange(m, N, 3)
+        a, b_, c = oracle.attn_bwd_given_stats(q, k[:, idx], v[:, idx], do, o, lse)
+        sdq += a
+        np.testing.assert_allclose(b_, dk[:, idx], atol=1e-12)
+        np.testing.assert_allclose(c, dv[:, idx], atol=1e-12)
+    np.testing.assert_allclose(sdq, dq, atol=1e-12)
+
+
+@pytest.mark.parametrize("R", [2, 3, 4])
+def test_shares_over_causal_ring_blocks_add_up_to_the_gradients(R):
+    """Split a causal sequence into R equal slices: slice pairs above the
+    diagonal are hidden, the diagonal pairs are causal, the rest are seen
+    whole.  attn_bwd_given_stats on each visible pair, with the full rows' O
+    and LSE, sums to attn_bwd (dQ over the key slices, dK / dV over the query
+    slices)."""
+    rng = np.random.default_rng(20 + R)
+    B, n, Hq, Hkv, d = 2, 4, 4, 2, 8
+    N = R * n
+    q, k, v, do = (rng.standard_normal(s) for s in ((B, N, Hq, d), (B, N, Hkv, d), (B, N, Hkv, d), (B, N, Hq, d)))
+    o, lse = oracle.attn_fwd(q, k, v, causal=True)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, do, causal=True)
+    sdq, sdk, sdv = np.zeros_like(dq), np.zeros_like(dk), np.zeros_like(dv)
+    for r in range(R):
+        qs = slice(r * n, (r + 1) * n)
+        for s in range(r + 1):
+            ks = slice(s * n, (s + 1) * n)
+            a, b_, c = oracle.attn_bwd_given_stats(q[:, qs], k[:, ks], v[:, ks], do[:, qs], o[:, qs],
+                                                   lse[:, :, qs], causal=(s == r))
+            sdq[:, qs] += a
+            sdk[:, ks] += b_
+            sdv[:, ks] += c
+    np.testing.assert_allclose(sdq, dq, atol=1e-12)
+    np.testing.assert_allclose(sdk, dk, atol=1e-12)
+    np.testing.assert_allclose(sdv, dv, atol=1e-12)
+
+
+def test_share_of_a_set_no_row_sees_is_zero():
+    """Rows with LSE = -inf (they see no key) contribute nothing."""
+    rng = np.random.default_rng(5)
+    q, k, v, do, o = (rng.standard_normal((1, 4, 1, 4)) for _ in range(5))
+    lse = np.full((1, 1, 4), -np.inf)
+    for g in oracle.attn_bwd_given_stats(q, k, v, do, o, lse):
+        assert not np.any(g)

@@ -1,0 +1,117 @@
+"""Ring (context-parallel) attention on the GPU, against the fp64 oracle.
+
+* fa_lse_merge folding partial results in order equals oracle.merge_partials
+  on the same (bf16-rounded) partials; fa_grad_accumulate equals the fp64 sum.
+* The ring of R ranks, emulated on one GPU (each rank's slices in its own
+  buffers, the exchange a device copy), run through the library's kernels
+  (fa_fwd / fa_bwd per slice pair, the merge and accumulate kernels), equals
+  the oracle's attention over the whole sequence within the bf16 tolerances
+  of the other parity tests, and gives the same bits on every run.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_io_aware_89_b200 as fa
+import oracle
+from exact_io_aware_89_b200 import ring
+from parity_utils import TOL_BF16, compare_lse, half_ulp, o_error, rel_fro
+from seeded_inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _need_cuda(cuda_ok):
+    return cuda_ok
+
+
+@pytest.mark.parametrize("S,d", [(1, 64), (2, 128), (4, 128), (3, 256)])
+def test_lse_merge_equals_the_oracle_merge(S, d):
+    dev = torch.device("cuda")
+    g = torch.Generator().manual_seed(100 + S)
+    B, Nq, H = 2, 77, 3
+    o_parts = [torch.randn((B, Nq, H, d), generator=g).to(torch.bfloat16) for _ in range(S)]
+    lse_parts = [(3.0 * torch.randn((B, H, Nq), generator=g)).float() for _ in range(S)]
+    # some rows see no key in some parts (lse = -inf, O = 0); row 0 of head 0 in none
+    for s in range(S):
+        dead = torch.rand((B, H, Nq), generator=g) < 0.2
+        dead[0, 0, 0] = True
+        lse_parts[s][dead] = -math.inf
+        o_parts[s].permute(0, 2, 1, 3)[dead] = 0
+    o_acc = torch.empty((B, Nq, H, d), dtype=torch.float32, device=dev)
+    lse_acc = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    out = torch.empty((B, Nq, H, d), dtype=torch.bfloat16, device=dev)
+    for s in range(S):
+        fa.lse_merge(o_acc, lse_acc, o_parts[s].to(dev), lse_parts[s].to(dev), first=(s == 0),
+                     out=out if s == S - 1 else None)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.merge_partials([x.double().numpy() for x in o_parts],
+                                           [x.double().numpy() for x in lse_parts])
+    compare_lse(lse_acc.cpu().numpy(), lse_ref, 1e-5, "merge")
+    # fp32 arithmetic on bf16 inputs: relative error a few units of 2^-24
+    assert np.abs(o_acc.cpu().numpy() - o_ref).max() <= 1e-5
+    assert o_error(out.float().cpu().numpy(), o_ref) <= 1e-5
+    assert not out.float()[0, 0, 0].any()
+
+
+def test_grad_accumulate_sums_in_fp32_and_rounds_once():
+    dev = torch.device("cuda")
+    g = torch.Generator().manual_seed(7)
+    n = 3 * 1000 * 8
+    parts = [torch.randn(n, generator=g).to(torch.bfloat16) for _ in range(5)]
+    acc = torch.empty(n, dtype=torch.float32, device=dev)
+    for s, p in enumerate(parts):
+        fa.grad_accumulate(acc, p.to(dev), first=(s == 0))
+    out = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    fa.grad_accumulate(acc, None, out=out)
+    torch.cuda.synchronize()
+    ref = sum(p.double().numpy() for p in parts)
+    assert np.abs(acc.cpu().numpy() - ref).max() <= 1e-5
+    assert (np.abs(out.float().cpu().numpy() - ref) <= half_ulp(ref) + 1e-5).all()
+
+
+CASES = [
+    # (R, B, n per rank, Hq, Hkv, d, causal)
+    (2, 1, 256, 2, 2, 128, True),
+    (4, 1, 192, 4, 2, 128, True),
+    (3, 2, 128, 2, 1, 64, False),
+    (4, 1, 160, 2, 2, 64, True),
+]
+
+
+def _run_ring(R, qs, ks, vs, dos, scale, causal):
+    os_, lses = ring.local_ring_forward(qs, ks, vs, scale=scale, causal=causal)
+    dq, dk, dv = ring.local_ring_backward(qs, ks, vs, os_, lses, dos, scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status(None) == 0
+    cat = lambda xs, ax: torch.cat(xs, dim=ax)
+    return cat(os_, 1), cat(lses, 2), cat(dq, 1), cat(dk, 1), cat(dv, 1)
+
+
+@pytest.mark.parametrize("R,B,n,Hq,Hkv,d,causal", CASES)
+def test_emulated_ring_equals_attention_over_the_whole_sequence(R, B, n, Hq, Hkv, d, causal):
+    N = R * n
+    inp = make_inputs(B, N, N, Hq, Hkv, d, 5000 + R * 10 + d)
+    scale = 1.0 / math.sqrt(d)
+    dev = torch.device("cuda")
+    x = {k_: t.to(dev) for k_, t in inp.items()}
+    sl = lambda t: [t[:, r * n:(r + 1) * n].contiguous() for r in range(R)]
+    qs, ks, vs, dos = sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["do"])
+    o, lse, dq, dk, dv = _run_ring(R, qs, ks, vs, dos, scale, causal)
+    f64 = {k_: t.double().numpy() for k_, t in inp.items()}
+    o_ref, lse_ref = oracle.attn_fwd(f64["q"], f64["k"], f64["v"], scale=scale, causal=causal)
+    what = "ring R%d B%d N%d Hq%d Hkv%d d%d causal%d" % (R, B, N, Hq, Hkv, d, causal)
+    err = o_error(o.float().cpu().numpy(), o_ref)
+    assert err <= TOL_BF16["o"], "%s: O err %.3e" % (what, err)
+    compare_lse(lse.cpu().numpy(), lse_ref, TOL_BF16["lse"], what)
+    refs = oracle.attn_bwd(f64["q"], f64["k"], f64["v"], f64["do"], scale=scale, causal=causal)
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
+        e = rel_fro(got.float().cpu().numpy(), ref)
+        assert e <= TOL_BF16["grad"], "%s: %s rel err %.3e" % (what, name, e)
+    # the same bits on a second run
+    again = _run_ring(R, qs, ks, vs, dos, scale, causal)
+    for a, b_ in zip((o, lse, dq, dk, dv), again):
+        assert torch.equal(a, b_)
