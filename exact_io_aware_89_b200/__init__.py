@@ -35,7 +35,7 @@ __all__ = [
     "KERNEL_KINDS", "attention_forward", "attention_backward", "attention_forward_splitkv",
     "attention_forward_kvcache", "attention_forward_varlen", "attention_backward_varlen",
     "fa_lse_merge", "fa_lse_merge_f16", "fa_grad_accumulate", "fa_grad_accumulate_f16",
-    "lse_merge", "grad_accumulate",
+    "lse_merge", "grad_accumulate", "fa_test_withhold_next_load",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -103,6 +103,8 @@ def load_library():
                  "fa_fwd_kvcache", "fa_fwd_blocksparse", "fa_bwd_blocksparse"):
         getattr(lib, base + "_f16").argtypes = getattr(lib, base).argtypes
         getattr(lib, base + "_f16").restype = i
+    lib.fa_test_withhold_next_load.argtypes = []
+    lib.fa_test_withhold_next_load.restype = i
     for name in ("fa_lse_merge", "fa_lse_merge_f16"):
         getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp]
         getattr(lib, name).restype = i
@@ -254,6 +256,12 @@ def fa_lse_merge_f16(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first
 def fa_grad_accumulate(acc, part, out, n, first, stream):
     """acc (fp32) = (first ? 0 : acc) + part (bf16); out (bf16) = rounded acc."""
     return load_library().fa_grad_accumulate(acc, part, out, n, first, stream)
+
+
+def fa_test_withhold_next_load():
+    """Test only: the next dense forward launch's first CTA withholds a key/value
+    load, so its bounded wait runs out (see include/fa.h)."""
+    return load_library().fa_test_withhold_next_load()
 
 
 def fa_grad_accumulate_f16(acc, part, out, n, first, stream):

@@ -58,6 +58,10 @@ struct TraceScope {
   }
 };
 
+// Test only: arms fa_test_withhold_next_load's one-shot for the next dense
+// forward launch.
+std::atomic<int> g_test_withhold{0};
+
 // A device-side wait gives up after this long (the kernels' own waits are
 // microseconds; the limit only matters when something is broken).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -170,6 +174,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   p.bm_sb = p.bm_sh = 0;
   p.bm_cols = 0;
   p.wait_limit_ns = kWaitLimitNs;
+  p.test_withhold = g_test_withhold.exchange(0);
   auto kern = fa_fwd_kernel<C>;
   if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
   const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
@@ -213,6 +218,7 @@ int launch_fwd_bs(const void* q, const void* k, const void* v, void* o, float* l
   p.bm_sh = sh;
   p.bm_cols = (Nk + kBlockSparseTile - 1) / kBlockSparseTile;
   p.wait_limit_ns = kWaitLimitNs;
+  p.test_withhold = 0;
   auto kern = fa_fwd_kernel<C, false, true>;
   if (smem_attr_once(kern, 232448, attr_done) != cudaSuccess) return FA_ERR_CUDA;
   const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
@@ -249,6 +255,7 @@ int launch_fwd_varlen(const void* q, const void* k, const void* v, void* o, floa
   p.bm_sb = p.bm_sh = 0;
   p.bm_cols = 0;
   p.wait_limit_ns = kWaitLimitNs;
+  p.test_withhold = 0;
   auto kern = fa_fwd_kernel<C, true>;
   if (smem_attr_once(kern, C::SMEM_BYTES, attr_done) != cudaSuccess) return FA_ERR_CUDA;
   const long long grid = static_cast<long long>(p.n_qgroups) * B * Hq;
@@ -313,6 +320,17 @@ int side_stream(cudaStream_t caller, SideStream** out) {
   return FA_OK;
 }
 
+// The split backward runs dQ beside dK/dV while the smaller of the two grids
+// is at most this many waves (CTAs per SM).
+constexpr long long kOverlapWaves = 4;
+
+int current_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
 // Packed sequences of a backward call (all null / 0 when dense).
 struct Varlen {
   const int* cu_q = nullptr;
@@ -342,8 +360,16 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   const long long kv_smem =
       CKV::SMEM_BYTES + (BS ? 4ll * (Hq / Hkv) * ((Nq + CKV::BM - 1) / CKV::BM + 1) : 0);
   if (dq_smem > 232448 || kv_smem > 232448) return FA_ERR_UNSUPPORTED;
+  // dQ beside dK/dV pays off while one of the kernels runs few waves (the
+  // other kernel's CTAs fill its partial waves: the training shape, GQA with a
+  // window); when both run many waves they only compete for the SMs and for
+  // L2 (32 heads at N = 8192: 7% slower side by side), and they run one after
+  // the other
+  const long long dq_ctas = static_cast<long long>((Nq + CQ::NQT * CQ::BM - 1) / (CQ::NQT * CQ::BM)) * B * Hq;
+  const long long kv_ctas = static_cast<long long>((Nk + CKV::BN - 1) / CKV::BN) * B * Hkv * (CQ::D / CKV::DV);
+  const bool overlap = (dq_ctas < kv_ctas ? dq_ctas : kv_ctas) <= kOverlapWaves * static_cast<long long>(current_sm_count());
   SideStream* side = nullptr;
-  if (side_stream(stream, &side) != FA_OK) return FA_ERR_CUDA;
+  if (overlap && side_stream(stream, &side) != FA_OK) return FA_ERR_CUDA;
   std::unique_lock<std::mutex> side_lock;
   if (side != nullptr) side_lock = std::unique_lock<std::mutex>(side->mu);
   TraceScope whole(FA_KERNEL_BWD_CALL, stream);  // ends after the join below
@@ -498,13 +524,6 @@ int plan_decode(int B, int Nq, int Hq, int Hkv, int d, const MaskSpec& m, int n_
   pl->n_splits = tiles > 0 ? (tiles + pl->split_tiles - 1) / pl->split_tiles : 1;
   if (pl->units * pl->n_splits > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
   return FA_OK;
-}
-
-int current_sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
 }
 
 // Workspace of a split call: the partial O rows (fp32), their LSE, then one
@@ -1164,6 +1183,11 @@ int fa_grad_accumulate(float* acc, const void* part, void* out, long long n, int
 }
 int fa_grad_accumulate_f16(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream) {
   return grad_accumulate_impl<true>(acc, part, out, n, first, stream);
+}
+
+int fa_test_withhold_next_load(void) {
+  g_test_withhold.store(1);
+  return FA_OK;
 }
 
 int fa_get_device_status(fa_stream_t stream) {

@@ -57,6 +57,10 @@ struct FwdParams {
   long long bm_sb, bm_sh;
   int bm_cols;
   unsigned long long wait_limit_ns;
+  // test only (fa_test_withhold_next_load): the producer of CTA 0 issues no
+  // key/value load after its first ring stages, so the MMA thread's bounded
+  // wait for the next one runs out; 0 in every ordinary launch
+  int test_withhold;
 };
 
 template <int D_, int NQT_, int BN_, int KST_, int NPOLY_ = 2, bool SPLITP_ = false>
@@ -325,6 +329,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       // Q and key tiles 0 .. n_pre-1 were issued before the block-wide sync
       int nk = n_pre, nv = NQT == 1 ? n_pre : 0;
       for (int it = n_pre; it < n_kv; ++it) {
+        if (p.test_withhold && blockIdx.x == 0) break;  // test only: key tile `it` is never loaded
         const int s = it % KST, use = it / KST;
         // the stage is free once the last MMA reading the tile held there
         // before has completed (NQT == 2: K_j and V_j share the stage)

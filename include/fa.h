@@ -370,6 +370,19 @@ int fa_grad_accumulate_f16(float* acc, const void* part, void* out, long long n,
  */
 int fa_get_device_status(fa_stream_t stream);
 
+/*
+ * Test only (failure detection): arms a one-shot for the next dense fa_fwd /
+ * fa_fwd_f16 launch in this process, in which the producer of the first CTA
+ * issues no key/value load after its first ring stages.  That CTA's MMA
+ * thread then waits for a copy that never comes; its bounded wait (2 s) runs
+ * out, the CTA raises the device status word, waits for the copies it did
+ * issue and frees its tensor memory, and the launch ends normally with that
+ * CTA's output rows unwritten.  fa_get_device_status then returns
+ * FA_ERR_TIMEOUT; the context stays usable.  Nothing is faulted, trapped or
+ * hung.  Returns FA_OK.
+ */
+int fa_test_withhold_next_load(void);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);
 

@@ -30,7 +30,8 @@ def test_header_declares_the_expected_entry_points():
         "fa_bwd_f16", "fa_fwd_varlen_f16", "fa_bwd_varlen_f16", "fa_fwd_splitkv_f16", "fa_fwd_kvcache_f16",
         "fa_fwd_blocksparse", "fa_fwd_blocksparse_f16", "fa_bwd_blocksparse", "fa_bwd_blocksparse_f16",
         "fa_get_device_status", "fa_status_string", "fa_trace_enable", "fa_trace_read",
-        "fa_lse_merge", "fa_lse_merge_f16", "fa_grad_accumulate", "fa_grad_accumulate_f16"])
+        "fa_lse_merge", "fa_lse_merge_f16", "fa_grad_accumulate", "fa_grad_accumulate_f16",
+        "fa_test_withhold_next_load"])
 
 
 def test_kernel_kinds_match_the_header():
