@@ -313,34 +313,72 @@ def time_gpu(w, steps, warmup, world, rank, dev, with_e2e=True, with_trace=True)
     out = dict(step_ms=step_ms, fwd_ms=fwd_ms, trace_ms=trace_ms, trace_n=trace_n,
                clocks=clocks.summary())
 
-    # --- end to end through the public API: pinned host inputs in, results out
+    # --- end to end through the public API: pinned host inputs in, results
+    # out.  Every step copies its inputs from pinned host memory and reads O,
+    # LSE, dQ, dK and dV back; the copies run on their own streams (host to
+    # device and device to host use separate copy engines), so step i's
+    # kernels overlap step i+1's upload and step i-1's download, with two
+    # device buffer sets taking turns.
     if with_e2e:
         hin = {n: t.pin_memory() for n, t in host.items()}
-        hout = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
-        dbuf = {n: torch.empty_like(x[n]) for n in ("q", "k", "v", "do")}
+        names_out = ("o", "lse", "dq", "dk", "dv")
+        shapes_out = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+        hout = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in shapes_out.items()}
+        sets = []
+        for _ in range(2):
+            dbuf = {n: torch.empty_like(x[n]) for n in ("q", "k", "v", "do")}
+            dbuf.update({n: torch.empty_like(t) for n, t in shapes_out.items()})
+            sets.append(dbuf)
         h2d = sum(t.numel() * t.element_size() for t in hin.values())
         d2h = sum(t.numel() * t.element_size() for t in hout.values())
         e_steps = max(3, min(steps, 10))
-        eev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(e_steps)]
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()
+        in_done = [ev() for _ in range(e_steps)]
+        comp_done = [ev() for _ in range(e_steps)]
+        out_done = [ev() for _ in range(e_steps)]
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def e2e_step(b, out_b):
+            st = fa.fa_fwd(b["q"].data_ptr(), b["k"].data_ptr(), b["v"].data_ptr(), out_b["o"].data_ptr(),
+                           out_b["lse"].data_ptr(), B, N, N, H, Hkv, d, scale, c, wl, wr, sp)
+            if st:
+                raise fa.FAError("fa_fwd", st)
+            st = fa.fa_bwd(b["q"].data_ptr(), b["k"].data_ptr(), b["v"].data_ptr(), out_b["o"].data_ptr(),
+                           out_b["lse"].data_ptr(), b["do"].data_ptr(), out_b["dq"].data_ptr(),
+                           out_b["dk"].data_ptr(), out_b["dv"].data_ptr(), B, N, N, H, Hkv, d, scale, c, wl, wr,
+                           ws.data_ptr(), ws.numel(), sp)
+            if st:
+                raise fa.FAError("fa_bwd", st)
+
         barrier(world)
         torch.cuda.synchronize()
+        t_start.record(stream)
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
         for i in range(e_steps):
-            eev[i][0].record(stream)
-            for n in ("q", "k", "v", "do"):
-                dbuf[n].copy_(hin[n], non_blocking=True)
-            step(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["do"])
-            hout["o"].copy_(o, non_blocking=True)
-            hout["lse"].copy_(lse, non_blocking=True)
-            hout["dq"].copy_(dq, non_blocking=True)
-            hout["dk"].copy_(dk, non_blocking=True)
-            hout["dv"].copy_(dv, non_blocking=True)
-            eev[i][1].record(stream)
+            b = sets[i % 2]
+            if i >= 2:  # the set's previous step has been computed and read back
+                s_in.wait_event(out_done[i - 2])
+            with torch.cuda.stream(s_in):
+                for n in ("q", "k", "v", "do"):
+                    b[n].copy_(hin[n], non_blocking=True)
+                in_done[i].record(s_in)
+            stream.wait_event(in_done[i])
+            e2e_step(b, b)
+            comp_done[i].record(stream)
+            s_out.wait_event(comp_done[i])
+            with torch.cuda.stream(s_out):
+                for n in names_out:
+                    hout[n].copy_(b[n], non_blocking=True)
+                out_done[i].record(s_out)
+        stream.wait_event(out_done[e_steps - 1])
+        t_end.record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        out["e2e_ms"] = [a.elapsed_time(b) for a, b in eev]
+        out["e2e_ms"] = [t_start.elapsed_time(t_end) / e_steps] * e_steps
         out["h2d"], out["d2h"] = h2d, d2h
+        del sets
     if fa.fa_get_device_status(None) != 0:
         raise RuntimeError("device status reports a timed-out wait")
     del flush
@@ -950,6 +988,66 @@ def run_blocksparse(args, local):
         torch.cuda.empty_cache()
 
 
+def run_ring(args, world, rank, local):
+    """Ring (context-parallel) attention on the long wide workload: the one
+    sequence split into equal slices, fwd+bwd of the whole sequence per step.
+    Under torchrun (N ranks, NCCL) each rank holds one slice and the slices
+    travel between GPUs (strong scaling; time = max over ranks); on one GPU,
+    --ring R emulates R ranks (each with its own buffers, the exchange a device
+    copy), which measures what the split itself costs next to the plain call.
+    One JSON line (rank 0)."""
+    import torch
+    import exact_io_aware_89_b200 as fa
+    from exact_io_aware_89_b200 import ring
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS["wide"]
+    R = world if world > 1 else args.ring
+    if w["N"] % R:
+        raise SystemExit("the sequence does not split into %d equal slices" % R)
+    n = w["N"] // R
+    x, _ = make_device_inputs(w, 0, dev)  # the same sequence on every rank; each takes its slice
+    sl = lambda t, r: t[:, r * n:(r + 1) * n].contiguous()
+    causal = w["causal"]
+    flush = L2Flush(dev)
+    if world > 1:
+        q, k, v, do = (sl(x[name], rank) for name in ("q", "k", "v", "do"))
+
+        def step():
+            o, lse = ring.ring_attention_forward(q, k, v, causal=causal)
+            ring.ring_attention_backward(q, k, v, o, lse, do, causal=causal)
+    else:
+        qs, ks, vs, dos = ([sl(x[name], r) for r in range(R)] for name in ("q", "k", "v", "do"))
+
+        def step():
+            os_, lses = ring.local_ring_forward(qs, ks, vs, causal=causal)
+            ring.local_ring_backward(qs, ks, vs, os_, lses, dos, causal=causal)
+    del x
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    if fa.fa_get_device_status(None) != 0:
+        raise RuntimeError("device status reports a timed-out wait")
+    t_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
+    F = fwd_flops(w)
+    if rank == 0:
+        line = {"ring": w["name"], "ranks": R, "emulated_on_one_gpu": world == 1,
+                "scaling": "strong (one sequence split over the ranks)",
+                "ms_per_step": round(t_ms / args.steps, 4),
+                "fwd_bwd_tflops": round(3.5 * F * args.steps / (t_ms * 1e-3) / 1e12, 2),
+                "slice_rows": n}
+        print(json.dumps(line), flush=True)
+
+
 def run_ours(args, world, rank, local):
     import torch
     dev = torch.device("cuda", local)
@@ -1050,6 +1148,9 @@ def main(argv=None):
                     help="with --sweep: the element type of the inputs (bf16 or fp16 entry points)")
     ap.add_argument("--sweep-filter", default=None,
                     help="with --sweep: only workloads whose name contains this text")
+    ap.add_argument("--ring", type=int, default=0,
+                    help="instead of the benchmark line: ring (context-parallel) attention on the long wide "
+                         "workload, over the torchrun ranks, or with N emulated ranks on one GPU")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the benchmark line: the sequence-length sweep and the GQA/window "
                          "and d=256 workloads, fwd / bwd / fwd+bwd timed separately, one JSON line each")
@@ -1057,6 +1158,20 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     world, rank, local = dist_setup(args)
+    if args.ring:
+        if world > 1:
+            import datetime
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        try:
+            run_ring(args, world, rank, local)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     if args.sweep or args.decode or args.varlen or args.blocksparse:
         if world > 1:
             raise SystemExit("--sweep, --decode, --varlen and --blocksparse run on one GPU")
