@@ -317,21 +317,23 @@ def time_gpu(w, steps, warmup, world, rank, dev, with_e2e=True, with_trace=True)
     # out.  Every step copies its inputs from pinned host memory and reads O,
     # LSE, dQ, dK and dV back; the copies run on their own streams (host to
     # device and device to host use separate copy engines), so step i's
-    # kernels overlap step i+1's upload and step i-1's download, with two
-    # device buffer sets taking turns.
+    # kernels overlap step i+1's upload and step i-1's download, with three
+    # device buffer sets taking turns (with two, each set's upload, kernels and
+    # download would form one serial chain).
     if with_e2e:
         hin = {n: t.pin_memory() for n, t in host.items()}
         names_out = ("o", "lse", "dq", "dk", "dv")
         shapes_out = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
         hout = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in shapes_out.items()}
+        NSETS = 3
         sets = []
-        for _ in range(2):
+        for _ in range(NSETS):
             dbuf = {n: torch.empty_like(x[n]) for n in ("q", "k", "v", "do")}
             dbuf.update({n: torch.empty_like(t) for n, t in shapes_out.items()})
             sets.append(dbuf)
         h2d = sum(t.numel() * t.element_size() for t in hin.values())
         d2h = sum(t.numel() * t.element_size() for t in hout.values())
-        e_steps = max(3, min(steps, 10))
+        e_steps = max(6, min(steps, 12))
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
         ev = lambda: torch.cuda.Event()
         in_done = [ev() for _ in range(e_steps)]
@@ -357,9 +359,9 @@ def time_gpu(w, steps, warmup, world, rank, dev, with_e2e=True, with_trace=True)
         s_in.wait_stream(stream)
         s_out.wait_stream(stream)
         for i in range(e_steps):
-            b = sets[i % 2]
-            if i >= 2:  # the set's previous step has been computed and read back
-                s_in.wait_event(out_done[i - 2])
+            b = sets[i % NSETS]
+            if i >= NSETS:  # the set's previous step has been computed and read back
+                s_in.wait_event(out_done[i - NSETS])
             with torch.cuda.stream(s_in):
                 for n in ("q", "k", "v", "do"):
                     b[n].copy_(hin[n], non_blocking=True)
