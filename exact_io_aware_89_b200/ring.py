@@ -28,7 +28,7 @@ The slices land in this rank's own memory before any kernel reads them
 (NCCL point-to-point sends / receives through torch.distributed, or copies
 in the single-process emulation); no kernel reads another GPU's memory.
 
-Two drivers share the per-rank steps: ``ring_attention_forward`` /
+Two sets of entry points share the per-rank steps: ``ring_attention_forward`` /
 ``ring_attention_backward`` run one rank of a torch.distributed process group
 (the exchange of step t + 1's slice overlaps step t's kernels);
 ``local_ring_forward`` / ``local_ring_backward`` run all R ranks in one

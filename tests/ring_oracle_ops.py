@@ -1,5 +1,5 @@
-"""Block computations of the ring driver done by the fp64 oracle, on CPU torch
-tensors: the CPU tests run the driver's schedule (and, with gloo ranks, its
+"""Block computations of the ring schedule done by the fp64 oracle, on CPU torch
+tensors: the CPU tests run the ring schedule (and, with gloo ranks, its
 point-to-point exchange) with these in place of the library's kernels.
 Test-only."""
 import numpy as np

@@ -1,4 +1,4 @@
-"""Ring (context-parallel) attention on the CPU: the driver's schedule with the
+"""Ring (context-parallel) attention on the CPU: the ring schedule with the
 fp64 oracle doing each block (tests/ring_oracle_ops.py), checked against the
 oracle over the whole sequence; the block masks against brute force; and the
 point-to-point exchange through two and three gloo ranks."""
