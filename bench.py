@@ -1005,25 +1005,29 @@ def run_ring(args, world, rank, local):
     torch.cuda.set_device(dev)
     w = WORKLOADS["wide"]
     R = world if world > 1 else args.ring
-    if w["N"] % R:
-        raise SystemExit("the sequence does not split into %d equal slices" % R)
+    layout = args.ring_layout
+    n_chunks = R if layout == "contiguous" else 2 * R
+    if w["N"] % n_chunks:
+        raise SystemExit("the sequence does not split into %d equal chunks" % n_chunks)
+    c = w["N"] // n_chunks
     n = w["N"] // R
-    x, _ = make_device_inputs(w, 0, dev)  # the same sequence on every rank; each takes its slice
-    sl = lambda t, r: t[:, r * n:(r + 1) * n].contiguous()
+    x, _ = make_device_inputs(w, 0, dev)  # the same sequence on every rank; each takes its rows
+    sl = lambda t, r: torch.cat([t[:, i * c:(i + 1) * c] for i in ring.rank_chunks(r, R, layout)],
+                                dim=1).contiguous()
     causal = w["causal"]
     flush = L2Flush(dev)
     if world > 1:
         q, k, v, do = (sl(x[name], rank) for name in ("q", "k", "v", "do"))
 
         def step():
-            o, lse = ring.ring_attention_forward(q, k, v, causal=causal)
-            ring.ring_attention_backward(q, k, v, o, lse, do, causal=causal)
+            o, lse = ring.ring_attention_forward(q, k, v, causal=causal, layout=layout)
+            ring.ring_attention_backward(q, k, v, o, lse, do, causal=causal, layout=layout)
     else:
         qs, ks, vs, dos = ([sl(x[name], r) for r in range(R)] for name in ("q", "k", "v", "do"))
 
         def step():
-            os_, lses = ring.local_ring_forward(qs, ks, vs, causal=causal)
-            ring.local_ring_backward(qs, ks, vs, os_, lses, dos, causal=causal)
+            os_, lses = ring.local_ring_forward(qs, ks, vs, causal=causal, layout=layout)
+            ring.local_ring_backward(qs, ks, vs, os_, lses, dos, causal=causal, layout=layout)
     del x
     for _ in range(args.warmup):
         step()
@@ -1042,7 +1046,7 @@ def run_ring(args, world, rank, local):
     t_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
     F = fwd_flops(w)
     if rank == 0:
-        line = {"ring": w["name"], "ranks": R, "emulated_on_one_gpu": world == 1,
+        line = {"ring": w["name"], "ranks": R, "layout": layout, "emulated_on_one_gpu": world == 1,
                 "scaling": "strong (one sequence split over the ranks)",
                 "ms_per_step": round(t_ms / args.steps, 4),
                 "fwd_bwd_tflops": round(3.5 * F * args.steps / (t_ms * 1e-3) / 1e12, 2),
@@ -1153,6 +1157,9 @@ def main(argv=None):
     ap.add_argument("--ring", type=int, default=0,
                     help="instead of the benchmark line: ring (context-parallel) attention on the long wide "
                          "workload, over the torchrun ranks, or with N emulated ranks on one GPU")
+    ap.add_argument("--ring-layout", choices=["contiguous", "zigzag"], default="zigzag",
+                    help="with --ring: each rank's chunk of the sequence ('contiguous') or two chunks, one "
+                         "from each end ('zigzag', the same causal work on every rank)")
     ap.add_argument("--sweep", action="store_true",
                     help="instead of the benchmark line: the sequence-length sweep and the GQA/window "
                          "and d=256 workloads, fwd / bwd / fwd+bwd timed separately, one JSON line each")

@@ -2,17 +2,21 @@
 ranks (zocula.com fla guide, the flame bullets and the glossary entry on
 context parallelism: long contexts are divided over several GPUs).
 
-Rank r of R holds rows [r n, (r + 1) n) of q, k, v (and o, lse, dO for the
-backward), n = N / R.  It keeps its query rows; the key/value slices travel
-around the ring, rank r passing what it holds to rank r + 1 after each step,
-so at step t it holds slice (r - t) mod R.  Each (query slice, key slice)
-pair is an ordinary attention call of the library:
+The sequence of N rows is cut into equal chunks.  In the 'contiguous'
+layout rank r of R holds chunk r of R (rows [r n, (r + 1) n), n = N / R); in
+the 'zigzag' layout it holds chunks r and 2R - 1 - r of 2R, one from each end,
+so that under a causal mask every rank has the same work at every step (with
+contiguous chunks rank R - 1 does 2R - 1 times rank 0's work).  A
+rank keeps its query rows (and o, lse, dO for the backward); the key/value
+chunks travel around the ring, rank r passing what it holds to rank r + 1
+after each step, so at step t it holds rank (r - t) mod R's.  Each (query
+chunk, key chunk) pair is an ordinary attention call of the library:
 
-* causal: the diagonal pair (slice r) is causal attention of two equal
-  slices; slices before it are seen whole; slices after it are hidden and
-  skipped (the plain reading of "causal" for the whole sequence, i.e. key j
-  visible to query i iff j <= i, split into blocks).  Non-causal: every pair
-  is seen whole.  Sliding windows are not supported here.
+* causal: the diagonal pair (a chunk against itself) is causal attention of
+  two equal chunks; earlier key chunks are seen whole; later ones are hidden
+  and skipped (the plain reading of "causal" for the whole sequence, i.e.
+  key j visible to query i iff j <= i, split into blocks).  Non-causal: every
+  pair is seen whole.  Sliding windows are not supported here.
 * forward: fa_fwd gives each pair's (O_t, LSE_t); fa_lse_merge folds them,
   in step order, into an fp32 running result (abeam.tech FlashAttention
   summary, "computing softmax blockwise correctly", applied to whole key
@@ -38,16 +42,44 @@ process, the exchange being a copy (tests, and single-GPU measurement).
 """
 import math
 
-__all__ = ["block_mode", "LibraryOps", "ForwardRank", "BackwardRank", "ring_attention_forward",
-           "ring_attention_backward", "local_ring_forward", "local_ring_backward"]
+__all__ = ["block_mode", "rank_chunks", "LibraryOps", "ForwardRank", "BackwardRank",
+           "ring_attention_forward", "ring_attention_backward", "local_ring_forward", "local_ring_backward"]
+
+LAYOUTS = ("contiguous", "zigzag")
 
 
-def block_mode(r, src, causal):
-    """How query slice r attends to key slice src of an equal split:
-    'full', 'causal' (the diagonal pair) or None (every key hidden)."""
-    if not causal or src < r:
+def block_mode(qc, kc, causal):
+    """How query chunk qc attends to key chunk kc of an equal split of the
+    sequence: 'full', 'causal' (the diagonal pair) or None (every key hidden)."""
+    if not causal or kc < qc:
         return "full"
-    return "causal" if src == r else None
+    return "causal" if kc == qc else None
+
+
+def rank_chunks(r, R, layout="contiguous"):
+    """The sequence chunks rank r of R holds, in its row order.  'contiguous':
+    the r-th of R equal chunks.  'zigzag': chunks r and 2R - 1 - r of 2R, which
+    gives every rank the same causal work at every step."""
+    if layout == "contiguous":
+        return [r]
+    if layout == "zigzag":
+        return [r, 2 * R - 1 - r]
+    raise ValueError("layout must be one of %s" % (LAYOUTS,))
+
+
+def _split(x, n, dim=1):
+    """The rank's rows as n equal chunks, each a contiguous tensor."""
+    if n == 1:
+        return [x]
+    size = x.shape[dim] // n
+    return [x.narrow(dim, i * size, size).contiguous() for i in range(n)]
+
+
+def _join(xs, dim=1):
+    if len(xs) == 1:
+        return xs[0]
+    import torch
+    return torch.cat(xs, dim=dim)
 
 
 class LibraryOps:
@@ -91,54 +123,86 @@ class LibraryOps:
         return out
 
 
+def _schedule(r, R, layout, causal):
+    """[(t, query chunk position, key chunk position, mode)] of rank r's
+    visible pairs, in the order they are computed: steps, then query chunks,
+    then key chunks."""
+    mine = rank_chunks(r, R, layout)
+    out = []
+    for t in range(R):
+        theirs = rank_chunks((r - t) % R, R, layout)
+        for i, qc in enumerate(mine):
+            for j, kc in enumerate(theirs):
+                mode = block_mode(qc, kc, causal)
+                if mode is not None:
+                    out.append((t, i, j, mode))
+    return out
+
+
 class ForwardRank:
-    """Rank r's forward steps: step(t, k_slice, v_slice) for t = 0 .. R - 1,
-    then result() -> (o, lse) of its query rows over the whole sequence."""
+    """Rank r's forward steps: step(t, k_chunks, v_chunks) for t = 0 .. R - 1
+    with the key/value chunks held at step t, then result() -> (o, lse) of its
+    query rows over the whole sequence, in its row order."""
 
-    def __init__(self, r, R, q, ops, scale, causal):
-        self.r, self.R, self.q, self.ops = r, R, q, ops
-        self.scale, self.causal = scale, causal
-        active = [t for t in range(R) if block_mode(r, (r - t) % R, causal)]
-        self.last = active[-1]  # always >= 0: the diagonal pair (t = 0) is seen
-        self.o_acc, self.lse_acc = ops.new_fwd_acc(q)
-        self.out = ops.new_out(q)
-        self.first = True
+    def __init__(self, r, R, q, ops, scale, causal, layout="contiguous"):
+        self.r, self.R, self.ops = r, R, ops
+        self.scale, self.causal, self.layout = scale, causal, layout
+        self.qs = _split(q, len(rank_chunks(r, R, layout)))
+        self.sched = _schedule(r, R, layout, causal)
+        # the last pair of each query chunk writes its rounded output
+        self.last = {}
+        for t, i, j, _ in self.sched:
+            self.last[i] = (t, j)
+        self.acc = [ops.new_fwd_acc(x) for x in self.qs]
+        self.out = [ops.new_out(x) for x in self.qs]
+        self.first = [True] * len(self.qs)
 
-    def step(self, t, k, v):
-        mode = block_mode(self.r, (self.r - t) % self.R, self.causal)
-        if mode is None:
-            return
-        o_p, lse_p = self.ops.fwd(self.q, k, v, self.scale, mode == "causal")
-        self.ops.merge(self.o_acc, self.lse_acc, o_p, lse_p, self.first, self.out if t == self.last else None)
-        self.first = False
+    def step(self, t, ks, vs):
+        for tt, i, j, mode in self.sched:
+            if tt != t:
+                continue
+            o_p, lse_p = self.ops.fwd(self.qs[i], ks[j], vs[j], self.scale, mode == "causal")
+            o_acc, lse_acc = self.acc[i]
+            self.ops.merge(o_acc, lse_acc, o_p, lse_p, self.first[i],
+                           self.out[i] if self.last[i] == (t, j) else None)
+            self.first[i] = False
 
     def result(self):
-        return self.out, self.lse_acc
+        return _join(self.out, 1), _join([lse for _, lse in self.acc], 2)
 
 
 class BackwardRank:
-    """Rank r's backward steps.  step(t, k, v, dk_acc, dv_acc) adds the pair's
-    shares: dQ into this rank's accumulator, dK / dV into the travelling
-    accumulators of the key slice (the slice's owner initialises them at
-    t = 0, the diagonal pair, which every rank computes)."""
+    """Rank r's backward steps.  step(t, k_chunks, v_chunks, dk_accs,
+    dv_accs) adds each visible pair's shares: dQ into this rank's
+    accumulators, dK / dV into the travelling accumulators of the key chunks
+    (every rank computes the diagonal pairs of its own chunks at t = 0, so the
+    owner initialises them then)."""
 
-    def __init__(self, r, R, q, o, lse, do, ops, scale, causal):
-        self.r, self.R = r, R
-        self.q, self.o, self.lse, self.do = q, o, lse, do
-        self.ops, self.scale, self.causal = ops, scale, causal
-        self.dq_acc = ops.new_grad_acc(q)
+    def __init__(self, r, R, q, o, lse, do, ops, scale, causal, layout="contiguous"):
+        n = len(rank_chunks(r, R, layout))
+        self.r, self.R, self.ops = r, R, ops
+        self.scale, self.causal, self.layout = scale, causal, layout
+        self.qs, self.os, self.dos = _split(q, n), _split(o, n), _split(do, n)
+        self.lses = _split(lse, n, dim=2)
+        self.sched = _schedule(r, R, layout, causal)
+        self.dq_acc = [ops.new_grad_acc(x) for x in self.qs]
+        self.dq_first = [True] * n
 
-    def step(self, t, k, v, dk_acc, dv_acc):
-        mode = block_mode(self.r, (self.r - t) % self.R, self.causal)
-        if mode is None:
-            return
-        dq, dk, dv = self.ops.bwd(self.q, k, v, self.o, self.lse, self.do, self.scale, mode == "causal")
-        self.ops.accumulate(self.dq_acc, dq, t == 0)
-        self.ops.accumulate(dk_acc, dk, t == 0)
-        self.ops.accumulate(dv_acc, dv, t == 0)
+    def step(self, t, ks, vs, dk_accs, dv_accs):
+        kv_first = [t == 0] * len(ks)
+        for tt, i, j, mode in self.sched:
+            if tt != t:
+                continue
+            dq, dk, dv = self.ops.bwd(self.qs[i], ks[j], vs[j], self.os[i], self.lses[i], self.dos[i],
+                                      self.scale, mode == "causal")
+            self.ops.accumulate(self.dq_acc[i], dq, self.dq_first[i])
+            self.ops.accumulate(dk_accs[j], dk, kv_first[j])
+            self.ops.accumulate(dv_accs[j], dv, kv_first[j])
+            self.dq_first[i] = False
+            kv_first[j] = False
 
     def dq(self):
-        return self.ops.finish_grad(self.dq_acc, self.q)
+        return _join([self.ops.finish_grad(a, x) for a, x in zip(self.dq_acc, self.qs)], 1)
 
 
 def _default_scale(q, scale):
@@ -147,39 +211,45 @@ def _default_scale(q, scale):
 
 # ------------------------------------------------------------ all ranks in one process
 
-def local_ring_forward(qs, ks, vs, scale=None, causal=False, ops=None):
-    """Forward of R ranks emulated in one process (lists of per-rank slices);
-    returns the lists of per-rank o and lse."""
+def local_ring_forward(qs, ks, vs, scale=None, causal=False, ops=None, layout="contiguous"):
+    """Forward of R ranks emulated in one process (lists of per-rank rows, in
+    each rank's row order for the layout); returns the lists of per-rank o and
+    lse."""
     ops = ops or LibraryOps()
     R = len(qs)
     scale = _default_scale(qs[0], scale)
-    ranks = [ForwardRank(r, R, qs[r], ops, scale, causal) for r in range(R)]
-    kv = [(ks[r], vs[r]) for r in range(R)]
+    n = len(rank_chunks(0, R, layout))
+    ranks = [ForwardRank(r, R, qs[r], ops, scale, causal, layout) for r in range(R)]
+    kv = [(_split(ks[r], n), _split(vs[r], n)) for r in range(R)]
     for t in range(R):
         for r in range(R):
             ranks[r].step(t, *kv[r])
-        if t < R - 1:  # rank r receives what rank r - 1 held, in its own buffer
-            kv = [(kv[(r - 1) % R][0].clone(), kv[(r - 1) % R][1].clone()) for r in range(R)]
+        if t < R - 1:  # rank r receives what rank r - 1 held, in its own buffers
+            kv = [tuple([x.clone() for x in part] for part in kv[(r - 1) % R]) for r in range(R)]
     res = [x.result() for x in ranks]
     return [o for o, _ in res], [lse for _, lse in res]
 
 
-def local_ring_backward(qs, ks, vs, os_, lses, dos, scale=None, causal=False, ops=None):
+def local_ring_backward(qs, ks, vs, os_, lses, dos, scale=None, causal=False, ops=None, layout="contiguous"):
     """Backward of R ranks emulated in one process; returns lists of per-rank
-    dq, dk, dv (each rank's own slices)."""
+    dq, dk, dv (each rank's own rows, in its row order)."""
     ops = ops or LibraryOps()
     R = len(qs)
     scale = _default_scale(qs[0], scale)
-    ranks = [BackwardRank(r, R, qs[r], os_[r], lses[r], dos[r], ops, scale, causal) for r in range(R)]
-    carry = [(ks[r], vs[r], ops.new_grad_acc(ks[r]), ops.new_grad_acc(vs[r])) for r in range(R)]
+    n = len(rank_chunks(0, R, layout))
+    ranks = [BackwardRank(r, R, qs[r], os_[r], lses[r], dos[r], ops, scale, causal, layout) for r in range(R)]
+    carry = []
+    for r in range(R):
+        kc, vc = _split(ks[r], n), _split(vs[r], n)
+        carry.append((kc, vc, [ops.new_grad_acc(x) for x in kc], [ops.new_grad_acc(x) for x in vc]))
     for t in range(R):
         for r in range(R):
             ranks[r].step(t, *carry[r])
-        # every slice moves on; after the last step this returns it to its owner
-        carry = [tuple(x.clone() for x in carry[(r - 1) % R]) for r in range(R)]
+        # every chunk moves on; after the last step this returns it to its owner
+        carry = [tuple([x.clone() for x in part] for part in carry[(r - 1) % R]) for r in range(R)]
     dq = [x.dq() for x in ranks]
-    dk = [ops.finish_grad(carry[r][2], ks[r]) for r in range(R)]
-    dv = [ops.finish_grad(carry[r][3], vs[r]) for r in range(R)]
+    dk = [_join([ops.finish_grad(a, x) for a, x in zip(carry[r][2], carry[r][0])], 1) for r in range(R)]
+    dv = [_join([ops.finish_grad(a, x) for a, x in zip(carry[r][3], carry[r][1])], 1) for r in range(R)]
     return dq, dk, dv
 
 
@@ -206,41 +276,50 @@ def _wait(reqs):
         q.wait()
 
 
-def ring_attention_forward(q, k, v, scale=None, causal=False, group=None, ops=None):
-    """This rank's (o, lse) of ring attention over a torch.distributed group.
-    The next key/value slice is exchanged while this step's kernels run."""
+def ring_attention_forward(q, k, v, scale=None, causal=False, group=None, ops=None, layout="contiguous"):
+    """This rank's (o, lse) of ring attention over a torch.distributed group,
+    its rows in the layout's order.  The next key/value chunks are exchanged
+    while this step's kernels run."""
     import torch.distributed as dist
     ops = ops or LibraryOps()
     R, r = dist.get_world_size(group), dist.get_rank(group)
-    me = ForwardRank(r, R, q, ops, _default_scale(q, scale), causal)
-    kv = (k, v)
+    n = len(rank_chunks(r, R, layout))
+    me = ForwardRank(r, R, q, ops, _default_scale(q, scale), causal, layout)
+    kc, vc = _split(k, n), _split(v, n)
     for t in range(R):
-        pending = _shift(kv, group) if t < R - 1 else None
-        me.step(t, *kv)
+        pending = _shift(kc + vc, group) if t < R - 1 else None
+        me.step(t, kc, vc)
         if pending is not None:
             _wait(pending[0])
-            kv = tuple(pending[1])
+            kc, vc = pending[1][:n], pending[1][n:]
     return me.result()
 
 
-def ring_attention_backward(q, k, v, o, lse, do, scale=None, causal=False, group=None, ops=None):
+def ring_attention_backward(q, k, v, o, lse, do, scale=None, causal=False, group=None, ops=None,
+                            layout="contiguous"):
     """This rank's (dq, dk, dv) of ring attention over a torch.distributed
     group: dq of its query rows, dk / dv of its own key/value rows (summed
-    over every rank's queries).  The next key/value slice is exchanged while
-    this step's kernels run; the dK / dV accumulators follow after the step."""
+    over every rank's queries), in the layout's row order.  The next
+    key/value chunks are exchanged while this step's kernels run; the dK / dV
+    accumulators follow after the step."""
     import torch.distributed as dist
     ops = ops or LibraryOps()
     R, r = dist.get_world_size(group), dist.get_rank(group)
-    me = BackwardRank(r, R, q, o, lse, do, ops, _default_scale(q, scale), causal)
-    kv = (k, v)
-    acc = (ops.new_grad_acc(k), ops.new_grad_acc(v))
+    n = len(rank_chunks(r, R, layout))
+    me = BackwardRank(r, R, q, o, lse, do, ops, _default_scale(q, scale), causal, layout)
+    kc, vc = _split(k, n), _split(v, n)
+    dk_acc = [ops.new_grad_acc(x) for x in kc]
+    dv_acc = [ops.new_grad_acc(x) for x in vc]
     for t in range(R):
-        pending = _shift(kv, group) if t < R - 1 else None
-        me.step(t, kv[0], kv[1], acc[0], acc[1])
-        reqs, got = _shift(acc, group)
+        pending = _shift(kc + vc, group) if t < R - 1 else None
+        me.step(t, kc, vc, dk_acc, dv_acc)
+        reqs, got = _shift(dk_acc + dv_acc, group)
         _wait(reqs)
-        acc = tuple(got)
+        dk_acc, dv_acc = got[:n], got[n:]
         if pending is not None:
             _wait(pending[0])
-            kv = tuple(pending[1])
-    return me.dq(), ops.finish_grad(acc[0], k), ops.finish_grad(acc[1], v)
+            kc, vc = pending[1][:n], pending[1][n:]
+    like_k = _split(k, n)
+    dk = _join([ops.finish_grad(a, x) for a, x in zip(dk_acc, like_k)], 1)
+    dv = _join([ops.finish_grad(a, x) for a, x in zip(dv_acc, like_k)], 1)
+    return me.dq(), dk, dv

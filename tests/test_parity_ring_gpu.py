@@ -74,36 +74,57 @@ def test_grad_accumulate_sums_in_fp32_and_rounds_once():
 
 
 CASES = [
-    # (R, B, n per rank, Hq, Hkv, d, causal)
-    (2, 1, 256, 2, 2, 128, True),
-    (4, 1, 192, 4, 2, 128, True),
-    (3, 2, 128, 2, 1, 64, False),
-    (4, 1, 160, 2, 2, 64, True),
+    # (R, B, n per rank, Hq, Hkv, d, causal, layout)
+    (2, 1, 256, 2, 2, 128, True, "contiguous"),
+    (4, 1, 192, 4, 2, 128, True, "contiguous"),
+    (3, 2, 128, 2, 1, 64, False, "contiguous"),
+    (4, 1, 160, 2, 2, 64, True, "contiguous"),
+    (2, 1, 256, 2, 2, 128, True, "zigzag"),
+    (4, 2, 192, 4, 2, 128, True, "zigzag"),
+    (3, 1, 128, 2, 2, 64, True, "zigzag"),
 ]
 
 
-def _run_ring(R, qs, ks, vs, dos, scale, causal):
-    os_, lses = ring.local_ring_forward(qs, ks, vs, scale=scale, causal=causal)
-    dq, dk, dv = ring.local_ring_backward(qs, ks, vs, os_, lses, dos, scale=scale, causal=causal)
+def _rank_rows(x, R, layout):
+    """Each rank's rows of the whole-sequence tensor x (dim 1), in its order."""
+    n_chunks = R if layout == "contiguous" else 2 * R
+    c = x.shape[1] // n_chunks
+    return [torch.cat([x[:, i * c:(i + 1) * c] for i in ring.rank_chunks(r, R, layout)], dim=1).contiguous()
+            for r in range(R)]
+
+
+def _whole(xs, R, layout, dim=1):
+    """The whole sequence back from the ranks' rows."""
+    per = len(ring.rank_chunks(0, R, layout))
+    chunks = {}
+    for r in range(R):
+        parts = torch.chunk(xs[r], per, dim=dim)
+        for p, i in enumerate(ring.rank_chunks(r, R, layout)):
+            chunks[i] = parts[p]
+    return torch.cat([chunks[i] for i in sorted(chunks)], dim=dim)
+
+
+def _run_ring(R, qs, ks, vs, dos, scale, causal, layout):
+    os_, lses = ring.local_ring_forward(qs, ks, vs, scale=scale, causal=causal, layout=layout)
+    dq, dk, dv = ring.local_ring_backward(qs, ks, vs, os_, lses, dos, scale=scale, causal=causal, layout=layout)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status(None) == 0
-    cat = lambda xs, ax: torch.cat(xs, dim=ax)
-    return cat(os_, 1), cat(lses, 2), cat(dq, 1), cat(dk, 1), cat(dv, 1)
+    return (_whole(os_, R, layout), _whole(lses, R, layout, dim=2), _whole(dq, R, layout),
+            _whole(dk, R, layout), _whole(dv, R, layout))
 
 
-@pytest.mark.parametrize("R,B,n,Hq,Hkv,d,causal", CASES)
-def test_emulated_ring_equals_attention_over_the_whole_sequence(R, B, n, Hq, Hkv, d, causal):
+@pytest.mark.parametrize("R,B,n,Hq,Hkv,d,causal,layout", CASES)
+def test_emulated_ring_equals_attention_over_the_whole_sequence(R, B, n, Hq, Hkv, d, causal, layout):
     N = R * n
     inp = make_inputs(B, N, N, Hq, Hkv, d, 5000 + R * 10 + d)
     scale = 1.0 / math.sqrt(d)
     dev = torch.device("cuda")
     x = {k_: t.to(dev) for k_, t in inp.items()}
-    sl = lambda t: [t[:, r * n:(r + 1) * n].contiguous() for r in range(R)]
-    qs, ks, vs, dos = sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["do"])
-    o, lse, dq, dk, dv = _run_ring(R, qs, ks, vs, dos, scale, causal)
+    qs, ks, vs, dos = (_rank_rows(x[name], R, layout) for name in ("q", "k", "v", "do"))
+    o, lse, dq, dk, dv = _run_ring(R, qs, ks, vs, dos, scale, causal, layout)
     f64 = {k_: t.double().numpy() for k_, t in inp.items()}
     o_ref, lse_ref = oracle.attn_fwd(f64["q"], f64["k"], f64["v"], scale=scale, causal=causal)
-    what = "ring R%d B%d N%d Hq%d Hkv%d d%d causal%d" % (R, B, N, Hq, Hkv, d, causal)
+    what = "ring %s R%d B%d N%d Hq%d Hkv%d d%d causal%d" % (layout, R, B, N, Hq, Hkv, d, causal)
     err = o_error(o.float().cpu().numpy(), o_ref)
     assert err <= TOL_BF16["o"], "%s: O err %.3e" % (what, err)
     compare_lse(lse.cpu().numpy(), lse_ref, TOL_BF16["lse"], what)
@@ -112,6 +133,6 @@ def test_emulated_ring_equals_attention_over_the_whole_sequence(R, B, n, Hq, Hkv
         e = rel_fro(got.float().cpu().numpy(), ref)
         assert e <= TOL_BF16["grad"], "%s: %s rel err %.3e" % (what, name, e)
     # the same bits on a second run
-    again = _run_ring(R, qs, ks, vs, dos, scale, causal)
+    again = _run_ring(R, qs, ks, vs, dos, scale, causal, layout)
     for a, b_ in zip((o, lse, dq, dk, dv), again):
         assert torch.equal(a, b_)

@@ -22,6 +22,8 @@ def _visible(i, j, causal):
 @pytest.mark.parametrize("R", [1, 2, 3, 5])
 @pytest.mark.parametrize("causal", [False, True])
 def test_block_mode_matches_the_mask_of_the_whole_sequence(R, causal):
+    """Chunks r and src of an equal split (the contiguous layout's chunks, the
+    zig-zag layout's are the same function of the chunk indices)."""
     n = 4
     for r in range(R):
         for src in range(R):
@@ -44,30 +46,67 @@ def _inputs(B, N, Hq, Hkv, d, seed):
     return q, k, v, do
 
 
-def _split(x, R):
-    n = x.shape[1] // R
-    return [torch.from_numpy(np.ascontiguousarray(x[:, r * n:(r + 1) * n])) for r in range(R)]
+def _split(x, R, layout="contiguous"):
+    """Each rank's rows, in its row order for the layout (chunks along dim 1)."""
+    n_chunks = R if layout == "contiguous" else 2 * R
+    c = x.shape[1] // n_chunks
+    out = []
+    for r in range(R):
+        parts = [x[:, i * c:(i + 1) * c] for i in ring.rank_chunks(r, R, layout)]
+        out.append(torch.from_numpy(np.ascontiguousarray(np.concatenate(parts, axis=1))))
+    return out
 
 
+def _join(xs, R, layout="contiguous", dim=1):
+    """The whole sequence back from the ranks' rows."""
+    n_chunks = R if layout == "contiguous" else 2 * R
+    per = len(ring.rank_chunks(0, R, layout))
+    chunks = [None] * n_chunks
+    for r in range(R):
+        a = np.asarray(xs[r])
+        for p, i in enumerate(ring.rank_chunks(r, R, layout)):
+            c = a.shape[dim] // per
+            chunks[i] = np.take(a, range(p * c, (p + 1) * c), axis=dim)
+    return np.concatenate(chunks, axis=dim)
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
 @pytest.mark.parametrize("R,Hq,Hkv,causal", [(1, 2, 2, True), (2, 2, 2, True), (3, 4, 2, True),
                                               (4, 2, 1, False), (3, 2, 2, False)])
-def test_local_ring_equals_attention_over_the_whole_sequence(R, Hq, Hkv, causal):
-    B, n, d = 2, 5, 8
+def test_local_ring_equals_attention_over_the_whole_sequence(R, Hq, Hkv, causal, layout):
+    B, n, d = 2, 6, 8
     N = R * n
     q, k, v, do = _inputs(B, N, Hq, Hkv, d, seed=R * 10 + Hq)
     scale = 1.0 / math.sqrt(d)
     o_ref, lse_ref = oracle.attn_fwd(q, k, v, scale=scale, causal=causal)
     g_ref = oracle.attn_bwd(q, k, v, do, scale=scale, causal=causal)
     ops = OracleOps()
-    qs, ks, vs, dos = (_split(x, R) for x in (q, k, v, do))
-    os_, lses = ring.local_ring_forward(qs, ks, vs, scale=scale, causal=causal, ops=ops)
-    o = np.concatenate([x.numpy() for x in os_], axis=1)
-    lse = np.concatenate([x.numpy() for x in lses], axis=2)
-    np.testing.assert_allclose(o, o_ref, atol=1e-12)
-    np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
-    dq, dk, dv = ring.local_ring_backward(qs, ks, vs, os_, lses, dos, scale=scale, causal=causal, ops=ops)
+    qs, ks, vs, dos = (_split(x, R, layout) for x in (q, k, v, do))
+    os_, lses = ring.local_ring_forward(qs, ks, vs, scale=scale, causal=causal, ops=ops, layout=layout)
+    np.testing.assert_allclose(_join([x.numpy() for x in os_], R, layout), o_ref, atol=1e-12)
+    np.testing.assert_allclose(_join([x.numpy() for x in lses], R, layout, dim=2), lse_ref, atol=1e-12)
+    dq, dk, dv = ring.local_ring_backward(qs, ks, vs, os_, lses, dos, scale=scale, causal=causal, ops=ops,
+                                          layout=layout)
     for got, ref in zip((dq, dk, dv), g_ref):
-        np.testing.assert_allclose(np.concatenate([x.numpy() for x in got], axis=1), ref, atol=1e-11)
+        np.testing.assert_allclose(_join([x.numpy() for x in got], R, layout), ref, atol=1e-11)
+
+
+@pytest.mark.parametrize("R", [2, 3, 4, 8])
+def test_zigzag_gives_every_rank_the_same_causal_work_at_every_step(R):
+    """Visible (query chunk, key chunk) pairs per rank and step, counted in
+    units of a causal diagonal pair (half a full one): with the zig-zag layout
+    every rank does the same at every step; with contiguous chunks rank 0
+    does one diagonal pair in all and rank R - 1 does 2R - 1 times that."""
+    def work(layout):
+        w = np.zeros((R, R))
+        for r in range(R):
+            for t, i, j, mode in ring._schedule(r, R, layout, True):
+                w[r, t] += 1 if mode == "causal" else 2
+        return w
+    z = work("zigzag")
+    assert (z == z[0, 0]).all() and z[0, 0] == 4
+    c = work("contiguous").sum(axis=1)
+    assert c[0] == 1 and c[R - 1] == 2 * R - 1
 
 
 def _free_port():
@@ -78,33 +117,33 @@ def _free_port():
     return port
 
 
-def _rank_main(rank, world, port, causal, q_all, k_all, v_all, do_all, queue):
+def _rank_main(rank, world, port, causal, q_all, k_all, v_all, do_all, queue, layout="contiguous"):
     import datetime
     import torch.distributed as dist
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
-        n = q_all.shape[1] // world
-        sl = lambda x: torch.from_numpy(np.ascontiguousarray(x[:, rank * n:(rank + 1) * n]))
-        q, k, v, do = sl(q_all), sl(k_all), sl(v_all), sl(do_all)
+        q, k, v, do = (_split(x, world, layout)[rank] for x in (q_all, k_all, v_all, do_all))
         ops = OracleOps()
-        o, lse = ring.ring_attention_forward(q, k, v, causal=causal, ops=ops)
-        dq, dk, dv = ring.ring_attention_backward(q, k, v, o, lse, do, causal=causal, ops=ops)
+        o, lse = ring.ring_attention_forward(q, k, v, causal=causal, ops=ops, layout=layout)
+        dq, dk, dv = ring.ring_attention_backward(q, k, v, o, lse, do, causal=causal, ops=ops, layout=layout)
         dist.barrier()
         queue.put((rank, o.numpy(), lse.numpy(), dq.numpy(), dk.numpy(), dv.numpy()))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,causal", [(2, True), (3, True), (2, False)])
-def test_gloo_ranks_run_the_ring_exchange(world, causal):
+@pytest.mark.parametrize("world,causal,layout", [(2, True, "contiguous"), (3, True, "contiguous"),
+                                                 (2, False, "contiguous"), (2, True, "zigzag"),
+                                                 (3, True, "zigzag")])
+def test_gloo_ranks_run_the_ring_exchange(world, causal, layout):
     import torch.multiprocessing as mp
     B, n, Hq, Hkv, d = 1, 4, 2, 1, 8
     q, k, v, do = _inputs(B, world * n, Hq, Hkv, d, seed=77 + world)
     ctx = mp.get_context("spawn")
     queue = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, causal, q, k, v, do, queue))
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, causal, q, k, v, do, queue, layout))
              for r in range(world)]
     for p in procs:
         p.start()
@@ -115,7 +154,7 @@ def test_gloo_ranks_run_the_ring_exchange(world, causal):
     scale = 1.0 / math.sqrt(d)
     o_ref, lse_ref = oracle.attn_fwd(q, k, v, scale=scale, causal=causal)
     g_ref = oracle.attn_bwd(q, k, v, do, scale=scale, causal=causal)
-    np.testing.assert_allclose(np.concatenate([x[1] for x in out], axis=1), o_ref, atol=1e-12)
-    np.testing.assert_allclose(np.concatenate([x[2] for x in out], axis=2), lse_ref, atol=1e-12)
+    np.testing.assert_allclose(_join([x[1] for x in out], world, layout), o_ref, atol=1e-12)
+    np.testing.assert_allclose(_join([x[2] for x in out], world, layout, dim=2), lse_ref, atol=1e-12)
     for idx, ref in zip((3, 4, 5), g_ref):
-        np.testing.assert_allclose(np.concatenate([x[idx] for x in out], axis=1), ref, atol=1e-11)
+        np.testing.assert_allclose(_join([x[idx] for x in out], world, layout), ref, atol=1e-11)
