@@ -1024,10 +1024,14 @@ def run_ring(args, world, rank, local):
             ring.ring_attention_backward(q, k, v, o, lse, do, causal=causal, layout=layout)
     else:
         qs, ks, vs, dos = ([sl(x[name], r) for r in range(R)] for name in ("q", "k", "v", "do"))
+        timers = []
 
-        def step():
-            os_, lses = ring.local_ring_forward(qs, ks, vs, causal=causal, layout=layout)
-            ring.local_ring_backward(qs, ks, vs, os_, lses, dos, causal=causal, layout=layout)
+        def step(timed=False):
+            tf, tb = (RankStepTimer(R), RankStepTimer(R)) if timed else (None, None)
+            os_, lses = ring.local_ring_forward(qs, ks, vs, causal=causal, layout=layout, timer=tf)
+            ring.local_ring_backward(qs, ks, vs, os_, lses, dos, causal=causal, layout=layout, timer=tb)
+            if timed:
+                timers.append((tf, tb))
     del x
     for _ in range(args.warmup):
         step()
@@ -1044,6 +1048,15 @@ def run_ring(args, world, rank, local):
     if fa.fa_get_device_status(None) != 0:
         raise RuntimeError("device status reports a timed-out wait")
     t_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
+    crit = None
+    if world == 1:
+        # a second set of steps with events around every emulated rank's work
+        # at every ring step (kept apart, so the run above times the plain calls)
+        for _ in range(args.steps):
+            flush()
+            step(timed=True)
+        torch.cuda.synchronize()
+        crit = sum(tf.critical_path_ms() + tb.critical_path_ms() for tf, tb in timers) / args.steps
     F = fwd_flops(w)
     if rank == 0:
         line = {"ring": w["name"], "ranks": R, "layout": layout, "emulated_on_one_gpu": world == 1,
@@ -1051,7 +1064,33 @@ def run_ring(args, world, rank, local):
                 "ms_per_step": round(t_ms / args.steps, 4),
                 "fwd_bwd_tflops": round(3.5 * F * args.steps / (t_ms * 1e-3) / 1e12, 2),
                 "slice_rows": n}
+        if crit is not None:
+            line["critical_path_ms"] = round(crit, 4)
+            line["critical_path_note"] = ("sum over ring steps of the slowest emulated rank's kernel time at "
+                                          "that step, forward and backward: the step time R GPUs would "
+                                          "need if every exchange hid behind the kernels (not measured on "
+                                          "R GPUs)")
         print(json.dumps(line), flush=True)
+
+
+class RankStepTimer:
+    """CUDA events around each emulated rank's work at each ring step."""
+
+    def __init__(self, R):
+        import torch
+        self.R = R
+        self.ev = {(t, r): (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for t in range(R) for r in range(R)}
+
+    def start(self, t, r):
+        self.ev[(t, r)][0].record()
+
+    def stop(self, t, r):
+        self.ev[(t, r)][1].record()
+
+    def critical_path_ms(self):
+        return sum(max(a.elapsed_time(b) for a, b in (self.ev[(t, r)] for r in range(self.R)))
+                   for t in range(self.R))
 
 
 def run_ours(args, world, rank, local):

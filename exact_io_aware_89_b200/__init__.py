@@ -106,10 +106,10 @@ def load_library():
     lib.fa_test_withhold_next_load.argtypes = []
     lib.fa_test_withhold_next_load.restype = i
     for name in ("fa_lse_merge", "fa_lse_merge_f16"):
-        getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+        getattr(lib, name).argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
         getattr(lib, name).restype = i
     for name in ("fa_grad_accumulate", "fa_grad_accumulate_f16"):
-        getattr(lib, name).argtypes = [vp, vp, vp, ll, i, vp]
+        getattr(lib, name).argtypes = [vp, vp, vp, i, i, i, i, ll, i, vp]
         getattr(lib, name).restype = i
     for name in ("fa_fwd", "fa_bwd", "fa_bwd_noalloc", "fa_fwd_f32", "fa_bwd_f32", "fa_fwd_splitkv", "fa_fwd_kvcache", "fa_fwd_varlen", "fa_bwd_varlen",
                  "fa_get_device_status",
@@ -244,18 +244,22 @@ def fa_status_string(status):
     return load_library().fa_status_string(int(status)).decode()
 
 
-def fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream):
-    """Fold one partial forward result (bf16 O, fp32 LSE) into a running fp32 one."""
-    return load_library().fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream)
+def fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, Nq_acc, row0, first, stream):
+    """Fold one partial forward result (bf16 O, fp32 LSE) into rows row0 ..
+    row0 + Nq - 1 of a running fp32 one."""
+    return load_library().fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, Nq_acc, row0, first,
+                                       stream)
 
 
-def fa_lse_merge_f16(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream):
-    return load_library().fa_lse_merge_f16(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream)
+def fa_lse_merge_f16(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, Nq_acc, row0, first, stream):
+    return load_library().fa_lse_merge_f16(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, Nq_acc, row0,
+                                           first, stream)
 
 
-def fa_grad_accumulate(acc, part, out, n, first, stream):
-    """acc (fp32) = (first ? 0 : acc) + part (bf16); out (bf16) = rounded acc."""
-    return load_library().fa_grad_accumulate(acc, part, out, n, first, stream)
+def fa_grad_accumulate(acc, part, out, B, rows_acc, row0, rows, row_elems, first, stream):
+    """acc (fp32) = (first ? 0 : acc) + part (bf16) on rows row0 .. row0 + rows - 1;
+    out (bf16) = rounded acc on the same rows."""
+    return load_library().fa_grad_accumulate(acc, part, out, B, rows_acc, row0, rows, row_elems, first, stream)
 
 
 def fa_test_withhold_next_load():
@@ -264,8 +268,8 @@ def fa_test_withhold_next_load():
     return load_library().fa_test_withhold_next_load()
 
 
-def fa_grad_accumulate_f16(acc, part, out, n, first, stream):
-    return load_library().fa_grad_accumulate_f16(acc, part, out, n, first, stream)
+def fa_grad_accumulate_f16(acc, part, out, B, rows_acc, row0, rows, row_elems, first, stream):
+    return load_library().fa_grad_accumulate_f16(acc, part, out, B, rows_acc, row0, rows, row_elems, first, stream)
 
 
 KERNEL_KINDS = ("fwd", "bwd_prep", "bwd_dq", "bwd_dkdv", "f32", "decode", "kvcache_append",
@@ -563,26 +567,59 @@ def attention_backward(q, k, v, o, lse, do, scale=None, causal=False, window=(-1
     return dq, dk, dv
 
 
-def lse_merge(o_acc, lse_acc, o_part, lse_part, first=False, out=None):
-    """Fold (o_part [B, Nq, H, d] bf16/fp16, lse_part [B, H, Nq] fp32) into the
-    running fp32 result (o_acc, lse_acc), in place; with ``out`` given, also
-    write the merged O rounded to out's type.  Returns ``out``."""
+def _need(cond, what):
+    if not cond:
+        raise ValueError(what)
+
+
+def lse_merge(o_acc, lse_acc, o_part, lse_part, first=False, out=None, row0=0):
+    """Fold (o_part [B, Nq, H, d] bf16/fp16, lse_part [B, H, Nq] fp32) into
+    rows row0 .. row0 + Nq - 1 of the running fp32 result (o_acc [B, Nq_acc, H,
+    d], lse_acc [B, H, Nq_acc]), in place; with ``out`` given (o_acc's shape),
+    also write those merged rows of O rounded to out's type.  Returns ``out``."""
     import torch
     B, Nq, H, d = o_part.shape
+    Nq_acc = o_acc.shape[1]
+    _need(o_acc.shape == (B, Nq_acc, H, d) and lse_acc.shape == (B, H, Nq_acc) and lse_part.shape == (B, H, Nq)
+          and (out is None or out.shape == o_acc.shape), "lse_merge: mismatched shapes")
+    _need(0 <= row0 <= Nq_acc - Nq, "lse_merge: rows out of range")
+    _need(o_acc.dtype == torch.float32 and lse_acc.dtype == torch.float32 and lse_part.dtype == torch.float32
+          and o_part.dtype in (torch.bfloat16, torch.float16) and (out is None or out.dtype == o_part.dtype),
+          "lse_merge: dtypes")
+    _need(all(t.is_contiguous() for t in (o_acc, lse_acc, o_part, lse_part) + ((out,) if out is not None else ())),
+          "lse_merge: tensors must be contiguous")
     fn = fa_lse_merge_f16 if o_part.dtype == torch.float16 else fa_lse_merge
     _check(fn.__name__, fn(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(),
-                           out.data_ptr() if out is not None else None, B, Nq, H, d, int(bool(first)),
-                           _stream()))
+                           out.data_ptr() if out is not None else None, B, Nq, H, d, Nq_acc, int(row0),
+                           int(bool(first)), _stream()))
     return out
 
 
-def grad_accumulate(acc, part=None, first=False, out=None):
+def grad_accumulate(acc, part=None, first=False, out=None, row0=0):
     """acc (fp32) = (first ? 0 : acc) + part (bf16/fp16), in place; with ``out``
-    given, also write acc rounded to out's type.  Returns ``out``."""
+    given (acc's shape), also write acc rounded to out's type.  Returns ``out``.
+    A 1-D acc is one flat sum.  Otherwise acc is [B, rows_acc, ...] and part
+    [B, rows, ...] covers acc's rows row0 .. row0 + rows - 1 (without part, every
+    row from row0 on is converted)."""
+    import math as _m
     import torch
     ref = part if part is not None else out
+    _need(ref is not None, "grad_accumulate: part or out needed")
+    _need(acc.dtype == torch.float32 and ref.dtype in (torch.bfloat16, torch.float16)
+          and (part is None or out is None or out.dtype == part.dtype), "grad_accumulate: dtypes")
+    _need(all(t.is_contiguous() for t in (acc, part, out) if t is not None), "grad_accumulate: tensors must be contiguous")
+    _need(out is None or out.shape == acc.shape, "grad_accumulate: out must have acc's shape")
+    if acc.dim() == 1:
+        _need(row0 == 0 and (part is None or part.shape == acc.shape), "grad_accumulate: mismatched shapes")
+        B, rows_acc, rows, row_elems = 1, 1, 1, acc.numel()
+    else:
+        B, rows_acc = acc.shape[0], acc.shape[1]
+        row_elems = _m.prod(acc.shape[2:])
+        rows = part.shape[1] if part is not None else rows_acc - row0
+        _need(part is None or part.shape == (B, rows) + tuple(acc.shape[2:]), "grad_accumulate: mismatched shapes")
+        _need(0 <= row0 and 1 <= rows and row0 + rows <= rows_acc, "grad_accumulate: rows out of range")
     fn = fa_grad_accumulate_f16 if ref.dtype == torch.float16 else fa_grad_accumulate
     _check(fn.__name__, fn(acc.data_ptr(), part.data_ptr() if part is not None else None,
-                           out.data_ptr() if out is not None else None, acc.numel(), int(bool(first)),
-                           _stream()))
+                           out.data_ptr() if out is not None else None, B, rows_acc, int(row0), rows, row_elems,
+                           int(bool(first)), _stream()))
     return out

@@ -1120,31 +1120,29 @@ namespace {
 
 template <bool F16>
 int lse_merge_impl(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
-                   int Nq, int H, int d, int first, fa_stream_t stream) {
+                   int Nq, int H, int d, int Nq_acc, int row0, int first, fa_stream_t stream) {
   if (!aligned16(o_acc) || !aligned16(lse_acc) || !aligned16(o_part) || !aligned16(lse_part) ||
       (o_out != nullptr && !aligned16(o_out)))
     return FA_ERR_INVALID_ARG;
-  if (B < 1 || Nq < 1 || H < 1) return FA_ERR_INVALID_ARG;
+  if (B < 1 || Nq < 1 || H < 1 || row0 < 0 || Nq_acc < Nq || row0 > Nq_acc - Nq) return FA_ERR_INVALID_ARG;
   const long long rows = static_cast<long long>(B) * Nq * H;
-  if (rows > (1ll << 40)) return FA_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * Nq_acc * H > (1ll << 40)) return FA_ERR_INVALID_ARG;
   const long long blocks = (rows * 32 + 255) / 256;
   if (blocks > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   auto* op = static_cast<const uint16_t*>(o_part);
   auto* oo = static_cast<uint16_t*>(o_out);
   TraceScope tr(FA_KERNEL_MERGE, s);
+  const unsigned g = static_cast<unsigned>(blocks);
   switch (d) {
     case 64:
-      fa_lse_merge_kernel<64, F16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo, B,
-                                                                                Nq, H, first);
+      fa_lse_merge_kernel<64, F16><<<g, 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo, B, Nq, H, Nq_acc, row0, first);
       break;
     case 128:
-      fa_lse_merge_kernel<128, F16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo,
-                                                                                 B, Nq, H, first);
+      fa_lse_merge_kernel<128, F16><<<g, 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo, B, Nq, H, Nq_acc, row0, first);
       break;
     case 256:
-      fa_lse_merge_kernel<256, F16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo,
-                                                                                 B, Nq, H, first);
+      fa_lse_merge_kernel<256, F16><<<g, 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo, B, Nq, H, Nq_acc, row0, first);
       break;
     default:
       return FA_ERR_UNSUPPORTED;
@@ -1153,16 +1151,20 @@ int lse_merge_impl(float* o_acc, float* lse_acc, const void* o_part, const float
 }
 
 template <bool F16>
-int grad_accumulate_impl(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream) {
+int grad_accumulate_impl(float* acc, const void* part, void* out, int B, int rows_acc, int row0, int rows,
+                         long long row_elems, int first, fa_stream_t stream) {
   if (!aligned16(acc) || (part != nullptr && !aligned16(part)) || (out != nullptr && !aligned16(out)))
     return FA_ERR_INVALID_ARG;
-  if (n < 8 || n % 8 != 0 || (part == nullptr && out == nullptr)) return FA_ERR_INVALID_ARG;
-  const long long blocks = (n / 8 + 255) / 256;
+  if (part == nullptr && out == nullptr) return FA_ERR_INVALID_ARG;
+  if (B < 1 || B > 65535 || rows < 1 || row0 < 0 || rows_acc < rows || row0 > rows_acc - rows)
+    return FA_ERR_INVALID_ARG;
+  if (row_elems < 8 || row_elems % 8 != 0 || row_elems > (1ll << 40) / rows_acc) return FA_ERR_INVALID_ARG;
+  const long long blocks = (static_cast<long long>(rows) * row_elems / 8 + 255) / 256;
   if (blocks > (1ll << 31) - 1) return FA_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   TraceScope tr(FA_KERNEL_MERGE, s);
-  fa_grad_accumulate_kernel<F16><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-      acc, static_cast<const uint16_t*>(part), static_cast<uint16_t*>(out), n, first);
+  fa_grad_accumulate_kernel<F16><<<dim3(static_cast<unsigned>(blocks), static_cast<unsigned>(B)), 256, 0, s>>>(
+      acc, static_cast<const uint16_t*>(part), static_cast<uint16_t*>(out), rows_acc, row0, rows, row_elems, first);
   return launch_status();
 }
 
@@ -1171,18 +1173,20 @@ int grad_accumulate_impl(float* acc, const void* part, void* out, long long n, i
 extern "C" {
 
 int fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
-                 int Nq, int H, int d, int first, fa_stream_t stream) {
-  return lse_merge_impl<false>(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream);
+                 int Nq, int H, int d, int Nq_acc, int row0, int first, fa_stream_t stream) {
+  return lse_merge_impl<false>(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, Nq_acc, row0, first, stream);
 }
 int fa_lse_merge_f16(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
-                     int Nq, int H, int d, int first, fa_stream_t stream) {
-  return lse_merge_impl<true>(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, first, stream);
+                     int Nq, int H, int d, int Nq_acc, int row0, int first, fa_stream_t stream) {
+  return lse_merge_impl<true>(o_acc, lse_acc, o_part, lse_part, o_out, B, Nq, H, d, Nq_acc, row0, first, stream);
 }
-int fa_grad_accumulate(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream) {
-  return grad_accumulate_impl<false>(acc, part, out, n, first, stream);
+int fa_grad_accumulate(float* acc, const void* part, void* out, int B, int rows_acc, int row0, int rows,
+                       long long row_elems, int first, fa_stream_t stream) {
+  return grad_accumulate_impl<false>(acc, part, out, B, rows_acc, row0, rows, row_elems, first, stream);
 }
-int fa_grad_accumulate_f16(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream) {
-  return grad_accumulate_impl<true>(acc, part, out, n, first, stream);
+int fa_grad_accumulate_f16(float* acc, const void* part, void* out, int B, int rows_acc, int row0, int rows,
+                           long long row_elems, int first, fa_stream_t stream) {
+  return grad_accumulate_impl<true>(acc, part, out, B, rows_acc, row0, rows, row_elems, first, stream);
 }
 
 int fa_test_withhold_next_load(void) {

@@ -18,16 +18,19 @@
 
 namespace fa {
 
-// One warp per (b, i, h) row of O [B, Nq, H, D] and LSE [B, H, Nq]:
+// One warp per (b, i, h) row of the part, O [B, Nq, H, D] and LSE [B, H, Nq],
+// folded into row row0 + i of the accumulator, O [B, Nq_acc, H, D] and LSE
+// [B, H, Nq_acc] (so a part may cover some of the accumulator's rows):
 //   first: acc = part; otherwise acc = merge(acc, part) as above.
 // Rows where both are empty (lse = -inf) stay O = 0, lse = -inf.  With o_out
-// given, the merged row is also written rounded to the element type.
+// given ([B, Nq_acc, H, D]), the merged row is also written rounded to the
+// element type.
 template <int D, bool F16>
 __global__ void __launch_bounds__(256) fa_lse_merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc,
                                                            const uint16_t* __restrict__ o_part,
                                                            const float* __restrict__ lse_part,
                                                            uint16_t* __restrict__ o_out, int B, int Nq, int H,
-                                                           int first) {
+                                                           int Nq_acc, int row0, int first) {
   constexpr int E = D / 32;  // elements per lane: 2, 4 or 8
   const long long row = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
@@ -36,8 +39,9 @@ __global__ void __launch_bounds__(256) fa_lse_merge_kernel(float* __restrict__ o
   const long long bi = row / H;
   const int i = static_cast<int>(bi % Nq);
   const int b = static_cast<int>(bi / Nq);
-  const long long li = (static_cast<long long>(b) * H + h) * Nq + i;
-  const float lp = lse_part[li];
+  const long long lp_i = (static_cast<long long>(b) * H + h) * Nq + i;
+  const long long li = (static_cast<long long>(b) * H + h) * Nq_acc + row0 + i;
+  const float lp = lse_part[lp_i];
   const float la = first ? -INFINITY : lse_acc[li];
   const float m = fmaxf(la, lp);
   float wa = 0.f, wp = 0.f, lnew = -INFINITY;
@@ -49,11 +53,12 @@ __global__ void __launch_bounds__(256) fa_lse_merge_kernel(float* __restrict__ o
     wa = ea / s;
     wp = ep / s;
   }
-  const long long off = row * D + lane * E;
+  const long long poff = row * D + lane * E;
+  const long long off = ((static_cast<long long>(b) * Nq_acc + row0 + i) * H + h) * D + lane * E;
   float acc[E], part[E];
 #pragma unroll
   for (int e = 0; e < E; e += 2) {
-    const uint32_t w = *reinterpret_cast<const uint32_t*>(o_part + off + e);
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(o_part + poff + e);
     part[e] = h16_to_f32<F16>(w & 0xFFFFu);
     part[e + 1] = h16_to_f32<F16>(w >> 16);
   }
@@ -80,15 +85,21 @@ __global__ void __launch_bounds__(256) fa_lse_merge_kernel(float* __restrict__ o
   if (lane == 0) lse_acc[li] = lnew;
 }
 
-// n elements, 8 per thread (n % 8 == 0, 16-byte aligned buffers):
-//   part given: acc = (first ? 0 : acc) + part;  out given: out = round(acc).
+// Rows of row_elems elements: part [B, rows, row_elems] added to rows
+// [row0, row0 + rows) of acc [B, rows_acc, row_elems] (fp32), 8 elements per
+// thread (row_elems % 8 == 0, 16-byte aligned buffers), blockIdx.y = b:
+//   part given: acc = (first ? 0 : acc) + part;  out given ([B, rows_acc,
+//   row_elems]): out = round(acc) on the same rows.
 template <bool F16>
 __global__ void __launch_bounds__(256) fa_grad_accumulate_kernel(float* __restrict__ acc,
                                                                  const uint16_t* __restrict__ part,
-                                                                 uint16_t* __restrict__ out, long long n,
-                                                                 int first) {
-  const long long x = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) * 8;
-  if (x >= n) return;
+                                                                 uint16_t* __restrict__ out, int rows_acc, int row0,
+                                                                 int rows, long long row_elems, int first) {
+  const long long n = static_cast<long long>(rows) * row_elems;
+  const long long xp = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) * 8;
+  if (xp >= n) return;
+  const long long b = blockIdx.y;
+  const long long x = (b * rows_acc + row0) * row_elems + xp;
   float a[8];
   if (first && part != nullptr) {
 #pragma unroll
@@ -100,7 +111,7 @@ __global__ void __launch_bounds__(256) fa_grad_accumulate_kernel(float* __restri
     a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
   }
   if (part != nullptr) {
-    const uint4 p = *reinterpret_cast<const uint4*>(part + x);
+    const uint4 p = *reinterpret_cast<const uint4*>(part + b * n + xp);
     const uint32_t w[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {

@@ -337,31 +337,44 @@ int fa_bwd_f32(const float* q, const float* k, const float* v, const float* o, c
  * blockwise correctly", applied to whole key sets): with lse_s the natural
  * log-sum-exp and O_s the normalised output of set s,
  *     lse = ln sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.
- *   o_acc  [B, Nq, H, d] fp32, lse_acc [B, H, Nq] fp32 : the running result,
- *            updated in place; with first != 0 they are overwritten by the part
- *            (their contents are ignored)
+ *   o_acc  [B, Nq_acc, H, d] fp32, lse_acc [B, H, Nq_acc] fp32 : the running
+ *            result, updated in place on rows [row0, row0 + Nq); with
+ *            first != 0 those rows are overwritten by the part (their
+ *            contents are ignored)
  *   o_part [B, Nq, H, d] bf16 (_f16: fp16), lse_part [B, H, Nq] fp32 : the
- *            result over the next key set, as fa_fwd wrote it
- *   o_out  [B, Nq, H, d] bf16 / fp16, or NULL: the merged O, rounded
- *   d in {64, 128, 256}.  Rows empty in both (lse = -inf) stay O = 0,
- *   lse = -inf.  Merging parts in a fixed order gives the same bits every time.
+ *            result of rows row0 .. row0 + Nq - 1 over the next key set, as
+ *            fa_fwd wrote it
+ *   o_out  [B, Nq_acc, H, d] bf16 / fp16, or NULL: the merged O of rows
+ *            [row0, row0 + Nq), rounded (other rows untouched)
+ *   d in {64, 128, 256}; 0 <= row0, row0 + Nq <= Nq_acc (Nq_acc = Nq,
+ *   row0 = 0 when the part covers every row).  Rows empty in both
+ *   (lse = -inf) stay O = 0, lse = -inf.  Merging parts in a fixed order
+ *   gives the same bits every time.
  *
  * fa_grad_accumulate sums backward shares in fp32: the gradients fa_bwd
  * computes for one key set, given the full rows' o and lse, are that set's
- * share of dq and its keys' dk / dv.
- *   acc  [n] fp32 : running sum, updated in place (first != 0: acc = part)
- *   part [n] bf16 / fp16, or NULL (only convert)
- *   out  [n] bf16 / fp16, or NULL: the sum, rounded
- *   n a multiple of 8; at least one of part, out given.
+ * share of dq and its keys' dk / dv.  Tensors are B batches of rows of
+ * row_elems elements (a row: all heads of one sequence position, H * d);
+ * the part covers rows [row0, row0 + rows) of the accumulator.
+ *   acc  [B, rows_acc, row_elems] fp32 : running sum, updated in place on
+ *          rows [row0, row0 + rows) (first != 0: those rows = part)
+ *   part [B, rows, row_elems] bf16 / fp16, or NULL (only convert)
+ *   out  [B, rows_acc, row_elems] bf16 / fp16, or NULL: the sum, rounded,
+ *          written on the same rows
+ *   1 <= B <= 65535, 0 <= row0, row0 + rows <= rows_acc, row_elems a
+ *   multiple of 8; at least one of part, out given.  A flat sum of n
+ *   elements is B = rows_acc = rows = 1, row0 = 0, row_elems = n.
  * Both return FA_OK or FA_ERR_INVALID_ARG / FA_ERR_UNSUPPORTED / FA_ERR_CUDA;
  * pointers are device pointers aligned to 16 bytes; stream-ordered.
  */
 int fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
-                 int Nq, int H, int d, int first, fa_stream_t stream);
+                 int Nq, int H, int d, int Nq_acc, int row0, int first, fa_stream_t stream);
 int fa_lse_merge_f16(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, void* o_out, int B,
-                     int Nq, int H, int d, int first, fa_stream_t stream);
-int fa_grad_accumulate(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream);
-int fa_grad_accumulate_f16(float* acc, const void* part, void* out, long long n, int first, fa_stream_t stream);
+                     int Nq, int H, int d, int Nq_acc, int row0, int first, fa_stream_t stream);
+int fa_grad_accumulate(float* acc, const void* part, void* out, int B, int rows_acc, int row0, int rows,
+                       long long row_elems, int first, fa_stream_t stream);
+int fa_grad_accumulate_f16(float* acc, const void* part, void* out, int B, int rows_acc, int row0, int rows,
+                           long long row_elems, int first, fa_stream_t stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word of

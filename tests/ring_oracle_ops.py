@@ -28,15 +28,17 @@ class OracleOps:
     def new_out(self, q):
         return torch.zeros(q.shape, dtype=torch.float64)
 
-    def merge(self, o_acc, lse_acc, o_part, lse_part, first, out):
+    def merge(self, o_acc, lse_acc, o_part, lse_part, first, out, row0):
+        rows = slice(row0, row0 + o_part.shape[1])
         if first:
             o, lse = _np(o_part), _np(lse_part)
         else:
-            o, lse = oracle.merge_partials([_np(o_acc), _np(o_part)], [_np(lse_acc), _np(lse_part)])
-        o_acc.copy_(_t(o))
-        lse_acc.copy_(_t(lse))
+            o, lse = oracle.merge_partials([_np(o_acc[:, rows]), _np(o_part)],
+                                           [_np(lse_acc[:, :, rows]), _np(lse_part)])
+        o_acc[:, rows] = _t(o)
+        lse_acc[:, :, rows] = _t(lse)
         if out is not None:
-            out.copy_(o_acc)
+            out[:, rows] = o_acc[:, rows]
 
     def bwd(self, q, k, v, o, lse, do, scale, causal):
         return tuple(_t(x) for x in oracle.attn_bwd_given_stats(_np(q), _np(k), _np(v), _np(do), _np(o),
@@ -45,11 +47,12 @@ class OracleOps:
     def new_grad_acc(self, x):
         return torch.zeros(x.shape, dtype=torch.float64)
 
-    def accumulate(self, acc, part, first):
+    def accumulate(self, acc, part, first, row0):
+        rows = slice(row0, row0 + part.shape[1])
         if first:
-            acc.copy_(part)
+            acc[:, rows] = part
         else:
-            acc.add_(part)
+            acc[:, rows] += part
 
     def finish_grad(self, acc, like):
         return acc.clone()

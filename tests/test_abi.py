@@ -278,19 +278,29 @@ def test_blocksparse_rejects_invalid_arguments():
 
 
 def test_ring_combining_calls_reject_invalid_arguments_before_launching():
-    ok = dict(o_acc=FAKE, lse_acc=FAKE, o_part=FAKE, lse_part=FAKE, o_out=None, B=1, Nq=8, H=2, d=64, first=1)
+    ok = dict(o_acc=FAKE, lse_acc=FAKE, o_part=FAKE, lse_part=FAKE, o_out=None, B=1, Nq=8, H=2, d=64, Nq_acc=8,
+              row0=0, first=1)
 
     def merge(**kw):
         a = dict(ok, **kw)
         return fa.fa_lse_merge(a["o_acc"], a["lse_acc"], a["o_part"], a["lse_part"], a["o_out"], a["B"],
-                               a["Nq"], a["H"], a["d"], a["first"], None)
-    for kw in (dict(o_acc=0), dict(lse_part=FAKE + 4), dict(o_out=FAKE + 8), dict(B=0), dict(Nq=0), dict(H=-1)):
+                               a["Nq"], a["H"], a["d"], a["Nq_acc"], a["row0"], a["first"], None)
+    for kw in (dict(o_acc=0), dict(lse_part=FAKE + 4), dict(o_out=FAKE + 8), dict(B=0), dict(Nq=0), dict(H=-1),
+               dict(Nq_acc=7), dict(row0=-1), dict(Nq_acc=16, row0=9)):
         assert merge(**kw) == INVALID, kw
     assert merge(d=96) == UNSUPPORTED
-    assert fa.fa_lse_merge_f16(FAKE, FAKE, FAKE, FAKE, None, 1, 8, 2, 100, 0, None) == UNSUPPORTED
-    acc = fa.fa_grad_accumulate
-    assert acc(FAKE, FAKE, None, 12, 0, None) == INVALID        # n not a multiple of 8
-    assert acc(FAKE, FAKE, None, 0, 0, None) == INVALID
-    assert acc(FAKE, None, None, 16, 0, None) == INVALID         # nothing to do
-    assert acc(FAKE + 4, FAKE, None, 16, 0, None) == INVALID     # misaligned
-    assert fa.fa_grad_accumulate_f16(0, FAKE, None, 16, 0, None) == INVALID
+    assert merge(d=96, Nq_acc=16, row0=8) == UNSUPPORTED         # rows in range, head size not
+    assert fa.fa_lse_merge_f16(FAKE, FAKE, FAKE, FAKE, None, 1, 8, 2, 100, 8, 0, 0, None) == UNSUPPORTED
+    okg = dict(acc=FAKE, part=FAKE, out=None, B=1, rows_acc=1, row0=0, rows=1, row_elems=16, first=0)
+
+    def acc(**kw):
+        a = dict(okg, **kw)
+        return fa.fa_grad_accumulate(a["acc"], a["part"], a["out"], a["B"], a["rows_acc"], a["row0"], a["rows"],
+                                     a["row_elems"], a["first"], None)
+    for kw in (dict(row_elems=12),                 # not a multiple of 8
+               dict(row_elems=0), dict(part=None),  # nothing to do
+               dict(acc=FAKE + 4),                  # misaligned
+               dict(B=0), dict(B=65536), dict(rows=0), dict(rows_acc=2, rows=3),
+               dict(rows_acc=4, row0=2, rows=3), dict(row0=-1)):
+        assert acc(**kw) == INVALID, kw
+    assert fa.fa_grad_accumulate_f16(0, FAKE, None, 1, 1, 0, 1, 16, 0, None) == INVALID

@@ -1,7 +1,8 @@
 """Ring (context-parallel) attention on the GPU, against the fp64 oracle.
 
 * fa_lse_merge folding partial results in order equals oracle.merge_partials
-  on the same (bf16-rounded) partials; fa_grad_accumulate equals the fp64 sum.
+  on the same (bf16-rounded) partials; fa_grad_accumulate equals the fp64 sum;
+  a part covering some rows of the accumulator changes only those rows.
 * The ring of R ranks, emulated on one GPU (each rank's slices in its own
   buffers, the exchange a device copy), run through the library's kernels
   (fa_fwd / fa_bwd per slice pair, the merge and accumulate kernels), equals
@@ -73,15 +74,62 @@ def test_grad_accumulate_sums_in_fp32_and_rounds_once():
     assert (np.abs(out.float().cpu().numpy() - ref) <= half_ulp(ref) + 1e-5).all()
 
 
+def test_merge_and_accumulate_reach_only_the_given_rows():
+    """A part covering rows [row0, row0 + n) of a larger accumulator (B > 1,
+    so those rows are not one contiguous range): those rows merge / add as
+    the oracle says, every other row keeps its bits."""
+    dev = torch.device("cuda")
+    g = torch.Generator().manual_seed(11)
+    B, Nacc, row0, Nq, H, d = 2, 96, 32, 48, 3, 128
+    rows = slice(row0, row0 + Nq)
+    o_acc0 = torch.randn((B, Nacc, H, d), generator=g)
+    lse_acc0 = torch.randn((B, H, Nacc), generator=g)
+    o_part = torch.randn((B, Nq, H, d), generator=g).to(torch.bfloat16)
+    lse_part = torch.randn((B, H, Nq), generator=g)
+    o_acc, lse_acc = o_acc0.to(dev), lse_acc0.to(dev)
+    out = torch.full((B, Nacc, H, d), 7.0, dtype=torch.bfloat16, device=dev)
+    fa.lse_merge(o_acc, lse_acc, o_part.to(dev), lse_part.to(dev), first=False, out=out, row0=row0)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.merge_partials([o_acc0[:, rows].double().numpy(), o_part.double().numpy()],
+                                           [lse_acc0[:, :, rows].double().numpy(), lse_part.double().numpy()])
+    o_acc, lse_acc, out = o_acc.cpu(), lse_acc.cpu(), out.cpu()
+    assert np.abs(o_acc[:, rows].numpy() - o_ref).max() <= 1e-5
+    compare_lse(lse_acc[:, :, rows].numpy(), lse_ref, 1e-5, "merge rows")
+    assert o_error(out[:, rows].float().numpy(), o_ref) <= 1e-5
+    keep = torch.ones(Nacc, dtype=torch.bool)
+    keep[rows] = False
+    assert torch.equal(o_acc[:, keep], o_acc0[:, keep]) and torch.equal(lse_acc[:, :, keep], lse_acc0[:, :, keep])
+    assert (out[:, keep].float() == 7.0).all()
+
+    acc0 = torch.randn((B, Nacc, H, d), generator=g)
+    part = torch.randn((B, Nq, H, d), generator=g).to(torch.bfloat16)
+    for first in (False, True):
+        acc = acc0.to(dev)
+        fa.grad_accumulate(acc, part.to(dev), first=first, row0=row0)
+        torch.cuda.synchronize()
+        acc = acc.cpu()
+        want = part.float() if first else acc0[:, rows] + part.float()  # one fp32 rounding, as on the GPU
+        assert torch.equal(acc[:, rows], want)
+        assert torch.equal(acc[:, keep], acc0[:, keep])
+    out = torch.full((B, Nacc, H, d), 7.0, dtype=torch.bfloat16, device=dev)
+    fa.grad_accumulate(acc0.to(dev), None, out=out, row0=row0)
+    torch.cuda.synchronize()
+    out = out.cpu()
+    assert torch.equal(out[:, row0:], acc0[:, row0:].to(torch.bfloat16))
+    assert (out[:, :row0].float() == 7.0).all()
+
+
 CASES = [
-    # (R, B, n per rank, Hq, Hkv, d, causal, layout)
-    (2, 1, 256, 2, 2, 128, True, "contiguous"),
-    (4, 1, 192, 4, 2, 128, True, "contiguous"),
-    (3, 2, 128, 2, 1, 64, False, "contiguous"),
-    (4, 1, 160, 2, 2, 64, True, "contiguous"),
-    (2, 1, 256, 2, 2, 128, True, "zigzag"),
-    (4, 2, 192, 4, 2, 128, True, "zigzag"),
-    (3, 1, 128, 2, 2, 64, True, "zigzag"),
+    # (R, B, n per rank, Hq, Hkv, d, causal, layout, dtype)
+    (2, 1, 256, 2, 2, 128, True, "contiguous", "bf16"),
+    (4, 1, 192, 4, 2, 128, True, "contiguous", "bf16"),
+    (3, 2, 128, 2, 1, 64, False, "contiguous", "bf16"),
+    (4, 1, 160, 2, 2, 64, True, "contiguous", "bf16"),
+    (2, 1, 256, 2, 2, 128, True, "zigzag", "bf16"),
+    (4, 2, 192, 4, 2, 128, True, "zigzag", "bf16"),
+    (3, 1, 128, 2, 2, 64, True, "zigzag", "bf16"),
+    (3, 2, 256, 2, 1, 128, False, "zigzag", "bf16"),
+    (2, 1, 256, 2, 2, 64, True, "zigzag", "fp16"),
 ]
 
 
@@ -113,10 +161,10 @@ def _run_ring(R, qs, ks, vs, dos, scale, causal, layout):
             _whole(dk, R, layout), _whole(dv, R, layout))
 
 
-@pytest.mark.parametrize("R,B,n,Hq,Hkv,d,causal,layout", CASES)
-def test_emulated_ring_equals_attention_over_the_whole_sequence(R, B, n, Hq, Hkv, d, causal, layout):
+@pytest.mark.parametrize("R,B,n,Hq,Hkv,d,causal,layout,dtype", CASES)
+def test_emulated_ring_equals_attention_over_the_whole_sequence(R, B, n, Hq, Hkv, d, causal, layout, dtype):
     N = R * n
-    inp = make_inputs(B, N, N, Hq, Hkv, d, 5000 + R * 10 + d)
+    inp = make_inputs(B, N, N, Hq, Hkv, d, 5000 + R * 10 + d, dtype=dtype)
     scale = 1.0 / math.sqrt(d)
     dev = torch.device("cuda")
     x = {k_: t.to(dev) for k_, t in inp.items()}
@@ -124,8 +172,8 @@ def test_emulated_ring_equals_attention_over_the_whole_sequence(R, B, n, Hq, Hkv
     o, lse, dq, dk, dv = _run_ring(R, qs, ks, vs, dos, scale, causal, layout)
     f64 = {k_: t.double().numpy() for k_, t in inp.items()}
     o_ref, lse_ref = oracle.attn_fwd(f64["q"], f64["k"], f64["v"], scale=scale, causal=causal)
-    what = "ring %s R%d B%d N%d Hq%d Hkv%d d%d causal%d" % (layout, R, B, N, Hq, Hkv, d, causal)
-    err = o_error(o.float().cpu().numpy(), o_ref)
+    what = "ring %s R%d B%d N%d Hq%d Hkv%d d%d causal%d %s" % (layout, R, B, N, Hq, Hkv, d, causal, dtype)
+    err = o_error(o.float().cpu().numpy(), o_ref, dtype)
     assert err <= TOL_BF16["o"], "%s: O err %.3e" % (what, err)
     compare_lse(lse.cpu().numpy(), lse_ref, TOL_BF16["lse"], what)
     refs = oracle.attn_bwd(f64["q"], f64["k"], f64["v"], f64["do"], scale=scale, causal=causal)

@@ -100,13 +100,41 @@ def test_zigzag_gives_every_rank_the_same_causal_work_at_every_step(R):
     def work(layout):
         w = np.zeros((R, R))
         for r in range(R):
-            for t, i, j, mode in ring._schedule(r, R, layout, True):
-                w[r, t] += 1 if mode == "causal" else 2
+            for t in range(R):
+                for mode in ring._chunk_pairs(r, R, t, layout, True).values():
+                    w[r, t] += 1 if mode == "causal" else 2
         return w
     z = work("zigzag")
     assert (z == z[0, 0]).all() and z[0, 0] == 4
     c = work("contiguous").sum(axis=1)
     assert c[0] == 1 and c[R - 1] == 2 * R - 1
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("R", [1, 2, 3, 4, 8])
+def test_each_step_is_one_call_covering_exactly_the_visible_pairs(R, causal, layout):
+    """Brute force over the rows of a small split: the calls of a step, each a
+    rectangle of the rank's rows (causal within it or not), see exactly the
+    (query, key) pairs of the whole sequence that are visible, each once."""
+    c = 3
+    for r in range(R):
+        sched = ring._schedule(r, R, layout, causal)
+        for t in range(R):
+            calls = [x[1:] for x in sched if x[0] == t]
+            s = (r - t) % R
+            assert len(calls) == (0 if causal and layout == "contiguous" and s > r else 1)
+            qpos = [i * c + a for i in ring.rank_chunks(r, R, layout) for a in range(c)]
+            kpos = [j * c + b for j in ring.rank_chunks(s, R, layout) for b in range(c)]
+            seen = np.zeros((len(qpos), len(kpos)), dtype=int)
+            for (i0, i1), (j0, j1), cz in calls:
+                for a in range(i0 * c, i1 * c):
+                    for b in range(j0 * c, j1 * c):
+                        # causal calls are square: bottom-right = top-left
+                        if not cz or b - j0 * c <= a - i0 * c:
+                            seen[a, b] += 1
+            want = np.array([[_visible(qp, kp, causal) for kp in kpos] for qp in qpos], dtype=int)
+            assert (seen == want).all(), (r, t)
 
 
 def _free_port():
