@@ -83,7 +83,8 @@ using Dq128 = Dq2Cfg<128, 3, 2>;
 using Dq256 = DqCfg<256, 1, 64, 1>;
 // dK/dV: {d, accumulated d slice, query tile, Q/dO ring depth}
 using Dkv64 = DkvCfg<64, 64, 64, 4>;
-using Dkv128 = DkvCfg<128, 128, 64, 4>;
+// d = 128: 128-query steps {d, Q/dO ring depth, exp2 pairs of 8 on the FMA pipe}
+using Dkv128 = DkvWCfg<128, 2, 2>;
 using Dkv256 = DkvCfg<256, 128, 64, 1>;
 
 // split-KV decode: {d, key tile, K/V ring depth, TMEM lanes per copy of the packed rows}
@@ -347,6 +348,14 @@ struct BlockMask {
   long long sb = 0, sh = 0;
 };
 
+template <class CKV, bool VL, bool BS>
+constexpr auto dkdv_kernel() {
+  if constexpr (CKV::WIDE)
+    return fa_bwd_dkdv_wide_kernel<CKV, VL, BS>;
+  else
+    return fa_bwd_dkdv_kernel<CKV, VL, BS>;
+}
+
 template <class CQ, class CKV, bool VL = false, bool BS = false>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                const void* dO, void* dq, void* dk, void* dv, int B, int Nq, int Nk, int Hq, int Hkv,
@@ -448,7 +457,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
         !encode_bnhd(&tv, v, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)) || !encode_bnhd(&tdo, dO, mB, mNq, Hq, D, CKV::BM, tma_type(CKV::F16)) ||
         !encode_bnhd(&tdk, dk, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)) || !encode_bnhd(&tdv, dv, mB, mNk, Hkv, D, CKV::BN, tma_type(CKV::F16)))
       return FA_ERR_CUDA;
-    auto kern = fa_bwd_dkdv_kernel<CKV, VL, BS>;
+    auto kern = dkdv_kernel<CKV, VL, BS>();
     if (smem_attr_once(kern, BS ? 232448 : CKV::SMEM_BYTES, attr_kv) != cudaSuccess) return FA_ERR_CUDA;
     const dim3 grid(static_cast<unsigned>(static_cast<long long>(p.n_kvtiles) * B * Hkv), D / CKV::DV);
     {

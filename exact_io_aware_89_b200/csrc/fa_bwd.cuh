@@ -847,6 +847,7 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 template <int D_, int DV_, int BM_, int ST_>
 struct DkvCfg {
   static constexpr bool F16 = false;  // elements are bf16 (AsF16<> flips it to fp16)
+  static constexpr bool WIDE = false;
   static constexpr int D = D_, DV = DV_, BM = BM_, ST = ST_;
   static constexpr int BN = 128;
   static constexpr int LA = ST >= 2 ? 2 : 1;
@@ -1196,6 +1197,446 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       store_rows_sw128(sK, C::KCHUNK, nk - k0, DV, p.dk, sq.k_off + k0, p.total_k, p.Hkv, hk, D, dslice * DV,
                        threadIdx.x, 256);
       store_rows_sw128(sV, C::KCHUNK, nk - k0, DV, p.dv, sq.k_off + k0, p.total_k, p.Hkv, hk, D, dslice * DV,
+                       threadIdx.x, 256);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == C::MMA_WARP) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+// =====================================================================
+// 3b. dK, dV in steps of 128 query rows (d = 128)
+// =====================================================================
+// The work of fa_bwd_dkdv_kernel in steps of 128 query rows instead of 64.
+// S^T and dP^T then are N = 128 MMAs, which run at the tensor core's full
+// rate (an M = 128, K = 16 MMA with N = 64 takes about 1.3 times its share of
+// the time), and a step issues half as many MMAs.  TMEM holds one step: dK
+// [0, 128), dV [128, 256), S^T [256, 384), dP^T [384, 512).  Both warpgroups
+// work on the same step, warpgroup g on query columns [64 g, 64 g + 64); each
+// writes its P^T and dS^T (bf16 pairs, 32 columns each) over the S^T and dP^T
+// columns it has read.  Per step the tensor core runs dV += P^T dO as soon as
+// every P^T is in place, the next step's S^T, dK += dS^T Q once every dS^T is
+// in place, and the next step's dP^T (the MMAs of one CTA run in issue order,
+// so S^T and dP^T overwrite the columns dV and dK read only after them); dK
+// and dP^T run while the warpgroups compute the next step's P^T.  The
+// warpgroups' exponentials are on the step's critical path: in an unmasked
+// step NPOLY of every 8 pairs are computed on the FMA pipe (exp2_poly_pair)
+// beside the MUFU unit.
+template <int D_, int ST_, int NPOLY_>
+struct DkvWCfg {
+  static constexpr bool F16 = false;  // elements are bf16 (AsF16<> flips it to fp16)
+  static constexpr bool WIDE = true;
+  static constexpr int D = D_, DV = D_, BM = 128, ST = ST_, NPOLY = NPOLY_;
+  static constexpr int BN = 128;
+  static constexpr int NCHUNK = D / 64;
+  static constexpr int KCHUNK = BN * 128;
+  static constexpr int QCHUNK = BM * 128;
+  static constexpr int KTILE = NCHUNK * KCHUNK;
+  static constexpr int QTILE = NCHUNK * QCHUNK;
+  static constexpr int STAGE = 2 * QTILE;    // Q, dO (swizzled, 1 KiB aligned)
+  static constexpr int SSTAGE = 2 * BM * 4;  // lse2, D of the same step
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KTILE;
+  static constexpr int OFF_ST = OFF_V + KTILE;
+  static constexpr int OFF_STAT = OFF_ST + ST * STAGE;
+  static constexpr int OFF_BAR = OFF_STAT + ST * SSTAGE;
+  static constexpr int NBAR = 1 + 2 * ST + 6;  // kv_full, q_full/q_empty, s_full, dp_full, p_full, ds_full, acc_done, drain
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr int NWARPS = 10;
+  static constexpr int NTHREADS = 32 * NWARPS;
+  static constexpr int TMA_WARP = 8, MMA_WARP = 9;
+  static constexpr int COL_DK = 0, COL_DV = DV, COL_S = 2 * DV, COL_DP = COL_S + BM;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(D == 128, "one step of S^T and dP^T beside dK and dV fills TMEM at d = 128");
+  static_assert(COL_DP + BM <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(STAGE % 1024 == 0, "stages stay 1 KiB aligned");
+};
+
+// P^T of 32 columns [C0, C0 + 32) of one key row: 2^(s * scale_log2 - lse2),
+// the fp32 values over s (dS^T needs them), bf16 pairs into pk[C0 / 2 ..].
+// EDGE: masked (-inf) scores or padding rows (lse2 = +inf) may be present, so
+// MUFU ex2 only (exact zeros); otherwise NPOLY of every 8 pairs use
+// exp2_poly_pair.
+template <class C, int C0, bool EDGE>
+__device__ __forceinline__ void dkdv_p32(uint32_t* sv, const float4* lse4, uint64_t sl2x2, uint32_t* pk) {
+#pragma unroll
+  for (int c = C0; c < C0 + 32; c += 4) {
+    const float4 l4 = lse4[c / 4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int cc = c + 2 * h;
+      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[cc]), __uint_as_float(sv[cc + 1])), sl2x2,
+                                 h == 0 ? f2_pack(-l4.x, -l4.y) : f2_pack(-l4.z, -l4.w));
+      float p0, p1;
+      if (!EDGE && (cc / 2) % 8 < C::NPOLY) {
+        exp2_poly_pair(x2, p0, p1);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
+      sv[cc] = __float_as_uint(p0);
+      sv[cc + 1] = __float_as_uint(p1);
+      pk[cc / 2] = pack2<C::F16>(p0, p1);
+    }
+  }
+}
+
+// dS^T = P^T (dP^T - D) of 32 columns [C0, C0 + 32), bf16 pairs into pk[C0 / 2 ..]
+template <class C, int C0>
+__device__ __forceinline__ void dkdv_ds32(const uint32_t* pv, const uint32_t* dv, const float4* d4, uint32_t* pk) {
+#pragma unroll
+  for (int c = C0; c < C0 + 32; c += 4) {
+    const float4 D4 = d4[c / 4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int cc = c + 2 * h;
+      const uint64_t t = f2_add(f2_pack(__uint_as_float(dv[cc]), __uint_as_float(dv[cc + 1])),
+                                h == 0 ? f2_pack(-D4.x, -D4.y) : f2_pack(-D4.z, -D4.w));
+      float d0, d1;
+      f2_unpack(f2_mul(f2_pack(__uint_as_float(pv[cc]), __uint_as_float(pv[cc + 1])), t), d0, d1);
+      pk[cc / 2] = pack2<C::F16>(d0, d1);
+    }
+  }
+}
+
+template <class C, bool VL = false, bool BS = false>
+__global__ void __launch_bounds__(C::NTHREADS, 1)
+    fa_bwd_dkdv_wide_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                            const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                            const BwdParams p) {
+  constexpr int D = C::D, DV = C::DV, BM = C::BM, BN = C::BN, ST = C::ST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = q_full + ST;
+  uint64_t* s_full = q_empty + ST;
+  uint64_t* dp_full = s_full + 1;
+  uint64_t* p_full = dp_full + 1;
+  uint64_t* ds_full = p_full + 1;
+  uint64_t* acc_done = ds_full + 1;
+  uint64_t* bar_drain = acc_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  const uint32_t sK = sbase + C::OFF_K, sV = sbase + C::OFF_V, sSt = sbase + C::OFF_ST;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // ---- work unit: as in fa_bwd_dkdv_kernel (one d slice: DV = D)
+  const ChunkedOrder order(blockIdx.x, p.B * p.Hkv, p.n_kvtiles, p.head_chunk_kv);
+  const int bhk = order.head;
+  const int j = order.rank;
+  const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
+  const int k0 = j * BN;
+  const SeqView sq(p.mask, VL ? p.cu_q : nullptr, p.cu_k, b);
+  const int nq = sq.mask.Nq, nk = sq.mask.Nk;
+  if (VL && k0 >= nk) return;  // this packed sequence has no key tile j
+  const int k1 = min(nk - 1, k0 + BN - 1);
+  const int delta = sq.mask.delta();
+  int q_lo = (sq.mask.wr < 0) ? 0 : k0 - delta - sq.mask.wr;
+  int q_hi = (sq.mask.wl < 0) ? nq - 1 : k1 - delta + sq.mask.wl;
+  q_lo = max(q_lo, 0);
+  q_hi = min(q_hi, nq - 1);
+  const int i_begin = q_lo / BM;
+  const int n_qt = (q_hi >= q_lo) ? (q_hi / BM - i_begin + 1) : 0;
+  int n_steps = n_qt * p.group;  // (query head in group) x (query tile)
+  uint32_t* step_list = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC + 16);
+  volatile int* list_count = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  if constexpr (BS) {
+    if (warp == C::TMA_WARP) {
+      const uint8_t* mb = p.bmask + b * p.bm_sb + k0 / 128;
+      n_steps = warp_compact(n_steps, step_list, [&](int st) {
+        const int hq = hk * p.group + st / n_qt, qb = (i_begin + st % n_qt) * BM / 128;
+        return __ldg(mb + hq * p.bm_sh + static_cast<long long>(qb) * p.bm_cols) != 0;
+      });
+      if (lane == 0) *list_count = n_steps;
+      __syncwarp();
+    }
+  }
+  auto step_of = [&](int it) {
+    if constexpr (BS)
+      return static_cast<int>(step_list[it]);
+    else
+      return it;
+  };
+  auto step_head = [&](int it) { return hk * p.group + step_of(it) / n_qt; };
+  auto step_q0 = [&](int it) { return (i_begin + step_of(it) % n_qt) * BM; };
+  auto load_step = [&](int it) {
+    const int s = it % ST;
+    const int hq = step_head(it), q0 = step_q0(it);
+    const uint32_t st = sSt + s * C::STAGE;
+    mbar_expect_tx(&q_full[s], C::STAGE + C::SSTAGE);
+    for (int c = 0; c < C::NCHUNK; ++c) {
+      tma_load_4d(st + c * C::QCHUNK, &tm_q, &q_full[s], c * 64, hq, sq.q_off + q0, sq.tb);
+      tma_load_4d(st + C::QTILE + c * C::QCHUNK, &tm_do, &q_full[s], c * 64, hq, sq.q_off + q0, sq.tb);
+    }
+    const size_t srow = (static_cast<size_t>(b) * p.Hq + hq) * p.Nq_pad + q0;
+    const uint32_t stat = sbase + C::OFF_STAT + s * C::SSTAGE;
+    bulk_load(stat, p.lse2 + srow, BM * 4, &q_full[s]);
+    bulk_load(stat + BM * 4, p.D + srow, BM * 4, &q_full[s]);
+  };
+  const int n_pre = min(n_steps, ST);
+  if (warp == C::TMA_WARP && lane == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 2 * 128);
+    mbar_init(ds_full, 2 * 128);
+    mbar_init(acc_done, 1);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    if (n_steps > 0) {
+      mbar_expect_tx(kv_full, 2 * C::KTILE);
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        tma_load_4d(sK + c * C::KCHUNK, &tm_k, kv_full, c * 64, hk, sq.k_off + k0, sq.tb);
+        tma_load_4d(sV + c * C::KCHUNK, &tm_v, kv_full, c * 64, hk, sq.k_off + k0, sq.tb);
+      }
+      for (int it = 0; it < n_pre; ++it) load_step(it);
+    }
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(smem_addr(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if constexpr (BS) n_steps = *list_count;
+
+  if (warp == C::TMA_WARP) {
+    if (lane == 0 && n_steps > 0) {
+      int n_issued = n_pre;
+      for (int it = n_pre; it < n_steps; ++it) {
+        const int s = it % ST, use = it / ST;
+        if (!mbar_wait(&q_empty[s], (use - 1) & 1, abort_flag, &g_status, p.wait_limit_ns)) break;
+        load_step(it);
+        ++n_issued;
+      }
+      mbar_drain(kv_full, 0, p.wait_limit_ns);
+      for (int s = 0; s < ST; ++s)
+        if (n_issued > s) mbar_drain(&q_full[s], ((n_issued - 1 - s) / ST) & 1, p.wait_limit_ns);
+    }
+  } else if (warp == C::MMA_WARP) {
+    if (lane == 0 && n_steps > 0) {
+      constexpr uint32_t ID_S = idesc_kind_f16<C::F16>(128, BM, false, false);
+      constexpr uint32_t ID_ACC = idesc_kind_f16<C::F16>(128, DV, false, true);
+      auto wait = [&](uint64_t* bar, uint32_t par) {
+        const bool ok = mbar_wait(bar, par, abort_flag, &g_status, p.wait_limit_ns);
+        tc_fence_after();
+        return ok;
+      };
+      const uint64_t dk_k = sdesc_sw128(sK, 16, 1024), dk_v = sdesc_sw128(sV, 16, 1024);
+      const uint64_t dk_st = sdesc_sw128(sSt, 16, 1024);             // Q / dO, K-major B
+      const uint64_t dk_stmn = sdesc_sw128(sSt, C::QCHUNK, 1024);    // Q / dO, MN-major B
+      // S^T = K Q^T and dP^T = V dO^T (M = keys, N = the step's 128 queries)
+      auto issue_s = [&](int s) {
+        const uint64_t qb = dk_st + static_cast<uint64_t>((s * C::STAGE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t kofs = ((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4;
+          const uint32_t qofs = ((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + C::COL_S, dk_k + kofs, qb + qofs, ID_S, kk > 0);
+        }
+      };
+      auto issue_dp = [&](int s) {
+        const uint64_t dob = dk_st + static_cast<uint64_t>((s * C::STAGE + C::QTILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t kofs = ((kk >> 2) * C::KCHUNK + (kk & 3) * 32) >> 4;
+          const uint32_t qofs = ((kk >> 2) * C::QCHUNK + (kk & 3) * 32) >> 4;
+          mma_ss(tmem + C::COL_DP, dk_v + kofs, dob + qofs, ID_S, kk > 0);
+        }
+      };
+      // 16-query chunk kk of P^T / dS^T: warpgroup kk / 4's columns, pair kk % 4
+      auto a_col = [](int kk) { return 64 * (kk >> 2) + 8 * (kk & 3); };
+      auto issue_dv = [&](int s, bool acc) {  // dV += P^T dO
+        const uint64_t dob = dk_stmn + static_cast<uint64_t>((s * C::STAGE + C::QTILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tmem + C::COL_DV, tmem + C::COL_S + a_col(kk), dob + static_cast<uint64_t>(kk * 128), ID_ACC,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      auto issue_dk = [&](int s, bool acc) {  // dK += dS^T Q
+        const uint64_t qb = dk_stmn + static_cast<uint64_t>((s * C::STAGE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tmem + C::COL_DK, tmem + C::COL_DP + a_col(kk), qb + static_cast<uint64_t>(kk * 128), ID_ACC,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      // Order per step: dV(it) once P^T(it) is in place, S^T(it + 1), dK(it)
+      // once dS^T(it) is, dP^T(it + 1).  S^T(it + 1) overwrites the columns
+      // dV(it) reads and dP^T(it + 1) those dK(it) reads, each after them in
+      // issue order; dK(it) and dP^T(it + 1) run while the warpgroups compute
+      // P^T(it + 1), which needs only S^T(it + 1).
+      bool ok = wait(kv_full, 0) && wait(&q_full[0], 0);
+      if (ok) {
+        issue_s(0);
+        tc_commit(s_full);
+        issue_dp(0);
+        tc_commit(dp_full);
+      }
+      for (int it = 0; it < n_steps && ok; ++it) {
+        const int s = it % ST, nx = it + 1;
+        if (!(ok = wait(p_full, it & 1))) break;
+        issue_dv(s, it > 0);
+        if (nx < n_steps) {
+          if (!(ok = wait(&q_full[nx % ST], (nx / ST) & 1))) break;
+          issue_s(nx % ST);
+          tc_commit(s_full);
+        }
+        if (!(ok = wait(ds_full, it & 1))) break;
+        issue_dk(s, it > 0);
+        tc_commit(&q_empty[s]);
+        if (nx < n_steps) {
+          issue_dp(nx % ST);
+          tc_commit(dp_full);
+        }
+      }
+      if (ok) tc_commit(acc_done);
+    }
+    if (lane == 0) {
+      tc_commit(bar_drain);
+      mbar_drain(bar_drain, 0, p.wait_limit_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ P^T / dS^T warpgroups (thread = key row)
+    const int g = warp / 4;            // query columns [64 g, 64 g + 64) of every step
+    const int r = threadIdx.x % 128;   // TMEM lane == key within the tile
+    const int key = k0 + r;
+    const int kq_lo = (sq.mask.wr < 0) ? -0x3fffffff : key - delta - sq.mask.wr;
+    const int kq_hi = (sq.mask.wl < 0) ? 0x3fffffff : key - delta + sq.mask.wl;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
+    const uint32_t col_s = C::COL_S + 64 * g, col_dp = C::COL_DP + 64 * g;
+    bool ok = true;
+    for (int it = 0; it < n_steps; ++it) {
+      const int s = it % ST;
+      ok = mbar_wait(s_full, it & 1, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      // the stage's lse2 / D landed with the barrier the MMA thread waited on
+      ok = mbar_wait(&q_full[s], (it / ST) & 1, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const float* stat = reinterpret_cast<const float*>(smem + C::OFF_STAT + s * C::SSTAGE);
+      const float4* lse4 = reinterpret_cast<const float4*>(stat + 64 * g);
+      const float4* d4 = reinterpret_cast<const float4*>(stat + BM + 64 * g);
+      const int c0 = step_q0(it) + 64 * g;  // query of column 0
+      const bool need_mask = (c0 < kq_lo) || (c0 + 63 > kq_hi);
+      // masked scores and padding rows (lse2 = +inf) must take the MUFU exp2
+      const bool edge = need_mask || (c0 + 64 > nq);
+      // S^T in two 32-column halves (the second in flight during the first's
+      // exponentials); dP^T the same way once P^T is handed over
+      uint32_t sv[64], dv[64], pk[32];
+      auto mask32 = [&](int h) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int qi = c0 + 32 * h + c;
+          if (qi < kq_lo || qi > kq_hi) sv[32 * h + c] = __float_as_uint(-INFINITY);
+        }
+      };
+      tmem_ld_x32(lane_base + col_s, sv);
+      tmem_ld_wait_x32(sv);
+      tmem_ld_x32(lane_base + col_s + 32, sv + 32);
+      if (edge) {
+        if (need_mask) mask32(0);
+        dkdv_p32<C, 0, true>(sv, lse4, sl2x2, pk);
+      } else {
+        dkdv_p32<C, 0, false>(sv, lse4, sl2x2, pk);
+      }
+      tmem_ld_wait_x32(sv + 32);
+      if (edge) {
+        if (need_mask) mask32(1);
+        dkdv_p32<C, 32, true>(sv, lse4, sl2x2, pk);
+      } else {
+        dkdv_p32<C, 32, false>(sv, lse4, sl2x2, pk);
+      }
+      tmem_st_x16(lane_base + col_s, pk);
+      tmem_st_x16(lane_base + col_s + 16, pk + 16);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      ok = mbar_wait(dp_full, it & 1, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      tmem_ld_x32(lane_base + col_dp, dv);
+      tmem_ld_wait_x32(dv);
+      tmem_ld_x32(lane_base + col_dp + 32, dv + 32);
+      dkdv_ds32<C, 0>(sv, dv, d4, pk);
+      tmem_ld_wait_x32(dv + 32);
+      dkdv_ds32<C, 32>(sv, dv, d4, pk);
+      tmem_st_x16(lane_base + col_dp, pk);
+      tmem_st_x16(lane_base + col_dp + 16, pk + 16);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    if (ok && n_steps > 0) {
+      ok = mbar_wait(acc_done, 0, abort_flag, &g_status, p.wait_limit_ns);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+    // epilogue: warpgroup 0 stages dK * scale, warpgroup 1 stages dV, as bf16 in
+    // the K and V buffers; one thread then issues the TMA stores
+    if (ok) {
+      const uint32_t col = (g == 0) ? C::COL_DK : C::COL_DV;
+      const uint32_t stage = (g == 0) ? sK : sV;
+      const float sc = (g == 0) ? p.scale : 1.f;
+#pragma unroll 1
+      for (int c = 0; c < DV / 64; ++c) {
+        uint32_t ov[64];
+        if (n_steps > 0) {
+          tmem_ld_x32(lane_base + col + c * 64, ov);
+          tmem_ld_x32(lane_base + col + c * 64 + 32, ov + 32);
+          tmem_ld_wait_x32(ov);
+          tmem_ld_wait_x32(ov + 32);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) ov[i] = 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float* f = reinterpret_cast<const float*>(ov + 8 * u);
+          st_shared_v4(stage + c * C::KCHUNK + sw128_offset(r, u), pack2<C::F16>(f[0] * sc, f[1] * sc),
+                       pack2<C::F16>(f[2] * sc, f[3] * sc), pack2<C::F16>(f[4] * sc, f[5] * sc),
+                       pack2<C::F16>(f[6] * sc, f[7] * sc));
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    named_bar_sync(1, 256);
+    if (!VL || k0 + BN <= nk) {
+      if (threadIdx.x == 0 && *abort_flag == 0) {
+        for (int c = 0; c < DV / 64; ++c) {
+          tma_store_4d(&tm_dk, sK + c * C::KCHUNK, c * 64, hk, sq.k_off + k0, sq.tb);
+          tma_store_4d(&tm_dv, sV + c * C::KCHUNK, c * 64, hk, sq.k_off + k0, sq.tb);
+        }
+        tma_store_commit();
+        tma_store_wait_read();
+      }
+    } else if (*abort_flag == 0) {  // last key tile of a packed sequence
+      store_rows_sw128(sK, C::KCHUNK, nk - k0, DV, p.dk, sq.k_off + k0, p.total_k, p.Hkv, hk, D, 0,
+                       threadIdx.x, 256);
+      store_rows_sw128(sV, C::KCHUNK, nk - k0, DV, p.dv, sq.k_off + k0, p.total_k, p.Hkv, hk, D, 0,
                        threadIdx.x, 256);
     }
   }
