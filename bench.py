@@ -414,14 +414,14 @@ SPAN_KINDS = ("bwd_call",)  # traced spans that are not kernels
 
 
 def tensor_peak(peaks, clocks):
-    """The measured bf16 peak that applies to a kernel timed in this run: the
-    burst figure when the SM clock sampled over the timed region stayed at its
-    maximum with no power cap active (the cuBLAS burst ran under the same
-    conditions), else the sustained figure, measured under the power cap.
+    """The measured bf16 peak that applies to a kernel timed in this run, by
+    the clock it ran at: the burst figure when the median SM clock sampled
+    over the timed region stayed within 5% of its maximum (the cuBLAS burst
+    ran at full clock), whether or not the power cap was reported; else the
+    sustained figure, measured with the clock pulled down by the power cap.
     Returns (TFLOP/s, label)."""
     mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
-    capped = "sw_power_cap" in (clocks.get("reasons") or [])
-    if mhz and mx and mhz >= 0.95 * mx and not capped:
+    if mhz and mx and mhz >= 0.95 * mx:
         return peaks["bf16"], "burst"
     return peaks["bf16_sustained"], "sustained"
 

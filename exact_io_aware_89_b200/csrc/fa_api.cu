@@ -81,9 +81,10 @@ using FwdBs128 = FwdCfg<128, 1, 128, 2>;
 using Dq64 = Dq2Cfg<64, 4, 3>;
 using Dq128 = Dq2Cfg<128, 3, 2>;
 using Dq256 = DqCfg<256, 1, 64, 1>;
-// dK/dV: {d, accumulated d slice, query tile, Q/dO ring depth}
-using Dkv64 = DkvCfg<64, 64, 64, 4>;
-// d = 128: 128-query steps {d, Q/dO ring depth, exp2 pairs of 8 on the FMA pipe}
+// dK/dV, d = 64 and 128: 128-query steps {d, Q/dO ring depth, exp2 pairs of 8
+// on the FMA pipe}; d = 256: 64-query steps {d, accumulated d slice, query
+// tile, Q/dO ring depth}
+using Dkv64 = DkvWCfg<64, 4, 2>;
 using Dkv128 = DkvWCfg<128, 2, 2>;
 using Dkv256 = DkvCfg<256, 128, 64, 1>;
 

@@ -1208,13 +1208,13 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 }
 
 // =====================================================================
-// 3b. dK, dV in steps of 128 query rows (d = 128)
+// 3b. dK, dV in steps of 128 query rows (d = 64, 128)
 // =====================================================================
 // The work of fa_bwd_dkdv_kernel in steps of 128 query rows instead of 64.
 // S^T and dP^T then are N = 128 MMAs, which run at the tensor core's full
 // rate (an M = 128, K = 16 MMA with N = 64 takes about 1.3 times its share of
 // the time), and a step issues half as many MMAs.  TMEM holds one step: dK
-// [0, 128), dV [128, 256), S^T [256, 384), dP^T [384, 512).  Both warpgroups
+// [0, d), dV [d, 2d), S^T [2d, 2d + 128), dP^T [2d + 128, 2d + 256).  Both warpgroups
 // work on the same step, warpgroup g on query columns [64 g, 64 g + 64); each
 // writes its P^T and dS^T (bf16 pairs, 32 columns each) over the S^T and dP^T
 // columns it has read.  Per step the tensor core runs dV += P^T dO as soon as
@@ -1251,7 +1251,7 @@ struct DkvWCfg {
   static constexpr int TMA_WARP = 8, MMA_WARP = 9;
   static constexpr int COL_DK = 0, COL_DV = DV, COL_S = 2 * DV, COL_DP = COL_S + BM;
   static constexpr int TMEM_COLS = 512;
-  static_assert(D == 128, "one step of S^T and dP^T beside dK and dV fills TMEM at d = 128");
+  static_assert(D == 64 || D == 128, "one step of S^T and dP^T beside dK and dV fits TMEM up to d = 128");
   static_assert(COL_DP + BM <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(STAGE % 1024 == 0, "stages stay 1 KiB aligned");

@@ -184,13 +184,14 @@ def test_decode_bytes_of_ragged_lengths():
     assert bench.decode_bytes(w) == expect
 
 
-def test_tensor_peak_is_burst_at_full_clock_and_sustained_under_the_power_cap():
+def test_tensor_peak_is_burst_at_full_clock_and_sustained_when_the_clock_drops():
     peaks = dict(hbm_gbs=6000.0, bf16=1662.1, bf16_sustained=1414.8, source="test")
     full = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}
     assert bench.tensor_peak(peaks, full) == (1662.1, "burst")
+    # the cap reported, the clock still at its maximum: the full-clock figure
     capped = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]}
-    assert bench.tensor_peak(peaks, capped) == (1414.8, "sustained")
-    slow = {"sm_mhz": 1400, "sm_max_mhz": 1965, "reasons": []}
+    assert bench.tensor_peak(peaks, capped) == (1662.1, "burst")
+    slow = {"sm_mhz": 1400, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"]}
     assert bench.tensor_peak(peaks, slow) == (1414.8, "sustained")
     assert bench.tensor_peak(peaks, {}) == (1414.8, "sustained")
     w = bench.WORKLOADS["wide"]
