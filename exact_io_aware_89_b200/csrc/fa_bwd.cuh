@@ -502,10 +502,14 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
 // (bf16) goes to its own TMEM columns and feeds dQ += dS K_j as the A operand.
 // K is needed first (S) and last (dQ), V only for dP, so K gets the deeper
 // ring: each tile's loads are issued two steps ahead of their use.
-template <int D_, int KS_, int VS_>
+template <int D_, int KS_, int VS_, int NPOLY_ = 0>
 struct Dq2Cfg {
   static constexpr bool F16 = false;  // elements are bf16 (AsF16<> flips it to fp16)
   static constexpr int D = D_, KS = KS_, VS = VS_;
+  // of every 8 exponential pairs of an unmasked tile, NPOLY take exp2 on the
+  // FMA pipe (exp2_poly_pair).  0 by default: here the FMA work slows the
+  // MMA issue more than the MUFU unit limits the warpgroups (timed at 0-4).
+  static constexpr int NPOLY = NPOLY_;
   static constexpr int BM = 128, BN = 128;
   static constexpr int NQT = 1;
   static constexpr bool ONE_TILE = true;
@@ -535,6 +539,33 @@ struct Dq2Cfg {
   static_assert(TMEM_USED <= 512, "TMEM budget");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
+
+// dS of 64 score columns of one query row, bf16 pairs into pk[0 .. 32):
+// P = 2^(s * scale_log2 - lse2), dS = P (dP - D), on packed fp32 pairs.  nl2 and
+// nD hold (-lse2, -lse2) and (-D, -D).  EDGE: masked (-inf) scores or a row
+// with no visible key (lse2 = +inf) may be present, so MUFU ex2 only (exact
+// zeros); otherwise NPOLY of every 8 pairs use exp2_poly_pair.
+template <class C, bool EDGE>
+__device__ __forceinline__ void dq_ds64(const uint32_t* sv, const uint32_t* dv, uint64_t sl2x2, uint64_t nl2,
+                                        uint64_t nD, uint32_t* pk) {
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sl2x2, nl2);
+    float p0, p1;
+    if (!EDGE && (c / 2) % 8 < C::NPOLY) {
+      exp2_poly_pair(x2, p0, p1);
+    } else {
+      float x0, x1;
+      f2_unpack(x2, x0, x1);
+      p0 = ex2_approx(x0);
+      p1 = ex2_approx(x1);
+    }
+    float d0, d1;
+    f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(dv[c]), __uint_as_float(dv[c + 1])), nD)), d0,
+              d1);
+    pk[c / 2] = pack2<C::F16>(d0, d1);
+  }
+}
 
 template <class C, bool VL = false, bool BS = false>
 __global__ void __launch_bounds__(C::NTHREADS, 1)
@@ -743,7 +774,10 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
     const size_t srow = (static_cast<size_t>(b) * p.Hq + h) * p.Nq_pad + row;  // row < Nq_pad
     const float lse2 = p.lse2[srow];
     const float Drow = p.D[srow];
-    const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
+    const uint64_t nl2 = f2_pack(-lse2, -lse2), nD = f2_pack(-Drow, -Drow);
+    // a row with no visible key (or a padding row) has lse2 = +inf: P = 0
+    const bool dead = lse2 == INFINITY;
     bool ok = true;
     for (int it = 0; it < n_kv; ++it) {
       ok = mbar_wait(sp_full, it & 1, abort_flag, &g_status, p.wait_limit_ns);
@@ -762,19 +796,19 @@ __global__ void __launch_bounds__(C::NTHREADS, 1)
       tc_fence_before();
       mbar_arrive(sp_free);  // S/dP may now be overwritten by the next key tile
       const int k0 = tile_of(it) * BN + wg * 64;
-      if (k0 < lo || k0 + 63 > hi) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int key = k0 + c;
-          if (key < lo || key > hi) sv[c] = __float_as_uint(-INFINITY);
-        }
-      }
+      const bool masked = k0 < lo || k0 + 63 > hi;
       uint32_t pk[32];
+      if (masked || dead) {
+        if (masked) {
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sv[c]), sl2, -lse2));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sv[c + 1]), sl2, -lse2));
-        pk[c / 2] = pack2<C::F16>(p0 * (__uint_as_float(dv[c]) - Drow), p1 * (__uint_as_float(dv[c + 1]) - Drow));
+          for (int c = 0; c < 64; ++c) {
+            const int key = k0 + c;
+            if (key < lo || key > hi) sv[c] = __float_as_uint(-INFINITY);
+          }
+        }
+        dq_ds64<C, true>(sv, dv, sl2x2, nl2, nD, pk);
+      } else {
+        dq_ds64<C, false>(sv, dv, sl2x2, nl2, nD, pk);
       }
       // the previous key tile's dQ MMA must be done reading dS
       if (it > 0) {
